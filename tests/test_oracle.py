@@ -1,0 +1,379 @@
+"""Pins of the CPU oracle to things other than itself (no GPU needed).
+
+Each test checks the oracle against what the pages or the mathematics fix: the worked padding
+example, closed forms, invariants that determine the answer uniquely, brute-force enumeration on
+tiny inputs, a second (sort-based) statement of the slot assignment, the OCP E4M3 definition
+(hand table, nearest-value search, torch's own conversion), and round-trip / exactness bounds.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def align_up(n, a):
+    return -(-n // a) * a
+
+
+def check_layout_invariants(idx, E, R, A, lay):
+    """Independent checker: these properties determine slot/psum/rows uniquely."""
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    e_loc = E // R
+    valid = [(t, j, int(idx[t, j])) for t in range(T) for j in range(k) if idx[t, j] >= 0]
+    cnt = np.zeros(E, np.int64)
+    for _, _, e in valid:
+        cnt[e] += 1
+    assert (lay.cnt == cnt).all()
+    assert lay.cnt.sum() == T * k - int((idx == -1).sum())
+    for r in range(R):
+        start = 0
+        for e in range(r * e_loc, (r + 1) * e_loc):
+            seg = [(t, j) for (t, j, ee) in valid if ee == e]     # ascending (t, j)
+            got = [int(lay.slot[t, j]) for (t, j) in seg]
+            assert got == list(range(start, start + len(seg))), (e, got, start)
+            for (t, j) in seg:
+                assert lay.row_src[r, lay.slot[t, j]] == t
+            for row in range(start + len(seg), start + align_up(len(seg), A)):
+                assert lay.row_src[r, row] == -1
+                assert lay.row_w[r, row] == 0.0
+            start += align_up(len(seg), A)
+            assert lay.psum[e] == start
+        assert lay.rows_per_rank[r] == start
+    for t in range(T):
+        for j in range(k):
+            if idx[t, j] < 0:
+                assert lay.slot[t, j] == -1
+    members = [set(int(e) // e_loc for e in idx[t] if e >= 0) for t in range(T)]
+    for r in range(R):
+        assert lay.tokens_per_rank[r] == sum(r in m for m in members)
+        assert all(lay.token_in_rank[t, r] == (r in members[t]) for t in range(T))
+
+
+# ----------------------------------------------------------------------------- layout
+
+def test_padding_worked_example():
+    g = json.load(open(os.path.join(GOLDEN, "padding_worked_example.json")))
+    A, counts = g["alignment"], g["counts"]
+    idx = np.concatenate([np.full(c, e) for e, c in enumerate(counts)]).reshape(-1, 1)
+    lay = oracle.layout(idx, None, E=len(counts), R=1, A=A)
+    assert lay.status == oracle.OK
+    assert list(lay.cnt) == counts
+    assert list(lay.psum) == [128, 256, 384]
+    assert lay.rows_per_rank[0] == g["slots_total"]
+    assert lay.cnt.sum() == g["valid_rows"]
+    assert lay.rows_per_rank[0] / lay.cnt.sum() == g["A_pad"]
+
+
+def test_alignment_one_is_plain_inclusive_scan():
+    wl = W.WORKLOADS["tiny"].with_(alignment=1)
+    idx, w = W.gen_routing(wl)
+    lay = oracle.layout(idx.numpy(), w.numpy(), wl.experts, wl.ranks, 1)
+    cnt = np.bincount(idx.numpy().ravel(), minlength=wl.experts)
+    e_loc = wl.experts_per_rank
+    expect = np.concatenate([np.cumsum(cnt[r * e_loc:(r + 1) * e_loc]) for r in range(wl.ranks)])
+    assert (lay.psum == expect).all()
+
+
+@pytest.mark.parametrize("name", ["tiny", "skewed"])
+@pytest.mark.parametrize("mask", [0.0, 0.2])
+def test_layout_invariants_workloads(name, mask):
+    wl = W.WORKLOADS[name]
+    if name == "skewed":
+        wl = wl.with_(tokens_per_rank=8)   # 128 tokens keeps the pure-Python checker quick
+    idx, w = W.gen_routing(wl)
+    if mask:
+        idx = W.mask_entries(wl, idx, mask)
+    lay = oracle.layout(idx.numpy(), w.numpy(), wl.experts, wl.ranks, wl.alignment)
+    assert lay.status == oracle.OK
+    check_layout_invariants(idx.numpy(), wl.experts, wl.ranks, wl.alignment, lay)
+    # weights travel bit-exactly into row_w
+    for t in range(wl.tokens):
+        for j in range(wl.topk):
+            e = int(idx[t, j])
+            if e >= 0:
+                assert lay.row_w[e // wl.experts_per_rank, lay.slot[t, j]] == w[t, j].item()
+
+
+@pytest.mark.parametrize("E,R,A,k", [(8, 2, 16, 2), (256, 8, 128, 8), (12, 3, 5, 4), (5, 1, 1, 3),
+                                     (64, 64, 7, 2)])
+def test_layout_equals_sort_formulation(E, R, A, k):
+    rng = np.random.default_rng(E * 1000 + A)
+    T = 300
+    idx = rng.integers(-1, E, size=(T, k)).astype(np.int64)
+    lay = oracle.layout(idx, None, E, R, A)
+    st, cnt, psum, slot = oracle.layout_by_sort(idx, E, R, A)
+    assert lay.status == st == oracle.OK
+    assert (lay.cnt == cnt).all() and (lay.psum == psum).all() and (lay.slot == slot).all()
+
+
+def test_layout_brute_force_tiny():
+    """Every routing of T tokens over E experts (with masked entries) for tiny sizes."""
+    n = 0
+    for E, R, k, T in [(2, 1, 1, 4), (2, 2, 2, 2), (4, 2, 2, 2), (4, 1, 2, 2), (3, 3, 1, 3)]:
+        choices = list(range(-1, E))
+        for A in (1, 2, 3):
+            for flat in itertools.product(choices, repeat=T * k):
+                idx = np.array(flat, np.int64).reshape(T, k)
+                lay = oracle.layout(idx, None, E, R, A)
+                st, cnt, psum, slot = oracle.layout_by_sort(idx, E, R, A)
+                assert lay.status == st == oracle.OK
+                assert (lay.slot == slot).all() and (lay.psum == psum).all()
+                check_layout_invariants(idx, E, R, A, lay)
+                n += 1
+    assert n > 1000
+
+
+def test_layout_errors():
+    idx = np.array([[0, 1], [2, 7]], np.int64)
+    assert oracle.layout(idx, None, 8, 2, 4).status == oracle.OK
+    assert oracle.layout(np.array([[0, 8]]), None, 8, 2, 4).status == oracle.ERR_BAD_EXPERT
+    assert oracle.layout(np.array([[0, -2]]), None, 8, 2, 4).status == oracle.ERR_BAD_EXPERT
+    # rank 0 needs 4 rows (A=4) but capacity 3
+    assert oracle.layout(np.array([[0, 1]]), None, 8, 2, 4, cap=3).status == oracle.ERR_CAPACITY
+    assert oracle.layout(np.array([[0, 1]]), None, 8, 2, 4, cap=8).status == oracle.OK
+
+
+# ----------------------------------------------------------------------------- E4M3
+
+def _golden_e4m3():
+    rows = []
+    for line in open(os.path.join(GOLDEN, "e4m3_edges.txt")):
+        line = line.split("#")[0].strip()
+        if line:
+            v, c = line.split()[:2]
+            rows.append((float(v), int(c, 16)))
+    return rows
+
+
+def test_e4m3_hand_table():
+    for v, c in _golden_e4m3():
+        assert oracle.e4m3_from_float(v) == c, (v, hex(c), hex(oracle.e4m3_from_float(v)))
+
+
+def test_e4m3_decode_definition():
+    assert oracle.e4m3_to_double(0x7E) == 448.0
+    assert oracle.e4m3_to_double(0x01) == 2.0 ** -9
+    assert oracle.e4m3_to_double(0x08) == 2.0 ** -6
+    assert math.isnan(oracle.e4m3_to_double(0x7F)) and math.isnan(oracle.e4m3_to_double(0xFF))
+    finite = [c for c in range(256) if c & 0x7F != 0x7F]
+    vals = [oracle.e4m3_to_double(c) for c in finite]
+    pos = sorted(v for v in vals if v > 0)
+    assert len(pos) == 126 and len(set(pos)) == 126     # 126 distinct positive finite values
+
+
+def test_e4m3_matches_nearest_value_search():
+    """Encoder == argmin |v - value(code)| over all finite codes, ties to the even code,
+    magnitudes above 448 saturated: a brute-force statement of round-to-nearest-even."""
+    codes = [c for c in range(128) if c != 0x7F]
+    table = np.array([oracle.e4m3_to_double(c) for c in codes])
+    rng = np.random.default_rng(1)
+    samples = np.concatenate([
+        rng.standard_normal(3000) * 50, rng.standard_normal(2000) * 0.01,
+        rng.uniform(-500, 500, 2000), np.array(table),                      # exact codes
+        (table[:-1] + table[1:]) / 2,                                        # exact ties
+    ]).astype(np.float32)
+    for v in samples:
+        a = abs(float(v))
+        if a >= 448.0:
+            c = 0x7E
+        else:
+            d = np.abs(table - a)
+            best = np.flatnonzero(d == d.min())
+            c = codes[best[0]] if len(best) == 1 else [codes[i] for i in best if codes[i] % 2 == 0][0]
+        if math.copysign(1.0, float(v)) < 0:
+            c |= 0x80
+        assert oracle.e4m3_from_float(float(v)) == c, (float(v), hex(c))
+
+
+def test_e4m3_matches_torch_conversion_in_range():
+    """torch's float8_e4m3fn cast (round-to-nearest-even, no saturation) agrees wherever
+    saturation does not enter."""
+    rng = np.random.default_rng(2)
+    v = np.concatenate([rng.standard_normal(20000) * 30, rng.standard_normal(5000) * 1e-3]).astype(np.float32)
+    v = v[np.abs(v) <= 448.0]
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_from_float(float(a)) for a in v], np.uint8)
+    assert (ref == got).all()
+
+
+# ----------------------------------------------------------------------------- FP8 quantisation
+
+def test_quantize_block_roundtrip_bound_and_max_code():
+    wl = W.WORKLOADS["tiny"].with_(hidden=1024)
+    x = W.gen_x(wl)[:16]
+    xb = bits(x)
+    for row in xb:
+        for b in range(0, row.size, 128):
+            blk = row[b:b + 128]
+            codes, s = oracle.quantize_block(blk)
+            xf = np.array([oracle.bf16_to_float(u) for u in blk], np.float64)
+            q = np.array([oracle.e4m3_to_double(c) for c in codes])
+            amax = np.abs(xf).max()
+            assert s == np.float32(np.float32(max(amax, 1e-4)) / np.float32(448.0))
+            err = np.abs(xf - q * s)
+            normal = np.abs(xf) / s >= 2.0 ** -6
+            assert (err[normal] <= 2.0 ** -4 * np.abs(xf[normal]) * (1 + 1e-6)).all()
+            assert (err[~normal] <= s * 2.0 ** -10 * (1 + 1e-6)).all()
+            i = int(np.argmax(np.abs(xf)))
+            assert codes[i] & 0x7F == 0x7E            # the block's largest element codes to 448
+
+
+def test_quantize_block_zero_and_floor():
+    codes, s = oracle.quantize_block(np.zeros(128, np.uint16))
+    assert (codes == 0).all() and s == np.float32(1e-4) / np.float32(448.0)
+    neg0 = np.full(128, 0x8000, np.uint16)
+    codes, _ = oracle.quantize_block(neg0)
+    assert (codes == 0x80).all()
+
+
+# ----------------------------------------------------------------------------- dispatch
+
+def _tiny(mask=0.0, **kw):
+    wl = W.WORKLOADS["tiny"].with_(**kw)
+    idx, w = W.gen_routing(wl)
+    if mask:
+        idx = W.mask_entries(wl, idx, mask)
+    x = W.gen_x(wl)
+    return wl, idx.numpy(), w.numpy(), x
+
+
+@pytest.mark.parametrize("zero_padding", [True, False])
+@pytest.mark.parametrize("mask", [0.0, 0.25])
+def test_dispatch_bf16_is_a_gather(zero_padding, mask):
+    wl, idx, w, x = _tiny(mask)
+    E, R, A = wl.experts, wl.ranks, wl.alignment
+    lay = oracle.layout(idx, w, E, R, A)
+    cap = int(lay.rows_per_rank.max()) + 3
+    st, recv, rw = oracle.dispatch_bf16(lay, idx, w, bits(x), E, R, A, cap, zero_padding)
+    assert st == oracle.OK
+    xb = bits(x)
+    e_loc = E // R
+    for t in range(wl.tokens):
+        for j in range(wl.topk):
+            if idx[t, j] >= 0:
+                r = idx[t, j] // e_loc
+                assert (recv[r, lay.slot[t, j]] == xb[t]).all()
+                assert rw[r, lay.slot[t, j]] == w[t, j]
+    for r in range(R):
+        pad = lay.row_src[r, :lay.rows_per_rank[r]] == -1
+        rows = recv[r, :lay.rows_per_rank[r]][pad]
+        assert (rows == (0 if zero_padding else 0xA5A5)).all()
+        assert (rw[r, :lay.rows_per_rank[r]][pad] == 0).all()
+        assert (recv[r, lay.rows_per_rank[r]:] == 0xA5A5).all()      # beyond the rows: untouched
+
+
+def test_dispatch_fp8_rows_match_block_quantiser():
+    wl, idx, w, x = _tiny(0.1, hidden=512)
+    E, R, A = wl.experts, wl.ranks, wl.alignment
+    lay = oracle.layout(idx, w, E, R, A)
+    cap = int(lay.rows_per_rank.max())
+    st, codes, scales, rw = oracle.dispatch_fp8(lay, idx, w, bits(x), E, R, A, cap, True)
+    assert st == oracle.OK
+    xb = bits(x)
+    e_loc = E // R
+    for t in range(wl.tokens):
+        ref = [oracle.quantize_block(xb[t, b:b + 128]) for b in range(0, 512, 128)]
+        for j in range(wl.topk):
+            if idx[t, j] >= 0:
+                r, s = idx[t, j] // e_loc, lay.slot[t, j]
+                assert (codes[r, s] == np.concatenate([c for c, _ in ref])).all()
+                assert (scales[r, s] == np.array([v for _, v in ref], np.float32)).all()
+    for r in range(R):
+        pad = lay.row_src[r, :lay.rows_per_rank[r]] == -1
+        assert (codes[r, :lay.rows_per_rank[r]][pad] == 0).all()
+        assert (scales[r, :lay.rows_per_rank[r]][pad] == 0).all()
+
+
+# ----------------------------------------------------------------------------- combine
+
+def _roundtrip(wl, idx, w, x):
+    E, R, A = wl.experts, wl.ranks, wl.alignment
+    lay = oracle.layout(idx, w, E, R, A)
+    cap = int(lay.rows_per_rank.max())
+    _, recv, _ = oracle.dispatch_bf16(lay, idx, w, bits(x), E, R, A, cap, True)
+    return lay, recv
+
+
+def test_combine_identity_expert_unit_weights_reproduces_x():
+    wl, idx, w, x = _tiny()
+    lay, recv = _roundtrip(wl, idx, w, x)
+    st, out = oracle.combine(idx, lay.slot, recv, wl.experts, wl.ranks, w=w)
+    assert st == oracle.OK
+    xf = x.float().numpy()
+    of = out.astype(np.uint32) << 16
+    of = of.view(np.float32)
+    assert (np.abs(of - xf) <= 2.0 ** -7 * np.abs(xf) + 1e-6).all()
+
+
+def test_combine_single_expert_unit_weight_exact():
+    wl, idx, w, x = _tiny(topk=1)
+    lay, recv = _roundtrip(wl, idx, w, x)
+    st, out = oracle.combine(idx, lay.slot, recv, wl.experts, wl.ranks, w=np.ones_like(w))
+    assert (out == bits(x)).all()
+    st, out = oracle.combine(idx, lay.slot, recv, wl.experts, wl.ranks)
+    assert (out == bits(x)).all()
+
+
+def test_combine_bias_only_exact():
+    wl, idx, w, x = _tiny(mask=0.3)
+    lay, recv = _roundtrip(wl, idx, w, x)
+    bias = W.gen_bias(wl)
+    st, out = oracle.combine(idx, lay.slot, np.zeros_like(recv), wl.experts, wl.ranks, w=w, bias_bits=bits(bias))
+    assert (out == bits(bias)).all()
+
+
+def test_combine_unweighted_sum_of_copies():
+    """With an identity expert and no weights, each token gets k_valid * x: exact in fp32 and,
+    for k_valid a power of two, exact in bf16 too."""
+    wl, idx, w, x = _tiny()
+    lay, recv = _roundtrip(wl, idx, w, x)
+    st, out = oracle.combine(idx, lay.slot, recv, wl.experts, wl.ranks)
+    assert (out == bits((x.float() * 2).to(torch.bfloat16))).all()   # tiny has k = 2
+
+
+@pytest.mark.parametrize("weighted", [False, True])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_combine_fp32_within_tolerance_of_f64(weighted, with_bias):
+    wl, idx, w, x = _tiny(mask=0.1, topk=4)
+    lay = oracle.layout(idx, w, wl.experts, wl.ranks, wl.alignment)
+    cap = int(lay.rows_per_rank.max())
+    y = W.gen_y(wl, cap)
+    bias = bits(W.gen_bias(wl)) if with_bias else None
+    ww = w if weighted else None
+    st, out = oracle.combine(idx, lay.slot, bits(y), wl.experts, wl.ranks, w=ww, bias_bits=bias)
+    ref = oracle.combine_f64(idx, lay.slot, bits(y), wl.experts, wl.ranks, w=ww, bias_bits=bias)
+    got = (out.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert (np.abs(got - ref) <= 2.0 ** -7 * np.abs(ref) + 1e-6).all()
+    # the f64 statement against a numpy gather-and-sum of the same rows
+    e_loc = wl.experts // wl.ranks
+    yf = y.float().numpy().astype(np.float64)
+    for t in range(0, wl.tokens, 7):
+        acc = np.zeros(wl.hidden)
+        for j in range(wl.topk):
+            if idx[t, j] >= 0:
+                acc += (float(w[t, j]) if weighted else 1.0) * yf[idx[t, j] // e_loc, lay.slot[t, j]]
+        if with_bias:
+            acc += W.gen_bias(wl)[t].float().numpy()
+        assert np.allclose(acc, ref[t], rtol=0, atol=1e-12)
+
+
+def test_bf16_rounding_definition():
+    for v in [1.0, -2.5, 3.0e38, 1e-40, 0.1, 1.00390625, 1.01171875]:
+        assert oracle.float_to_bf16(v) == bits(torch.tensor([v], dtype=torch.float32).to(torch.bfloat16))[0]
+    assert oracle.float_to_bf16(float("nan")) == 0x7FC0
+    # ties: 1 + 2^-8 is halfway between 1 and 1 + 2^-7 -> even (1.0)
+    assert oracle.float_to_bf16(1.00390625) == 0x3F80
