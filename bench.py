@@ -1,0 +1,409 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE token round trip (layout -> dispatch -> combine) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload deepseek] [--impl ours|reference]
+
+One step = one pass of the whole path over one synthetic batch: layout (count, scan, host count
+sync, assign), FP8 dispatch (with zero padding), BF16 combine, handle release.  The metric is
+dispatch+combine algorithmic HBM bytes / step time (layout time counts against it).  N > 1 runs
+one independent replica per GPU under torchrun (logical ranks live inside one GPU, so nothing
+crosses GPUs); the value is the sum over GPUs of the bytes / max-over-ranks time.
+
+--impl reference times the CPU oracle (single-threaded C, test infrastructure) on a bounded sample
+of the same workload each step; only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "dispatch+combine GB/s & % of B200 HBM peak at 4096×7168 top-8/256 experts"
+UNIT = "GB/s"
+WORKLOAD_NAMES = {"deepseek": "deepseek-v3-prefill", "decode": "decode-low-latency", "large": "large-capacity",
+                  "skewed": "skewed-load", "tiny": "tiny"}
+FALLBACK_HBM_GBS = 6650.0
+
+
+# --------------------------------------------------------------------------- byte model
+def algorithmic_bytes(wl: W.Workload, valid_pairs: int, pad_rows: int, weighted: bool = False) -> dict:
+    """Bytes the method must move (not what a kernel happens to move)."""
+    T, H, k = wl.tokens, wl.hidden, wl.topk
+    row = (H + 4 * (H // 128)) if wl.fp8 else 2 * H
+    dispatch = T * H * 2 + valid_pairs * row + (pad_rows * row if wl.zero_padding else 0) + T * k * 8
+    combine = valid_pairs * H * 2 + T * H * 2 + (T * H * 2 if wl.bias else 0) + T * k * 8 + (T * k * 4 if weighted else 0)
+    layout = 2 * T * k * 8 + T * k * 4 + (valid_pairs + pad_rows) * 8
+    return {"dispatch": dispatch, "combine": combine, "layout": layout}
+
+
+def kernel_source_digest(*files: str) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "combine_moe_layout_07_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+KERNEL_SOURCES = {"combine": ("combine.cu", "moe_internal.cuh"), "dispatch": ("dispatch.cu", "moe_internal.cuh")}
+
+
+def measured_traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch recorded from an ncu capture of the same kernel source;
+    None if no record or if the kernel source changed since."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    if not os.path.exists(path):
+        return None
+    digest = kernel_source_digest(*KERNEL_SOURCES[kernel])
+    for line in open(path):
+        m = re.match(r"\|\s*(\w+)\s*\|\s*([\w-]+)\s*\|\s*([0-9.e+]+)\s*\|\s*([0-9a-f]{12})\s*\|", line)
+        if m and m.group(1) == kernel and m.group(2) == workload and m.group(4) == digest:
+            return float(m.group(3))
+    return None
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        return float(json.load(open(path))["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r.split(",") for r in self.out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- distributed plumbing
+def dist_setup(backend: str):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def reduce_max(value: float, device) -> float:
+    """Max of a scalar over all ranks (identity when not distributed)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------- CPU oracle sample
+def oracle_sample(wl: W.Workload, tokens: int):
+    """Run the CPU oracle (layout, dispatch, combine) on the first `tokens` tokens of the
+    workload's batch; returns (seconds, algorithmic bytes, description)."""
+    import oracle
+    tpr = max(1, tokens // wl.ranks)
+    sw = wl.with_(tokens_per_rank=tpr)
+    idx, w = W.gen_routing(wl)
+    idx, w = idx[: sw.tokens].numpy(), w[: sw.tokens].numpy()
+    x = W.gen_x(sw)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    E, R, A = sw.experts, sw.ranks, sw.alignment
+    lay = oracle.layout(idx, w, E, R, A)
+    cap = int(lay.rows_per_rank.max())
+    y = W.gen_y(sw, cap).view(torch.int16).numpy().view(np.uint16)
+    bias = W.gen_bias(sw).view(torch.int16).numpy().view(np.uint16) if sw.bias else None
+    t0 = time.perf_counter()
+    lay = oracle.layout(idx, w, E, R, A, cap=cap)
+    if sw.fp8:
+        oracle.dispatch_fp8(lay, idx, w, xb, E, R, A, cap, sw.zero_padding, want_w=False)
+    else:
+        oracle.dispatch_bf16(lay, idx, w, xb, E, R, A, cap, sw.zero_padding, want_w=False)
+    oracle.combine(idx, lay.slot, y, E, R, bias_bits=bias)
+    dt = time.perf_counter() - t0
+    valid = int(lay.cnt.sum())
+    pad = int(lay.rows_per_rank.sum()) - valid
+    b = algorithmic_bytes(sw, valid, pad)
+    desc = (f"first {sw.tokens} tokens ({tpr}/rank) of the {wl.name} batch, same E/R/k/H/A; "
+            f"layout+dispatch+combine by the single-threaded C oracle")
+    return dt, b["dispatch"] + b["combine"], desc
+
+
+def workload_config(wl: W.Workload, cap: int, extra: dict | None = None) -> dict:
+    cfg = {"workload": WORKLOAD_NAMES.get(wl.name, wl.name), "tokens": wl.tokens,
+           "tokens_per_rank": wl.tokens_per_rank, "logical_ranks": wl.ranks, "hidden": wl.hidden,
+           "experts": wl.experts, "topk": wl.topk, "expert_alignment": wl.alignment, "routing": wl.routing,
+           "dispatch": "fp8_e4m3 1x128 block scales" if wl.fp8 else "bf16",
+           "combine": "bf16 out, fp32 accumulate" + (", weighted" if wl.weighted_combine else ", pre-weighted rows")
+                      + (", shared-expert bias" if wl.bias else ", no bias"),
+           "do_cpu_sync": int(wl.cpu_sync), "do_zero_padding": int(wl.zero_padding),
+           "num_sms": wl.num_sms or "all", "recv_capacity_rows": cap,
+           "l2": "no flush: every step moves several GB (> 126 MB L2)"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args) -> int:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = W.WORKLOADS[args.workload]
+    tokens = args.ref_tokens
+    times, nbytes, desc = [], 0, ""
+    for i in range(args.warmup + args.steps):
+        dt, nbytes, desc = oracle_sample(wl, tokens)
+        if i >= args.warmup:
+            times.append(dt)
+    mean = sum(times) / len(times)
+    value = nbytes / mean / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(wl, 0, {"sample_tokens": tokens}),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- our arm
+def run_ours(args) -> int:
+    world, rank, local = dist_setup("nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import combine_moe_layout_07_b200 as moe
+
+    wl = W.WORKLOADS[args.workload]
+    stream = torch.cuda.current_stream()
+    idx_c, w_c = W.gen_routing(wl)
+    x_c = W.gen_x(wl)
+    bias_c = W.gen_bias(wl) if wl.bias else None
+    idx, w, x = idx_c.to(dev), w_c.to(dev), x_c.to(dev)
+    bias = bias_c.to(dev) if bias_c is not None else None
+    weights_for_combine = w if wl.weighted_combine else None
+
+    def make_params(cap_rows: int):
+        return moe.params(wl.tokens, wl.ranks, wl.experts, wl.topk, wl.hidden, wl.alignment,
+                          recv_capacity_rows=cap_rows, num_sms=wl.num_sms, do_cpu_sync=wl.cpu_sync)
+
+    # capacity: worst-case bound for the no-sync decode path, else the exact counts of this batch
+    if wl.max_tokens_per_rank:
+        cap = moe.moe_recv_capacity_hint(make_params(1), wl.max_tokens_per_rank)
+    else:
+        h0 = moe.moe_layout(make_params(0), idx, w)
+        cap = int(h0.host_rows_per_rank.max())
+        moe.moe_handle_free(h0)
+    p_cap = 0 if wl.cpu_sync else cap
+    h0 = moe.moe_layout(make_params(cap), idx, w)
+    counts = h0.counts().cpu().numpy()
+    rows = h0.rows_per_rank().cpu().numpy()
+    moe.moe_handle_free(h0)
+    valid_pairs = int(counts.sum())
+    pad_rows = int(rows.sum()) - valid_pairs
+    nb = algorithmic_bytes(wl, valid_pairs, pad_rows, weighted=wl.weighted_combine)
+    step_bytes = nb["dispatch"] + nb["combine"]
+
+    dtype_out = moe.MOE_DTYPE_FP8_E4M3 if wl.fp8 else moe.MOE_DTYPE_BF16
+    if wl.fp8:
+        recv = torch.empty(wl.ranks, cap, wl.hidden, dtype=torch.uint8, device=dev)
+        scales = torch.empty(wl.ranks, cap, wl.hidden // 128, dtype=torch.float32, device=dev)
+    else:
+        recv = torch.empty(wl.ranks, cap, wl.hidden, dtype=torch.bfloat16, device=dev)
+        scales = None
+    y = W.gen_y_device(wl, cap, device=dev)
+    out = torch.empty(wl.tokens, wl.hidden, dtype=torch.bfloat16, device=dev)
+
+    ev = {k: [] for k in ("l0", "l1", "d1", "c1")}
+
+    def step(record: bool):
+        if record:
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            e[0].record(stream)
+        h = moe.moe_layout(make_params(p_cap), idx, w, stream=stream)
+        if record:
+            e[1].record(stream)
+        moe.moe_dispatch(h, x, dtype_out, recv, scales, None, cap=cap, do_zero_padding=wl.zero_padding,
+                         num_sms=wl.num_sms, stream=stream)
+        if record:
+            e[2].record(stream)
+        moe.moe_combine(h, y, out, topk_weights=weights_for_combine, bias=bias, cap=cap, num_sms=wl.num_sms,
+                        stream=stream)
+        if record:
+            e[3].record(stream)
+            for key, val in zip(ev, e):
+                ev[key].append(val)
+        moe.moe_handle_free(h)
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    assert moe.moe_handle_status(moe.moe_layout(make_params(p_cap), idx, w)) == moe.MOE_OK
+
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = moe.moe_kernel_launch_count()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for _ in range(args.steps):
+            step(True)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    launches = moe.moe_kernel_launch_count() - launches0
+    ms = reduce_max(t_start.elapsed_time(t_end), dev) / args.steps
+    layout_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["l0"], ev["l1"]))
+    dispatch_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["l1"], ev["d1"]))
+    combine_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["d1"], ev["c1"]))
+    value = world * step_bytes / (ms * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host inputs -> device, round trip, result -> host
+    x_h = x_c.pin_memory()
+    idx_h, w_h = idx_c.pin_memory(), w_c.pin_memory()
+    y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    y_h.copy_(y)
+    bias_h = bias_c.pin_memory() if bias_c is not None else None
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = x_h.numel() * 2 + idx_h.numel() * 8 + w_h.numel() * 4 + y_h.numel() * 2 + (bias_h.numel() * 2 if bias_h is not None else 0)
+    d2h = out_h.numel() * 2
+
+    def e2e_step():
+        x.copy_(x_h, non_blocking=True)
+        idx.copy_(idx_h, non_blocking=True)
+        w.copy_(w_h, non_blocking=True)
+        y.copy_(y_h, non_blocking=True)
+        if bias_h is not None:
+            bias.copy_(bias_h, non_blocking=True)
+        step(False)
+        out_h.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, 10))
+    barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = reduce_max(a.elapsed_time(b), dev) / e2e_steps
+    e2e_value = world * step_bytes / (e2e_ms * 1e-3) / 1e9
+
+    peak, peak_kind = hbm_peak()
+    kern = {"dispatch": (dispatch_ms, nb["dispatch"]), "combine": (combine_ms, nb["combine"])}
+    dom = max(kern, key=lambda k: kern[k][0])
+    achieved = kern[dom][1] / (kern[dom][0] * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": f"k_{dom}", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "algorithmic_bytes_per_launch": kern[dom][1],
+                "traffic": measured_traffic(dom, args.workload)}
+
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        dt, cb, desc = oracle_sample(wl, args.cpu_tokens)
+        cpu = {"value": cb / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "data_types": {"x": "bf16", "recv": "e4m3 + f32 scales" if wl.fp8 else "bf16", "y,out": "bf16"},
+                "config": workload_config(wl, cap, {"parallelism": f"{world} independent replica(s), "
+                                                                   f"{wl.ranks} logical EP ranks each"}),
+                "frac_of_hbm_peak": value / world / peak,
+                "frac_of_8tbs_nominal": value / world / 8000.0,
+                "kernels_ms": {"layout": layout_ms, "dispatch": dispatch_ms, "combine": combine_ms},
+                "kernels_gbs": {"dispatch": nb["dispatch"] / dispatch_ms / 1e6, "combine": nb["combine"] / combine_ms / 1e6},
+                "bytes_per_step": nb, "valid_rows": valid_pairs, "padding_rows": pad_rows,
+                "A_pad": (valid_pairs + pad_rows) / max(valid_pairs, 1),
+                "rows_per_rank_max_over_mean": float(rows.max() / max(rows.mean(), 1e-9)),
+                "roofline": roofline, "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                        "ms_per_step": e2e_ms},
+                "gpu_launches": launches, "clocks": clk.summary(),
+                "library": os.path.relpath(moe.library_path(), ROOT)}
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def main() -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default="deepseek")
+    ap.add_argument("--cpu-tokens", type=int, default=16384, help="tokens in the CPU-oracle baseline sample")
+    ap.add_argument("--ref-tokens", type=int, default=4096, help="tokens per step of the reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return run_reference(args) if args.impl == "reference" else run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

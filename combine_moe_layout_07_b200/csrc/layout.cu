@@ -1,0 +1,288 @@
+// layout.cu -- routing -> counts, aligned prefix sums and the token->slot handle.
+//
+// Follows "From DeepEP to Mega MoE" (backyes.github.io) 2.2 (notify warps: per-expert counts
+// with block-local atomics, then an inclusive prefix sum psum_num_recv_tokens_per_expert) and
+// 2.4 (every routed row gets a position inside its expert's range), with expert_alignment and
+// the per-rank receive buffers of "Why MoE gets stuck on communication" (locsic.com) section 1,
+// and the rank count / expert count / membership outputs of layout.cu in "Chapter 2:
+// repository map" (bowenzhou.top) 2.1.
+//
+// The pages place rows with atomicAdd on the psum counter, whose order is undefined; here the
+// placement is a stable counting sort so the handle is deterministic:
+//   count  : per chunk of 512 tokens, a shared-memory histogram (atomicAdd_block) of expert ids
+//            and of token->rank membership;
+//   scan   : one CTA; per expert an exclusive scan of the chunk counts (chunk offsets), then a
+//            block-wide warp-shuffle scan of align_up(cnt, A), restarted at every rank;
+//   assign : per chunk, each warp takes a contiguous run of (t, j) pairs; per-warp histograms
+//            are scanned across warps, and inside a warp __match_any_sync + popc give each pair
+//            its rank among equal experts -- so rows keep ascending (t, j) order.
+#include "moe_internal.cuh"
+
+namespace moe {
+
+__device__ __forceinline__ int32_t align_up_dev(int32_t n, int32_t a) { return ((n + a - 1) / a) * a; }
+
+// ------------------------------------------------------------------------------------ count
+__global__ void __launch_bounds__(kLayoutThreads) k_layout_count(LayoutLaunch L) {
+  extern __shared__ int32_t sm[];
+  int32_t* hist = sm;          // [E]
+  int32_t* tok = sm + L.E;     // [R]
+  const int tid = threadIdx.x;
+  for (int c = blockIdx.x; c < L.num_chunks; c += gridDim.x) {
+    for (int i = tid; i < L.E + L.R; i += blockDim.x) sm[i] = 0;
+    __syncthreads();
+    const int64_t t0 = (int64_t)c * kChunkTokens;
+    const int64_t t1 = min(L.T, t0 + kChunkTokens);
+    bool bad = false;
+    for (int64_t p = t0 * L.k + tid; p < t1 * L.k; p += blockDim.x) {
+      const int64_t e = L.idx[p];
+      if (e >= 0 && e < L.E) atomicAdd_block(&hist[e], 1);
+      else if (e != -1) bad = true;
+    }
+    // membership: rank r holds token t if one of its k experts lives on r
+    for (int64_t t = t0 + tid; t < t1; t += blockDim.x) {
+      uint8_t* row = L.d.token_in_rank + t * L.R;
+      for (int r = 0; r < L.R; ++r) row[r] = 0;
+      for (int j = 0; j < L.k; ++j) {
+        const int64_t e = L.idx[t * L.k + j];
+        if (e < 0 || e >= L.E) continue;
+        const int r = (int)(e / L.E_loc);
+        if (!row[r]) {
+          row[r] = 1;
+          atomicAdd_block(&tok[r], 1);
+        }
+      }
+    }
+    if (bad) atomicOr(L.d.status, kStatusBadExpert);
+    __syncthreads();
+    for (int e = tid; e < L.E; e += blockDim.x) L.d.chunk_cnt[(int64_t)c * L.E + e] = hist[e];
+    for (int r = tid; r < L.R; r += blockDim.x) L.d.chunk_tok[(int64_t)c * L.R + r] = tok[r];
+    __syncthreads();
+  }
+}
+
+// Block-wide exclusive scan of one value per thread (warp shuffles + one smem pass).
+__device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_tot, int32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  int32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = lane < nwarps ? warp_tot[lane] : 0;
+    int32_t wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t n = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += n;
+    }
+    if (lane < nwarps) warp_tot[lane] = wi - w;  // exclusive warp offsets
+    if (lane == 31) *total = wi;
+  }
+  __syncthreads();
+  const int32_t r = warp_tot[warp] + incl - v;
+  __syncthreads();
+  return r;
+}
+
+// ------------------------------------------------------------------------------------ scan
+__global__ void __launch_bounds__(kScanThreads) k_layout_scan(LayoutLaunch L, int64_t cap_check) {
+  __shared__ int32_t warp_tot[32];
+  __shared__ int32_t totals[2];
+  extern __shared__ int32_t sm[];
+  int32_t* al = sm;              // [E] align_up(cnt, A)
+  int32_t* pad = sm + L.E;       // [E] align_up(cnt, A) - cnt
+  int32_t* gincl = sm + 2 * L.E; // [E] inclusive prefix of al over all experts
+  const int tid = threadIdx.x;
+  const int E = L.E;
+
+  // 1. per expert: exclusive scan over chunks (in place), total count
+  for (int e = tid; e < E; e += blockDim.x) {
+    int32_t run = 0;
+    for (int c = 0; c < L.num_chunks; ++c) {
+      int32_t* q = L.d.chunk_cnt + (int64_t)c * E + e;
+      const int32_t v = *q;
+      *q = run;
+      run += v;
+    }
+    L.d.cnt[e] = run;
+    al[e] = align_up_dev(run, L.A);
+    pad[e] = al[e] - run;
+  }
+  __syncthreads();
+
+  // 2. each thread owns a contiguous run of experts; block scan of the run sums
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
+  int32_t sa = 0, sp = 0;
+  for (int e = e0; e < e1; ++e) { sa += al[e]; sp += pad[e]; }
+  int32_t ra = block_exclusive_scan(sa, warp_tot, &totals[0]);
+  int32_t rp = block_exclusive_scan(sp, warp_tot, &totals[1]);
+  for (int e = e0; e < e1; ++e) {
+    L.d.pad_excl[e] = rp;
+    rp += pad[e];
+    ra += al[e];
+    gincl[e] = ra;
+  }
+  if (tid == 0) L.d.pad_excl[E] = totals[1];
+  __syncthreads();
+
+  // 3. restart at every rank: psum[e] = gincl[e] - (exclusive prefix at the rank's first expert)
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int first = (e / L.E_loc) * L.E_loc;
+    L.d.psum[e] = gincl[e] - (gincl[first] - al[first]);
+  }
+  for (int r = tid; r < L.R; r += blockDim.x) {
+    const int first = r * L.E_loc, last = first + L.E_loc - 1;
+    const int32_t rows = gincl[last] - (gincl[first] - al[first]);
+    L.d.rows_per_rank[r] = rows;
+    if (cap_check > 0 && rows > cap_check) atomicOr(L.d.status, kStatusCapacity);
+    int32_t tk = 0;
+    for (int c = 0; c < L.num_chunks; ++c) tk += L.d.chunk_tok[(int64_t)c * L.R + r];
+    L.d.tokens_per_rank[r] = tk;
+  }
+}
+
+// ------------------------------------------------------------------------------------ assign
+__global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L) {
+  extern __shared__ int32_t whist[];  // [kLayoutWarps][E]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int E = L.E;
+  int32_t* h = whist + warp * E;
+  const uint32_t lt = lanemask_lt();
+  bool overflow = false;
+
+  for (int c = blockIdx.x; c < L.num_chunks; c += gridDim.x) {
+    const int64_t t0 = (int64_t)c * kChunkTokens;
+    const int64_t t1 = min(L.T, t0 + kChunkTokens);
+    const int64_t p0 = t0 * L.k, np = (t1 - t0) * L.k;
+    const int64_t per = (np + kLayoutWarps - 1) / kLayoutWarps;
+    const int64_t wp0 = p0 + min(np, warp * per), wp1 = p0 + min(np, (warp + 1) * per);
+
+    // phase 1: this warp's histogram of its pairs
+    for (int e = lane; e < E; e += 32) h[e] = 0;
+    __syncwarp();
+    for (int64_t base = wp0; base < wp1; base += 32) {
+      const int64_t p = base + lane;
+      const int64_t e = p < wp1 ? L.idx[p] : -1;
+      const bool valid = e >= 0 && e < E;
+      const uint32_t peers = __match_any_sync(0xffffffffu, valid ? (int)e : -1);
+      if (valid && lane == __ffs(peers) - 1) h[e] += __popc(peers);
+      __syncwarp();
+    }
+    __syncthreads();
+
+    // phase 2: per expert, exclusive scan across warps, based at the expert's first row for
+    // this chunk (segment start + chunk offset)
+    for (int e = tid; e < E; e += blockDim.x) {
+      int32_t base = L.d.psum[e] - align_up_dev(L.d.cnt[e], L.A) + L.d.chunk_cnt[(int64_t)c * E + e];
+      for (int w = 0; w < kLayoutWarps; ++w) {
+        const int32_t v = whist[w * E + e];
+        whist[w * E + e] = base;
+        base += v;
+      }
+    }
+    __syncthreads();
+
+    // phase 3: walk the pairs again in order; equal experts inside a round are ranked by lane
+    for (int64_t base = wp0; base < wp1; base += 32) {
+      const int64_t p = base + lane;
+      const bool in = p < wp1;
+      const int64_t e = in ? L.idx[p] : -1;
+      const bool valid = in && e >= 0 && e < E;
+      const uint32_t peers = __match_any_sync(0xffffffffu, valid ? (int)e : -1);
+      int32_t row = -1;
+      if (valid) row = h[e] + __popc(peers & lt);
+      __syncwarp();
+      if (valid && lane == __ffs(peers) - 1) h[e] += __popc(peers);
+      __syncwarp();
+      if (in) {
+        const float wv = L.w ? L.w[p] : 0.0f;
+        L.d.slot[p] = row;
+        L.d.pair_rank[p] = valid ? (int32_t)(e / L.E_loc) : -1;
+        L.d.pair_w[p] = wv;
+        if (valid) {
+          const int r = (int)(e / L.E_loc);
+          if (row < L.row_cap) {
+            L.d.row_src[(int64_t)r * L.row_cap + row] = (int32_t)(p / L.k);
+            L.d.row_w[(int64_t)r * L.row_cap + row] = wv;
+          } else {
+            overflow = true;
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // padding rows of the row maps: global padding index i -> expert by binary search
+  const int32_t total_pad = L.d.pad_excl[E];
+  for (int32_t i = blockIdx.x * blockDim.x + tid; i < total_pad; i += gridDim.x * blockDim.x) {
+    int lo = 0, hi = E;  // largest e with pad_excl[e] <= i
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (L.d.pad_excl[mid] <= i) lo = mid; else hi = mid;
+    }
+    const int e = lo;
+    const int32_t pad_e = L.d.pad_excl[e + 1] - L.d.pad_excl[e];
+    const int32_t row = L.d.psum[e] - pad_e + (i - L.d.pad_excl[e]);
+    const int r = e / L.E_loc;
+    if (row < L.row_cap) {
+      L.d.row_src[(int64_t)r * L.row_cap + row] = -1;
+      L.d.row_w[(int64_t)r * L.row_cap + row] = 0.0f;
+    } else {
+      overflow = true;
+    }
+  }
+  if (overflow) atomicOr(L.d.status, kStatusCapacity);
+}
+
+// ------------------------------------------------------------------------------------ launch
+// Opt in to the dynamic shared memory the largest supported E needs, once per device.
+static cudaError_t ensure_smem_attrs() {
+  static unsigned long long done = 0;  // one bit per device ordinal
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 64 && (done >> dev) & 1ull) return cudaSuccess;
+  err = cudaFuncSetAttribute(k_layout_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(sizeof(int32_t) * 3 * kMaxExperts));
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(k_layout_assign, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)(sizeof(int32_t) * kLayoutWarps * kMaxExperts));
+  if (err == cudaSuccess && dev < 64) done |= 1ull << dev;
+  return err;
+}
+
+cudaError_t launch_layout_count(const LayoutLaunch& L, cudaStream_t s) {
+  if (L.num_chunks == 0) return cudaSuccess;
+  const size_t smem = sizeof(int32_t) * (size_t)(L.E + L.R);
+  k_layout_count<<<L.grid_chunks, kLayoutThreads, smem, s>>>(L);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_layout_scan(const LayoutLaunch& L, int64_t cap_check, cudaStream_t s) {
+  cudaError_t err = ensure_smem_attrs();
+  if (err != cudaSuccess) return err;
+  const size_t smem = sizeof(int32_t) * 3 * (size_t)L.E;
+  k_layout_scan<<<1, kScanThreads, smem, s>>>(L, cap_check);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_layout_assign(const LayoutLaunch& L, cudaStream_t s) {
+  cudaError_t err = ensure_smem_attrs();
+  if (err != cudaSuccess) return err;
+  const size_t smem = sizeof(int32_t) * (size_t)kLayoutWarps * L.E;
+  const int grid = L.grid_chunks > 0 ? L.grid_chunks : 1;
+  k_layout_assign<<<grid, kLayoutThreads, smem, s>>>(L);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,384 @@
+// moe_api.cu -- the C ABI declared in include/moe.h: argument checks, the handle's device
+// memory, and the order of kernel launches for layout, dispatch and combine.
+//
+// The handle follows "Why MoE gets stuck on communication" (locsic.com) section 1 and 2: it
+// records one dispatch's grouping and counts, combine reuses it, and it must outlive every
+// operation that uses it.  do_cpu_sync follows the same page and "deepep-expert-parallel-
+// dispatch-combine" (phantomic12.github.io): with it, the counts are copied to the host and
+// the call waits; without it, nothing waits and consumers read the device-side psum.
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+static std::atomic<int64_t> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+int sm_count(int device) {
+  static int cache[64] = {0};
+  if (device >= 0 && device < 64 && cache[device] > 0) return cache[device];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n <= 0) n = 1;
+  if (device >= 0 && device < 64) cache[device] = n;
+  return n;
+}
+
+static int grid_for(int num_sms, int device) {
+  const int n = sm_count(device);
+  return (num_sms > 0 && num_sms < n) ? num_sms : n;
+}
+
+// The handle's arrays come from a library-owned stream-ordered pool per device whose release
+// threshold keeps freed blocks mapped, so a layout -> free -> layout cycle reuses memory instead
+// of returning it to the driver at every synchronisation.
+static cudaError_t handle_pool(int device, cudaMemPool_t* out) {
+  static cudaMemPool_t pools[64] = {};
+  static std::mutex mu;
+  if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!pools[device]) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = device;
+    cudaMemPool_t pool;
+    cudaError_t err = cudaMemPoolCreate(&pool, &props);
+    if (err != cudaSuccess) return err;
+    uint64_t keep = ~0ull;
+    err = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (err != cudaSuccess) return err;
+    pools[device] = pool;
+  }
+  *out = pools[device];
+  return cudaSuccess;
+}
+
+static cudaError_t pool_alloc(void** p, size_t bytes, int device, cudaStream_t s) {
+  cudaMemPool_t pool;
+  cudaError_t err = handle_pool(device, &pool);
+  if (err != cudaSuccess) return err;
+  return cudaMallocFromPoolAsync(p, bytes, pool, s);
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+static int64_t align_up64(int64_t n, int64_t a) { return ((n + a - 1) / a) * a; }
+
+// Pinned host staging for the do_cpu_sync copy, one per host thread.
+struct PinnedStage {
+  void* p = nullptr;
+  size_t n = 0;
+  ~PinnedStage() {
+    if (p) cudaFreeHost(p);
+  }
+  void* get(size_t need) {
+    if (need <= n) return p;
+    if (p) cudaFreeHost(p);
+    p = nullptr;
+    n = 0;
+    if (cudaMallocHost(&p, need) != cudaSuccess) return nullptr;
+    n = need;
+    return p;
+  }
+};
+static thread_local PinnedStage g_stage;
+
+static int check_params(const moe_params_t* p) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (p->num_tokens < 0 || p->num_logical_ranks < 1 || p->num_experts < 1 || p->topk < 1 ||
+      p->expert_alignment < 1 || p->hidden < 8 || p->hidden % 8 != 0 || p->num_sms < 0 ||
+      p->reserved != 0 || (p->do_cpu_sync != 0 && p->do_cpu_sync != 1) || p->recv_capacity_rows < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (p->num_experts % p->num_logical_ranks != 0) return MOE_ERR_INVALID_ARG;
+  if (p->topk > kMaxTopk || p->num_experts > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+  // every row index and prefix sum must fit in int32
+  if (p->num_tokens * (int64_t)p->topk + (int64_t)p->num_experts * p->expert_alignment >= (int64_t)1 << 31)
+    return MOE_ERR_UNSUPPORTED;
+  if (p->recv_capacity_rows >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+  if (p->recv_capacity_rows == 0 && p->do_cpu_sync == 0) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+static void release(moe_handle_t* h) {
+  if (!h) return;
+  if (h->row_block) cudaFreeAsync(h->row_block, h->stream);
+  if (h->block) cudaFreeAsync(h->block, h->stream);
+  delete h;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int64_t moe_recv_capacity_hint(const moe_params_t* p, int64_t max_tokens_per_rank) {
+  if (check_params(p) == MOE_ERR_INVALID_ARG || max_tokens_per_rank < 0) return -1;
+  const int64_t e_loc = p->num_experts / p->num_logical_ranks;
+  const int64_t per_token = p->topk < e_loc ? p->topk : e_loc;
+  return (int64_t)p->num_logical_ranks * max_tokens_per_rank * per_token + e_loc * (p->expert_alignment - 1);
+}
+
+int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk_weights, void* stream,
+               moe_handle_t** out_handle, int32_t* host_rows_per_rank) {
+  if (!out_handle) return MOE_ERR_INVALID_ARG;
+  *out_handle = nullptr;
+  int rc = check_params(p);
+  if (rc != MOE_OK) return rc;
+  if (!topk_idx && p->num_tokens > 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned4(topk_weights)) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(topk_idx) & 7u) != 0) return MOE_ERR_INVALID_ARG;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  moe_handle_t* h = new (std::nothrow) moe_handle_t();
+  if (!h) return MOE_ERR_OOM;
+  h->p = *p;
+  h->stream = s;
+  if (cudaGetDevice(&h->device) != cudaSuccess) {
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  const int64_t T = p->num_tokens, k = p->topk, E = p->num_experts, R = p->num_logical_ranks;
+  h->num_chunks = (int)((T + kChunkTokens - 1) / kChunkTokens);
+  const int64_t C = h->num_chunks;
+
+  // one allocation for the fixed-size arrays (256-byte aligned sub-arrays)
+  int64_t off = 0;
+  auto take = [&](int64_t bytes) {
+    const int64_t at = off;
+    off = align_up64(off + bytes, 256);
+    return at;
+  };
+  const int64_t o_status = take(16), o_rows = take(4 * R), o_tok = take(4 * R), o_cnt = take(4 * E),
+                o_psum = take(4 * E), o_pad = take(4 * (E + 1)), o_tir = take(T * R), o_slot = take(4 * T * k),
+                o_prank = take(4 * T * k), o_pw = take(4 * T * k), o_ccnt = take(4 * C * E), o_ctok = take(4 * C * R);
+  const bool rows_now = p->recv_capacity_rows > 0;
+  int64_t o_rsrc = 0, o_rw = 0;
+  if (rows_now) {
+    h->row_cap = p->recv_capacity_rows;
+    o_rsrc = take(4 * R * h->row_cap);
+    o_rw = take(4 * R * h->row_cap);
+  }
+  if (pool_alloc(&h->block, (size_t)off, h->device, s) != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return MOE_ERR_OOM;
+  }
+  char* b = static_cast<char*>(h->block);
+  DeviceArrays& d = h->d;
+  d.status = reinterpret_cast<int32_t*>(b + o_status);
+  d.rows_per_rank = reinterpret_cast<int32_t*>(b + o_rows);
+  d.tokens_per_rank = reinterpret_cast<int32_t*>(b + o_tok);
+  d.cnt = reinterpret_cast<int32_t*>(b + o_cnt);
+  d.psum = reinterpret_cast<int32_t*>(b + o_psum);
+  d.pad_excl = reinterpret_cast<int32_t*>(b + o_pad);
+  d.token_in_rank = reinterpret_cast<uint8_t*>(b + o_tir);
+  d.slot = reinterpret_cast<int32_t*>(b + o_slot);
+  d.pair_rank = reinterpret_cast<int32_t*>(b + o_prank);
+  d.pair_w = reinterpret_cast<float*>(b + o_pw);
+  d.chunk_cnt = reinterpret_cast<int32_t*>(b + o_ccnt);
+  d.chunk_tok = reinterpret_cast<int32_t*>(b + o_ctok);
+  if (rows_now) {
+    d.row_src = reinterpret_cast<int32_t*>(b + o_rsrc);
+    d.row_w = reinterpret_cast<float*>(b + o_rw);
+  }
+
+  LayoutLaunch L{};
+  L.idx = topk_idx;
+  L.w = topk_weights;
+  L.T = T;
+  L.k = (int)k;
+  L.E = (int)E;
+  L.R = (int)R;
+  L.E_loc = (int)(E / R);
+  L.A = p->expert_alignment;
+  L.num_chunks = h->num_chunks;
+  L.grid_chunks = h->num_chunks;
+  if (p->num_sms > 0 && L.grid_chunks > p->num_sms) L.grid_chunks = p->num_sms;
+  L.row_cap = h->row_cap;
+  L.d = d;
+
+  cudaError_t err = cudaMemsetAsync(d.status, 0, 16, s);
+  if (err == cudaSuccess) err = launch_layout_count(L, s);
+  if (err == cudaSuccess) err = launch_layout_scan(L, p->recv_capacity_rows, s);
+  if (err != cudaSuccess) {
+    release(h);
+    return MOE_ERR_CUDA;
+  }
+
+  if (p->do_cpu_sync) {
+    // counts to the host: [status flags, rows_per_rank[R], padding total]
+    int32_t* stage = static_cast<int32_t*>(g_stage.get(sizeof(int32_t) * (size_t)(R + 2)));
+    if (!stage) {
+      release(h);
+      return MOE_ERR_CUDA;
+    }
+    err = cudaMemcpyAsync(stage, d.status, 4, cudaMemcpyDeviceToHost, s);
+    if (err == cudaSuccess) err = cudaMemcpyAsync(stage + 1, d.rows_per_rank, 4 * R, cudaMemcpyDeviceToHost, s);
+    if (err == cudaSuccess) err = cudaMemcpyAsync(stage + 1 + R, d.pad_excl + E, 4, cudaMemcpyDeviceToHost, s);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+    if (err != cudaSuccess) {
+      release(h);
+      return MOE_ERR_CUDA;
+    }
+    if (stage[0] & kStatusBadExpert) {
+      release(h);
+      return MOE_ERR_BAD_EXPERT;
+    }
+    if (stage[0] & kStatusCapacity) {
+      release(h);
+      return MOE_ERR_CAPACITY;
+    }
+    h->host_rows.assign(stage + 1, stage + 1 + R);
+    h->host_total_pad = stage[1 + R];
+    h->counts_on_host = true;
+    if (host_rows_per_rank) std::memcpy(host_rows_per_rank, stage + 1, sizeof(int32_t) * (size_t)R);
+    if (!rows_now) {
+      int32_t mx = 0;
+      for (int32_t v : h->host_rows) mx = v > mx ? v : mx;
+      h->row_cap = mx;
+      if (mx > 0) {
+        const int64_t bytes = align_up64(4 * R * (int64_t)mx, 256);
+        if (pool_alloc(&h->row_block, (size_t)(2 * bytes), h->device, s) != cudaSuccess) {
+          cudaGetLastError();
+          release(h);
+          return MOE_ERR_OOM;
+        }
+        d.row_src = static_cast<int32_t*>(h->row_block);
+        d.row_w = reinterpret_cast<float*>(static_cast<char*>(h->row_block) + bytes);
+      }
+      L.row_cap = h->row_cap;
+      L.d = d;
+    }
+  }
+
+  err = launch_layout_assign(L, s);
+  if (err != cudaSuccess) {
+    release(h);
+    return MOE_ERR_CUDA;
+  }
+  *out_handle = h;
+  return MOE_OK;
+}
+
+int moe_dispatch(const moe_handle_t* h, const void* x, int out_dtype, void* recv_x, float* recv_scales,
+                 float* recv_weights, int64_t cap, int do_expand, int do_zero_padding, int num_sms,
+                 void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (do_expand != 0 && do_expand != 1) return MOE_ERR_INVALID_ARG;
+  if (do_zero_padding != 0 && do_zero_padding != 1) return MOE_ERR_INVALID_ARG;
+  if (out_dtype != MOE_DTYPE_BF16 && out_dtype != MOE_DTYPE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+  if (cap < 0 || cap >= (int64_t)1 << 31 || num_sms < 0) return MOE_ERR_INVALID_ARG;
+  const bool fp8 = out_dtype == MOE_DTYPE_FP8_E4M3;
+  const moe_params_t& p = h->p;
+  if (fp8 && (p.hidden % 128 != 0 || !recv_scales || !aligned4(recv_scales))) return MOE_ERR_INVALID_ARG;
+  if (p.num_tokens > 0 && (!x || !recv_x)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(recv_x) || !aligned4(recv_weights)) return MOE_ERR_INVALID_ARG;
+  if (!do_expand) return MOE_ERR_UNSUPPORTED;
+  if (h->counts_on_host) {
+    for (int32_t v : h->host_rows)
+      if (v > cap) return MOE_ERR_CAPACITY;
+  }
+  if (p.num_tokens == 0) return MOE_OK;
+  DispatchLaunch L{};
+  L.x = x;
+  L.recv_x = recv_x;
+  L.recv_scales = recv_scales;
+  L.recv_w = recv_weights;
+  L.T = p.num_tokens;
+  L.cap = cap;
+  L.H = p.hidden;
+  L.k = p.topk;
+  L.E = p.num_experts;
+  L.E_loc = p.num_experts / p.num_logical_ranks;
+  L.zero_padding = do_zero_padding;
+  L.grid = grid_for(num_sms, h->device);
+  L.pair_rank = h->d.pair_rank;
+  L.slot = h->d.slot;
+  L.pair_w = h->d.pair_w;
+  L.psum = h->d.psum;
+  L.pad_excl = h->d.pad_excl;
+  L.status = h->d.status;
+  return launch_dispatch(L, fp8, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_combine(const moe_handle_t* h, const void* y, const float* topk_weights, const void* bias, void* out,
+                int64_t cap, int num_sms, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (cap < 0 || cap >= (int64_t)1 << 31 || num_sms < 0) return MOE_ERR_INVALID_ARG;
+  const moe_params_t& p = h->p;
+  if (p.num_tokens > 0 && (!y || !out)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(out) || !aligned16(bias) || !aligned4(topk_weights)) return MOE_ERR_INVALID_ARG;
+  if (h->counts_on_host) {
+    for (int32_t v : h->host_rows)
+      if (v > cap) return MOE_ERR_CAPACITY;
+  }
+  if (p.num_tokens == 0) return MOE_OK;
+  CombineLaunch L{};
+  L.y = y;
+  L.w = topk_weights;
+  L.bias = bias;
+  L.out = out;
+  L.T = p.num_tokens;
+  L.cap = cap;
+  L.H = p.hidden;
+  L.k = p.topk;
+  L.grid = grid_for(num_sms, h->device);
+  L.pair_rank = h->d.pair_rank;
+  L.slot = h->d.slot;
+  L.status = h->d.status;
+  return launch_combine(L, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_handle_status(const moe_handle_t* h, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* stage = static_cast<int32_t*>(g_stage.get(16));
+  if (!stage) return MOE_ERR_CUDA;
+  if (cudaMemcpyAsync(stage, h->d.status, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (stage[0] & kStatusBadExpert) return MOE_ERR_BAD_EXPERT;
+  if (stage[0] & kStatusCapacity) return MOE_ERR_CAPACITY;
+  return MOE_OK;
+}
+
+const int32_t* moe_handle_counts(const moe_handle_t* h) { return h ? h->d.cnt : nullptr; }
+const int32_t* moe_handle_psum(const moe_handle_t* h) { return h ? h->d.psum : nullptr; }
+const int32_t* moe_handle_rows_per_rank(const moe_handle_t* h) { return h ? h->d.rows_per_rank : nullptr; }
+const int32_t* moe_handle_tokens_per_rank(const moe_handle_t* h) { return h ? h->d.tokens_per_rank : nullptr; }
+const uint8_t* moe_handle_token_in_rank(const moe_handle_t* h) { return h ? h->d.token_in_rank : nullptr; }
+const int32_t* moe_handle_slots(const moe_handle_t* h) { return h ? h->d.slot : nullptr; }
+const int32_t* moe_handle_row_src(const moe_handle_t* h) { return h ? h->d.row_src : nullptr; }
+const float* moe_handle_row_weights(const moe_handle_t* h) { return h ? h->d.row_w : nullptr; }
+int64_t moe_handle_row_capacity(const moe_handle_t* h) { return h ? h->row_cap : -1; }
+
+int moe_handle_free(moe_handle_t* h) {
+  if (!h) return MOE_OK;
+  int rc = MOE_OK;
+  if (h->row_block && cudaFreeAsync(h->row_block, h->stream) != cudaSuccess) rc = MOE_ERR_CUDA;
+  if (h->block && cudaFreeAsync(h->block, h->stream) != cudaSuccess) rc = MOE_ERR_CUDA;
+  delete h;
+  return rc;
+}
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_BAD_EXPERT: return "expert id outside [-1, num_experts)";
+    case MOE_ERR_CAPACITY: return "a logical rank needs more rows than the receive capacity";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_OOM: return "device memory allocation failed";
+    case MOE_ERR_UNSUPPORTED: return "unsupported by this build";
+    default: return "unknown status";
+  }
+}
+
+int64_t moe_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

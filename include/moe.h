@@ -1,0 +1,165 @@
+/*
+ * moe.h -- C ABI of the single-B200 MoE token round trip: layout -> dispatch -> combine.
+ *
+ * One MoE layer's token round trip with expert-parallel ranks emulated as logical partitions
+ * of one GPU's memory.  Sources (page title, section):
+ *   "Why MoE gets stuck on communication -- one expert-parallel round trip, end to end"
+ *     (locsic.com), section 1: a long-lived buffer with a uniform per-rank capacity; dispatch
+ *     with expert_alignment / do_expand / do_zero_padding / do_cpu_sync; a handle that records
+ *     the grouping and counts of one dispatch and is reused by combine; combine sums the
+ *     already-weighted expert outputs and adds the shared expert's output as a bias.
+ *   "From DeepEP to Mega MoE" (backyes.github.io), sections 2.2-2.5: per-expert counts with
+ *     block-local atomics, an inclusive prefix sum psum_num_recv_tokens_per_expert, placement
+ *     of every routed row inside its expert's range, element-wise top-k reduction in combine.
+ *   "deepep-expert-parallel-dispatch-combine" (phantomic12.github.io), "Arithmetic
+ *     intensity": with do_cpu_sync off, outputs are sized to capacity and consumers read the
+ *     device-side psum.
+ *   "DeepEP expert-parallel communication" (blog.hotdry.top), "Key techniques": num_sms caps
+ *     the SMs the data-movement kernels occupy; FP8 dispatch with BF16 combine.
+ *
+ * Conventions for every call
+ *   - T tokens, k = topk, E experts, R logical ranks, E_loc = E / R, A = expert_alignment,
+ *     H = hidden, cap = receive capacity in rows per logical rank (uniform over ranks).
+ *   - Expert e lives on logical rank e / E_loc.  topk_idx == -1 marks a masked entry.
+ *   - Receive buffers are [R, cap, ...] row-major; rank r's rows start at row 0 of block r.
+ *     Inside rank r, expert e owns rows [psum[e] - align_up(cnt[e], A), psum[e]); its routed
+ *     rows come first, in ascending (token, j) order, then its padding rows.
+ *   - Pointers are DEVICE pointers unless the argument says host.  Row pointers (x, recv_x,
+ *     recv_scales, y, bias, out) must be 16-byte aligned.  bf16 data is passed as void*.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *     stream-ordered and returns without waiting for the GPU, except where stated.
+ *   - Return value: MOE_OK or a negative MOE_ERR_*.  Argument errors are reported before
+ *     anything is launched.  Conditions only the GPU can see (an expert id outside [-1, E),
+ *     a rank needing more than cap rows) set a status word in the handle; the kernels skip
+ *     every write they would make out of range.  They are returned by moe_layout when
+ *     do_cpu_sync is set and otherwise by moe_handle_status.
+ *   - The library never falls back to the CPU and never allocates memory for the caller's
+ *     tensors; the caller owns x, topk_idx, topk_weights, the receive buffers, y, bias, out.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+enum moe_status_code {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1, /* bad size, flag, null or misaligned pointer */
+  MOE_ERR_BAD_EXPERT = -2,  /* a topk_idx entry outside [-1, E) */
+  MOE_ERR_CAPACITY = -3,    /* some logical rank needs more rows than the given capacity */
+  MOE_ERR_CUDA = -4,        /* a CUDA runtime call failed */
+  MOE_ERR_OOM = -5,         /* the handle's device memory could not be allocated */
+  MOE_ERR_UNSUPPORTED = -6  /* a valid request outside what this build implements */
+};
+
+enum moe_dtype { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_E4M3 = 1 };
+
+/* Problem description for moe_layout.  All fields are read once; the handle keeps a copy. */
+typedef struct moe_params {
+  int64_t num_tokens;         /* T >= 0 */
+  int32_t num_logical_ranks;  /* R >= 1, E % R == 0 */
+  int32_t num_experts;        /* E, 1 <= E <= 4096 */
+  int32_t topk;               /* k, 1 <= k <= 32 */
+  int32_t hidden;             /* H >= 8, H % 8 == 0 (BF16) and H % 128 == 0 for FP8 */
+  int32_t expert_alignment;   /* A >= 1; T*k + E*A < 2^31 */
+  int32_t num_sms;            /* SMs the layout kernels may occupy; 0 = all */
+  int32_t do_cpu_sync;        /* 1: moe_layout waits for the counts and copies them to host */
+  int32_t reserved;           /* must be 0 */
+  int64_t recv_capacity_rows; /* cap per rank for the handle's row maps; 0 only with
+                                 do_cpu_sync=1 (the rows are then sized from the counts) */
+} moe_params_t;
+
+typedef struct moe_handle moe_handle_t; /* opaque; owns its device arrays */
+
+/*
+ * Rows one logical rank may need when every rank sends it at most max_tokens_per_rank tokens:
+ * R * max_tokens_per_rank * min(k, E_loc) + E_loc * (A - 1).  Host only; no GPU work.
+ * Returns -1 on invalid parameters.  (The buffer size hint of the round-trip page, section 1.)
+ */
+int64_t moe_recv_capacity_hint(const moe_params_t* params, int64_t max_tokens_per_rank);
+
+/*
+ * Layout ("From DeepEP to Mega MoE" 2.2 and 2.4; "Why MoE gets stuck on communication" 1).
+ *   topk_idx      int64 [T, k], device.
+ *   topk_weights  fp32 [T, k], device, nullable (row weights then read 0).
+ *   out_handle    receives a new handle on MOE_OK (NULL otherwise).  Its device arrays are
+ *                 allocated stream-ordered on `stream` and freed by moe_handle_free.
+ *   host_rows_per_rank  int32 [R], host, nullable; filled when do_cpu_sync = 1.
+ * Fills, in the handle: cnt[E], psum[E] (aligned inclusive prefix per rank), rows_per_rank[R],
+ * tokens_per_rank[R], token_in_rank[T, R] (uint8), slot[T, k] (row inside its rank, -1 if
+ * masked), row_src[R, row_cap] (source token, -1 for padding rows), row_w[R, row_cap].
+ * With do_cpu_sync = 1 the call blocks until the counts reach the host and returns
+ * MOE_ERR_BAD_EXPERT / MOE_ERR_CAPACITY directly (no handle is returned then).
+ */
+int moe_layout(const moe_params_t* params, const int64_t* topk_idx, const float* topk_weights,
+               void* stream, moe_handle_t** out_handle, int32_t* host_rows_per_rank);
+
+/*
+ * Dispatch ("From DeepEP to Mega MoE" 2.2 dispatch warps and 2.4 copy epilogue; "Why MoE gets
+ * stuck on communication" 1: do_expand, do_zero_padding; FP8 per "DeepEP expert-parallel
+ * communication", key techniques).
+ *   x             bf16 [T, H], device.
+ *   out_dtype     MOE_DTYPE_BF16: recv_x is bf16 [R, cap, H], a copy of x[t] per routed row.
+ *                 MOE_DTYPE_FP8_E4M3: recv_x is E4M3 [R, cap, H]; for each 1x128 block,
+ *                 a = max(amax, 1e-4), code = E4M3_rne_satfinite(x * (448 / a)) and
+ *                 recv_scales[r, row, b] = a / 448 (fp32 [R, cap, H/128]).
+ *   recv_weights  fp32 [R, cap], nullable: the pair's topk weight (0 on padding rows).
+ *   cap           rows per logical rank in recv_x / recv_scales / recv_weights.
+ *   do_expand     must be 1 (one row per (token, expert)); 0 returns MOE_ERR_UNSUPPORTED.
+ *   do_zero_padding  1: padding rows are written as zero bytes (codes, scales and bf16).
+ *   num_sms       SMs the kernel may occupy (0 = all).
+ * Rows beyond rows_per_rank[r] are never written.
+ */
+int moe_dispatch(const moe_handle_t* handle, const void* x, int out_dtype, void* recv_x,
+                 float* recv_scales, float* recv_weights, int64_t cap, int do_expand,
+                 int do_zero_padding, int num_sms, void* stream);
+
+/*
+ * Combine ("From DeepEP to Mega MoE" 2.3 and 2.5: element-wise top-k reduction; "Why MoE gets
+ * stuck on communication" 1: already-weighted rows, shared-expert output as bias).
+ *   y             bf16 [R, cap, H], device: the expert outputs in the dispatch layout.
+ *   topk_weights  fp32 [T, k], nullable.  NULL: y rows are already weighted and are summed.
+ *   bias          bf16 [T, H], nullable.
+ *   out           bf16 [T, H].
+ * For each element: acc = 0 (fp32); for j = 0..k-1 with a valid slot, acc = fma(w, y, acc)
+ * (or acc + y); then acc + bias; out = bf16 round-to-nearest-even(acc).
+ */
+int moe_combine(const moe_handle_t* handle, const void* y, const float* topk_weights,
+                const void* bias, void* out, int64_t cap, int num_sms, void* stream);
+
+/* Waits for `stream`, then returns the handle's device status (MOE_OK, MOE_ERR_BAD_EXPERT or
+ * MOE_ERR_CAPACITY) as left by every layout / dispatch / combine ordered before it. */
+int moe_handle_status(const moe_handle_t* handle, void* stream);
+
+/* Device arrays owned by the handle (valid until moe_handle_free). */
+const int32_t* moe_handle_counts(const moe_handle_t* handle);          /* [E] */
+const int32_t* moe_handle_psum(const moe_handle_t* handle);            /* [E] */
+const int32_t* moe_handle_rows_per_rank(const moe_handle_t* handle);   /* [R] */
+const int32_t* moe_handle_tokens_per_rank(const moe_handle_t* handle); /* [R] */
+const uint8_t* moe_handle_token_in_rank(const moe_handle_t* handle);   /* [T, R] */
+const int32_t* moe_handle_slots(const moe_handle_t* handle);           /* [T, k] */
+const int32_t* moe_handle_row_src(const moe_handle_t* handle);         /* [R, row_cap] */
+const float* moe_handle_row_weights(const moe_handle_t* handle);       /* [R, row_cap] */
+int64_t moe_handle_row_capacity(const moe_handle_t* handle);           /* row_cap */
+
+/* Releases the handle.  Its device memory is freed stream-ordered on the layout stream, so
+ * every dispatch / combine that uses the handle must be ordered before this call on that
+ * stream (or already complete).  NULL is accepted. */
+int moe_handle_free(moe_handle_t* handle);
+
+/* Static description of a status code. */
+const char* moe_status_string(int status);
+
+/* Number of kernels launched by this library in this process (all calls, all threads). */
+int64_t moe_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -160,3 +160,11 @@ def worst_case_rows_per_rank(wl: Workload, max_tokens_per_rank: int) -> int:
     may add up to A - 1 padding rows."""
     e_loc = wl.experts_per_rank
     return wl.ranks * max_tokens_per_rank * min(wl.topk, e_loc) + e_loc * (wl.alignment - 1)
+
+
+def gen_y_device(wl: Workload, cap: int, device="cuda") -> torch.Tensor:
+    """Expert outputs y [R, cap, H] drawn on the GPU (for full-size runs where a CPU draw of
+    several GB would dominate): bf16 rounding of N(0, 1) from a seeded CUDA generator."""
+    g = torch.Generator(device=device)
+    g.manual_seed(wl.seed * 1000 + _S_Y)
+    return torch.randn(wl.ranks, cap, wl.hidden, generator=g, device=device).to(torch.bfloat16)
