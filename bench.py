@@ -83,26 +83,39 @@ def hbm_peak():
 
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples (with the GPU's own timestamps) taken while the benchmark runs; the
+    summary keeps the samples inside [start, stop] of the timed region, widened by one sampling
+    period on each side so that short regions still get a sample."""
+    QUERY = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 50
 
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
+        self.out = ""
+        self.t0 = self.t1 = None
 
-    def __enter__(self):
+    def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+        time.sleep(0.5)   # let the sampler come up before the timed region
         return self
 
-    def __exit__(self, *exc):
-        self.out = ""
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_stop(self):
+        self.t1 = time.time()
+
+    def stop(self):
         if self.proc is not None:
+            time.sleep(2 * self.PERIOD_MS / 1000)
             self.proc.terminate()
             try:
                 self.out, _ = self.proc.communicate(timeout=5)
@@ -111,15 +124,27 @@ class ClockSampler:
                 self.out, _ = self.proc.communicate()
 
     def summary(self):
-        rows = [r.split(",") for r in self.out.strip().splitlines() if r.count(",") >= 8]
+        import datetime
+        rows = []
+        for r in self.out.strip().splitlines():
+            f = [c.strip() for c in r.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(f[1]), float(f[2]), f[5:9]))
+            except ValueError:
+                continue
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        pad = self.PERIOD_MS / 1000 * 1.5
+        inside = [r for r in rows if self.t0 is not None and self.t0 - pad <= r[0] <= self.t1 + pad]
+        use = inside or rows
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({names[i] for r in use for i in range(4) if r[3][i] == "Active"})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": reasons, "samples": len(use),
+                "window": "timed region" if inside else "whole run (no sample inside the timed region)"}
 
 
 # --------------------------------------------------------------------------- distributed plumbing
@@ -222,6 +247,45 @@ def run_reference(args) -> int:
     return 0
 
 
+def run_e2e(args, world, dev, stream, step, step_bytes, x, idx, w, y, bias, out, x_c, idx_c, w_c, bias_c):
+    """The same round trip with every step's inputs copied from pinned host memory (x, routing,
+    expert outputs, bias) and the combined output copied back, timed on the device."""
+    x_h = x_c.pin_memory()
+    idx_h, w_h = idx_c.pin_memory(), w_c.pin_memory()
+    y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    y_h.copy_(y)
+    bias_h = bias_c.pin_memory() if bias_c is not None else None
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = x_h.numel() * 2 + idx_h.numel() * 8 + w_h.numel() * 4 + y_h.numel() * 2 + (bias_h.numel() * 2 if bias_h is not None else 0)
+    d2h = out_h.numel() * 2
+
+    def e2e_step():
+        x.copy_(x_h, non_blocking=True)
+        idx.copy_(idx_h, non_blocking=True)
+        w.copy_(w_h, non_blocking=True)
+        y.copy_(y_h, non_blocking=True)
+        if bias_h is not None:
+            bias.copy_(bias_h, non_blocking=True)
+        step(False)
+        out_h.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 10))
+    barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = reduce_max(a.elapsed_time(b), dev) / n
+    return {"value": world * step_bytes / (ms * 1e-3) / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n}
+
+
 # --------------------------------------------------------------------------- our arm
 def run_ours(args) -> int:
     world, rank, local = dist_setup("nccl")
@@ -230,6 +294,8 @@ def run_ours(args) -> int:
     import combine_moe_layout_07_b200 as moe
 
     wl = W.WORKLOADS[args.workload]
+    if args.tokens_per_rank:
+        wl = wl.with_(tokens_per_rank=args.tokens_per_rank)
     stream = torch.cuda.current_stream()
     idx_c, w_c = W.gen_routing(wl)
     x_c = W.gen_x(wl)
@@ -290,6 +356,7 @@ def run_ours(args) -> int:
                 ev[key].append(val)
         moe.moe_handle_free(h)
 
+    clk = ClockSampler(local).start()
     for _ in range(args.warmup):
         step(False)
     torch.cuda.synchronize()
@@ -299,12 +366,14 @@ def run_ours(args) -> int:
     torch.cuda.synchronize()
     launches0 = moe.moe_kernel_launch_count()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        t_start.record(stream)
-        for _ in range(args.steps):
-            step(True)
-        t_end.record(stream)
-        torch.cuda.synchronize()
+    clk.mark_start()
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step(True)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk.mark_stop()
+    clk.stop()
     barrier()
     launches = moe.moe_kernel_launch_count() - launches0
     ms = reduce_max(t_start.elapsed_time(t_end), dev) / args.steps
@@ -314,40 +383,8 @@ def run_ours(args) -> int:
     value = world * step_bytes / (ms * 1e-3) / 1e9
 
     # end to end through the public API: pinned host inputs -> device, round trip, result -> host
-    x_h = x_c.pin_memory()
-    idx_h, w_h = idx_c.pin_memory(), w_c.pin_memory()
-    y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    y_h.copy_(y)
-    bias_h = bias_c.pin_memory() if bias_c is not None else None
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = x_h.numel() * 2 + idx_h.numel() * 8 + w_h.numel() * 4 + y_h.numel() * 2 + (bias_h.numel() * 2 if bias_h is not None else 0)
-    d2h = out_h.numel() * 2
-
-    def e2e_step():
-        x.copy_(x_h, non_blocking=True)
-        idx.copy_(idx_h, non_blocking=True)
-        w.copy_(w_h, non_blocking=True)
-        y.copy_(y_h, non_blocking=True)
-        if bias_h is not None:
-            bias.copy_(bias_h, non_blocking=True)
-        step(False)
-        out_h.copy_(out, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize()
-    e2e_steps = max(3, min(args.steps, 10))
-    barrier()
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    b.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = reduce_max(a.elapsed_time(b), dev) / e2e_steps
-    e2e_value = world * step_bytes / (e2e_ms * 1e-3) / 1e9
-
+    e2e = None if args.no_e2e else run_e2e(args, world, dev, stream, step, step_bytes, x, idx, w, y, bias, out,
+                                           x_c, idx_c, w_c, bias_c)
     peak, peak_kind = hbm_peak()
     kern = {"dispatch": (dispatch_ms, nb["dispatch"]), "combine": (combine_ms, nb["combine"])}
     dom = max(kern, key=lambda k: kern[k][0])
@@ -378,8 +415,7 @@ def run_ours(args) -> int:
                 "A_pad": (valid_pairs + pad_rows) / max(valid_pairs, 1),
                 "rows_per_rank_max_over_mean": float(rows.max() / max(rows.mean(), 1e-9)),
                 "roofline": roofline, "cpu_baseline": cpu,
-                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                        "ms_per_step": e2e_ms},
+                "e2e": e2e,
                 "gpu_launches": launches, "clocks": clk.summary(),
                 "library": os.path.relpath(moe.library_path(), ROOT)}
         print(json.dumps(line), flush=True)
@@ -392,13 +428,16 @@ def run_ours(args) -> int:
 def main() -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default="deepseek")
     ap.add_argument("--cpu-tokens", type=int, default=16384, help="tokens in the CPU-oracle baseline sample")
     ap.add_argument("--ref-tokens", type=int, default=4096, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--tokens-per-rank", type=int, default=0, help="override the workload's tokens per rank "
+                    "(smaller cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -117,7 +117,7 @@ class _DeviceView:
 
     def __init__(self, ptr: int, shape, typestr: str):
         self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
-                                         "data": (ptr, True), "version": 3, "strides": None}
+                                         "data": (ptr, False), "version": 3, "strides": None}
 
 
 class Handle:

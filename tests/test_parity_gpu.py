@@ -264,10 +264,11 @@ def test_determinism_three_runs():
     wl = W.WORKLOADS["tiny"].with_(fp8=True, hidden=2048, tokens_per_rank=1000, experts=64, ranks=4, topk=6)
     idx, w, x = inputs(wl)
     outs = []
+    cap = int(oracle.layout(idx.numpy(), w.numpy(), wl.experts, wl.ranks, wl.alignment).rows_per_rank.max())
     for _ in range(3):
-        h = gpu_layout(wl, idx, w, cap=6000)
-        recv = torch.zeros(wl.ranks, 6000, wl.hidden, dtype=torch.uint8, device="cuda")
-        sc = torch.zeros(wl.ranks, 6000, wl.hidden // 128, device="cuda")
+        h = gpu_layout(wl, idx, w, cap=cap)
+        recv = torch.zeros(wl.ranks, cap, wl.hidden, dtype=torch.uint8, device="cuda")
+        sc = torch.zeros(wl.ranks, cap, wl.hidden // 128, device="cuda")
         moe.moe_dispatch(h, x.cuda(), moe.MOE_DTYPE_FP8_E4M3, recv, sc)
         outs.append((h.slots().cpu(), recv.cpu(), sc.cpu()))
     for o in outs[1:]:
