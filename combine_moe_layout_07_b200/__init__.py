@@ -23,6 +23,7 @@ MOE_ERR_CAPACITY = -3
 MOE_ERR_CUDA = -4
 MOE_ERR_OOM = -5
 MOE_ERR_UNSUPPORTED = -6
+MOE_ERR_SCRATCH_LIMIT = -7
 MOE_DTYPE_BF16 = 0
 MOE_DTYPE_FP8_E4M3 = 1
 
@@ -220,3 +221,21 @@ def moe_handle_free(handle: Handle) -> None:
 
 def moe_kernel_launch_count() -> int:
     return int(lib().moe_kernel_launch_count())
+
+
+def moe_layout_static_scratch(p: MoeParams, topk_idx: torch.Tensor, topk_weights: Optional[torch.Tensor],
+                              counts: torch.Tensor, psum: torch.Tensor, rows_per_rank: torch.Tensor,
+                              tokens_per_rank: torch.Tensor, token_in_rank: torch.Tensor, slots: torch.Tensor,
+                              row_src: torch.Tensor, row_weights: torch.Tensor,
+                              device_status: Optional[torch.Tensor] = None, stream=None) -> Optional[np.ndarray]:
+    """The layout into caller-owned buffers, with no allocation by the library (see the C header).
+    Returns the host row counts when ``p.do_cpu_sync`` is set."""
+    L = lib()
+    f = L.moe_layout_static_scratch
+    f.argtypes = [ctypes.POINTER(MoeParams)] + [_P] * 13
+    rows = np.zeros(p.num_logical_ranks, np.int32) if p.do_cpu_sync else None
+    rc = f(ctypes.byref(p), _ptr(topk_idx), _ptr(topk_weights), _ptr(counts), _ptr(psum), _ptr(rows_per_rank),
+           _ptr(tokens_per_rank), _ptr(token_in_rank), _ptr(slots), _ptr(row_src), _ptr(row_weights),
+           _ptr(device_status), None if rows is None else rows.ctypes.data_as(_P), _stream(stream))
+    _check(rc, "moe_layout_static_scratch")
+    return rows

@@ -375,6 +375,7 @@ const char* moe_status_string(int status) {
     case MOE_ERR_CUDA: return "CUDA runtime error";
     case MOE_ERR_OOM: return "device memory allocation failed";
     case MOE_ERR_UNSUPPORTED: return "unsupported by this build";
+    case MOE_ERR_SCRATCH_LIMIT: return "problem needs more scratch than MOE_STATIC_SCRATCH_BYTES";
     default: return "unknown status";
   }
 }

@@ -54,7 +54,9 @@ enum moe_status_code {
   MOE_ERR_CAPACITY = -3,    /* some logical rank needs more rows than the given capacity */
   MOE_ERR_CUDA = -4,        /* a CUDA runtime call failed */
   MOE_ERR_OOM = -5,         /* the handle's device memory could not be allocated */
-  MOE_ERR_UNSUPPORTED = -6  /* a valid request outside what this build implements */
+  MOE_ERR_UNSUPPORTED = -6, /* a valid request outside what this build implements */
+  MOE_ERR_SCRATCH_LIMIT = -7 /* moe_layout_static_scratch: the problem needs more scratch than
+                                MOE_STATIC_SCRATCH_BYTES */
 };
 
 enum moe_dtype { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_E4M3 = 1 };
@@ -154,6 +156,40 @@ int moe_handle_free(moe_handle_t* handle);
 
 /* Static description of a status code. */
 const char* moe_status_string(int status);
+
+/*
+ * moe_layout_static_scratch -- the layout of moe_layout without any memory allocation.
+ * The pages have no counterpart: this entry point exists for callers that cannot call
+ * cudaMalloc -- code whose device memory is owned by another allocator (a framework caching
+ * allocator that has reserved the GPU, a runtime that hands out fixed arenas) and serving loops
+ * that forbid allocation calls on their hot path, where a driver allocation may block.
+ *
+ * Computes exactly what moe_layout computes, into caller-owned device buffers:
+ *   counts[E], psum[E], rows_per_rank[R], tokens_per_rank[R], token_in_rank[T, R] (uint8),
+ *   slots[T, k], row_src[R, cap] and row_weights[R, cap] with cap = recv_capacity_rows (>= 1).
+ * Its temporaries (status word, padding prefix, per-chunk counts, per-pair rank and weight)
+ * live in one file-scope device array of MOE_STATIC_SCRATCH_BYTES, which every GPU that loads
+ * the library holds until the process exits.  It needs
+ *   256 + r(4(E+1)) + r(4*C*E) + r(4*C*R) + 2*r(4*T*k) bytes, C = ceil(T/512), r = round up to 256;
+ * larger problems return MOE_ERR_SCRATCH_LIMIT before any GPU work.
+ *   device_status  int32, device, nullable: receives the device status flags of this call
+ *                  (bit 0: an expert id outside [-1, E); bit 1: a rank needs more than cap rows);
+ *                  cleared by the call.  NULL: the flags stay in the scratch array.
+ *   host_rows_per_rank  int32 [R], host, nullable: filled when do_cpu_sync = 1.
+ * With do_cpu_sync = 1 the call waits for the counts and returns MOE_ERR_BAD_EXPERT /
+ * MOE_ERR_CAPACITY directly; with 0 it returns after launching.
+ * All calls share the scratch array and it keeps the last call's contents: calls whose GPU
+ * work overlaps on the same device (two streams, two host threads) race.  The first call on a
+ * device looks up the array's device address with that device current; make that first call
+ * before any stream capture.  Calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define MOE_STATIC_SCRATCH_BYTES (4u << 20)
+int moe_layout_static_scratch(const moe_params_t* params, const int64_t* topk_idx,
+                              const float* topk_weights, int32_t* counts, int32_t* psum,
+                              int32_t* rows_per_rank, int32_t* tokens_per_rank,
+                              uint8_t* token_in_rank, int32_t* slots, int32_t* row_src,
+                              float* row_weights, int32_t* device_status,
+                              int32_t* host_rows_per_rank, void* stream);
 
 /* Number of kernels launched by this library in this process (all calls, all threads). */
 int64_t moe_kernel_launch_count(void);
