@@ -24,6 +24,7 @@ MOE_ERR_CUDA = -4
 MOE_ERR_OOM = -5
 MOE_ERR_UNSUPPORTED = -6
 MOE_ERR_SCRATCH_LIMIT = -7
+MOE_ERR_TIMEOUT = -8
 MOE_DTYPE_BF16 = 0
 MOE_DTYPE_FP8_E4M3 = 1
 
@@ -65,7 +66,7 @@ def lib() -> ctypes.CDLL:
     """Load (building first if the sources are newer) the in-tree CUDA library."""
     global _lib
     if _lib is None:
-        path = _build.build()
+        path = _build.build(debug=os.environ.get("MOE_B200_DEBUG") == "1")
         L = ctypes.CDLL(path)
         PP = ctypes.POINTER(MoeParams)
         L.moe_recv_capacity_hint.argtypes = [PP, _I64]
@@ -91,7 +92,7 @@ def lib() -> ctypes.CDLL:
 
 
 def library_path() -> str:
-    return _build.LIB
+    return _build.DEBUG_LIB if os.environ.get("MOE_B200_DEBUG") == "1" else _build.LIB
 
 
 def status_string(status: int) -> str:

@@ -1,117 +1,303 @@
 // combine.cu -- gather the expert outputs back to token order and reduce the top-k rows.
 //
 // Follows "From DeepEP to Mega MoE" (backyes.github.io) 2.3 / 2.5 (combine_reduce: an
-// element-wise sum of a token's top-k expert rows, not a GEMM) and "Why MoE gets stuck on
-// communication" (locsic.com) section 1 (the rows are already weighted; the shared expert's
-// output is added as the bias).  Optional per-pair weights are applied in fp32 when given.
+// element-wise sum of a token's top-k expert rows, not a GEMM; rows arrive by 1-D TMA loads) and
+// "Why MoE gets stuck on communication" (locsic.com) section 1 (the rows are already weighted;
+// the shared expert's output is added as the bias).  Optional per-pair weights are applied in
+// fp32 when given.
 //
 // Numerics, fixed so every run is bit-identical: acc = 0 (fp32); for j = 0..k-1 in order,
 // skipping masked pairs, acc = fma(w, y, acc) or acc + y; then acc + bias; one rounding to bf16.
 //
-// B200 mapping: HBM-bound gather.  One 1024-thread CTA per SM, a warp per token; each lane owns
-// 8 bf16 columns per step and issues the loads of all (up to 8) source rows before reducing
-// them, so 8 x 16 bytes per lane are in flight; streaming loads skip L1, the output row is
-// written with evict-first stores.
+// B200 mapping (HBM-bound gather, one CTA per SM so num_sms caps SMs).  A work item is one token
+// and one column chunk of CW elements (CW <= 2048, chosen so that several stages fit):
+//   warp 0      producer: reads the token's k (rank, slot) pairs from the handle and issues one
+//               cp.async.bulk load per valid source row segment (plus the bias segment) into a
+//               stage of a shared-memory ring, completed on the stage's mbarrier;
+//   warps 1..16 two consumer groups of 8 warps take alternate items; each thread owns 8
+//               columns; it reads the k staged segments in j order from shared memory,
+//               accumulates in fp32 registers, adds the bias, rounds and writes 16 bytes of the
+//               output row with an evict-first store; each warp releases the stage when done.
+// Stage index, phase and (token, chunk) advance as counters (no integer division in the loops).
+// All waits are mbarrier try_waits bounded by wall-clock time; there are no named barriers.
 #include "moe_internal.cuh"
 
 namespace moe {
 
-constexpr int kCombineWarps = kMoveThreads / 32;
-constexpr int kGroup = 8;  // source rows loaded before they are reduced
+constexpr int kCombGroups = 2;         // consumer groups reduce alternate items concurrently
+constexpr int kCombGroupWarps = 8;     // warps per consumer group
+constexpr int kCombConsumerWarps = kCombGroups * kCombGroupWarps;
+constexpr int kCombGroupThreads = 32 * kCombGroupWarps;
+constexpr int kCombConsumers = 32 * kCombConsumerWarps;
+constexpr int kCombThreads = 32 + kCombConsumers;
+constexpr int kCombMaxStages = 8;
+constexpr uint32_t kCombSmemBudget = 200 * 1024;
+
+struct CombMeta {
+  float w[kMaxTopk];  // weights of the valid pairs in j order (weighted combine)
+  int32_t n;          // valid pairs
+  int32_t pad_[3];
+};
+
+struct CombGeom {
+  int64_t cw;        // chunk width in elements (multiple of 8)
+  int64_t nch;       // chunks per token
+  int slots;         // staged rows per item: k (+1 for the bias)
+  int stages;
+  uint32_t full, empty, meta, data, stage_bytes, total;
+};
+
+__host__ __device__ inline uint32_t cround(uint32_t n, uint32_t a) { return (n + a - 1) / a * a; }
+
+__host__ __device__ inline CombGeom comb_geom(int64_t H, int k, bool bias, int stages, int64_t nch) {
+  CombGeom g;
+  g.cw = ((H + nch - 1) / nch + 7) / 8 * 8;
+  g.nch = (H + g.cw - 1) / g.cw;  // every chunk starts inside the row
+  g.slots = k + (bias ? 1 : 0);
+  g.stages = stages;
+  g.stage_bytes = (uint32_t)(g.slots * g.cw * 2);
+  uint32_t off = 0;
+  g.full = off;
+  off += 8 * stages;
+  g.empty = off;
+  off += 8 * stages;
+  off = cround(off, 16);
+  g.meta = off;
+  off += (uint32_t)sizeof(CombMeta) * stages;
+  off = cround(off, 128);
+  g.data = off;
+  off += g.stage_bytes * stages;
+  g.total = off;
+  return g;
+}
+
+// Chunks as wide as possible (<= 2048 columns) while at least 4 stages fit (2 for huge k).
+// The stage count is a multiple of the consumer-group count: stage s is then always consumed
+// by group s % G, which observes every phase of its stages in order (a parity wait can only
+// tell the current phase from the one before it).
+CombGeom combine_geometry(int64_t H, int k, bool bias) {
+  static_assert(kCombMaxStages % kCombGroups == 0 && 4 % kCombGroups == 0, "stages per group");
+  int64_t nch = (H + 2047) / 2048;
+  for (;;) {
+    for (int s = kCombMaxStages; s >= 4; s -= kCombGroups) {
+      const CombGeom g = comb_geom(H, k, bias, s, nch);
+      if (g.total <= kCombSmemBudget) return g;
+    }
+    if (comb_geom(H, k, bias, 4, nch).cw <= 8) break;
+    ++nch;
+  }
+  CombGeom g = comb_geom(H, k, bias, kCombGroups, nch);
+  if (g.total > kCombSmemBudget) g.stages = 0;
+  return g;
+}
 
 template <bool kWeighted, bool kBias>
-__global__ void __launch_bounds__(kMoveThreads, 1) k_combine(CombineLaunch L) {
-  __shared__ int64_t tab_off[kCombineWarps][kMaxTopk];  // element offset of the source row
-  __shared__ float tab_w[kCombineWarps][kMaxTopk];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t gw = (int64_t)blockIdx.x * kCombineWarps + warp;
-  const int64_t nw = (int64_t)gridDim.x * kCombineWarps;
+__global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, CombGeom g) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t base = smem_u32(smem);
+  const uint32_t full0 = base + g.full, empty0 = base + g.empty;
+  CombMeta* meta = reinterpret_cast<CombMeta*>(smem + g.meta);
+  const int S = g.stages;
   const int64_t H = L.H;
   const uint16_t* y = static_cast<const uint16_t*>(L.y);
   const uint16_t* bias = static_cast<const uint16_t*>(L.bias);
   uint16_t* out = static_cast<uint16_t*>(L.out);
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, kCombGroupWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  int64_t t_begin, t_end;
+  cta_token_range(L.T, t_begin, t_end);
+  const int64_t n_items = (t_end - t_begin) * g.nch;
   bool overflow = false;
 
-  for (int64_t t = gw; t < L.T; t += nw) {
-    int64_t off = -1;
-    float wv = 0.0f;
-    if (lane < L.k) {
-      const int64_t p = t * L.k + lane;
-      const int32_t r = __ldg(L.pair_rank + p);
-      const int32_t s = __ldg(L.slot + p);
-      if (r >= 0) {
-        if (s < L.cap) off = ((int64_t)r * L.cap + s) * H;
-        else overflow = true;
-      }
-      if (kWeighted) wv = __ldg(L.w + p);
-    }
-    const uint32_t vmask = __ballot_sync(0xffffffffu, off >= 0);
-    tab_off[warp][lane] = off;
-    tab_w[warp][lane] = wv;
-    __syncwarp();
-
-    for (int64_t c = lane * 8; c < H; c += 32 * 8) {
-      float acc[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-      for (uint32_t m = vmask; m;) {
-        uint4 d[kGroup];
-        float wg[kGroup];
-        int n = 0;
-#pragma unroll
-        for (int g = 0; g < kGroup; ++g) {
-          if (m) {
-            const int j = __ffs(m) - 1;
-            m &= m - 1;
-            d[g] = ld_stream_v4(y + tab_off[warp][j] + c);
-            wg[g] = tab_w[warp][j];
-            n = g + 1;
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    const int tpb = 32 / L.k, lanes_used = tpb * L.k;
+    const int64_t p_end = t_end * L.k;
+    const uint32_t slot_bytes = (uint32_t)(g.cw * 2);
+    PairBatch cur = load_pair_batch(L.pair_rank, L.slot, kWeighted ? L.w : nullptr, t_begin * L.k, p_end, lane,
+                                    lanes_used);
+    int64_t i = 0;
+    int s = 0;
+    uint32_t par = 0;  // parity of the stage's current use: (i / S) & 1
+    bool stop = false;
+    for (int64_t tb = t_begin; tb < t_end && !stop; tb += tpb) {
+      const PairBatch nxt = load_pair_batch(L.pair_rank, L.slot, kWeighted ? L.w : nullptr, (tb + tpb) * L.k,
+                                            p_end, lane, lanes_used);
+      const int nt = (int)min((int64_t)tpb, t_end - tb);
+      for (int q = 0; q < nt && !stop; ++q) {
+        const int64_t t = tb + q;
+        int64_t src = -1;
+        if (lane >= q * L.k && lane < (q + 1) * L.k && cur.rank >= 0) {
+          if (cur.slot < L.cap) src = ((int64_t)cur.rank * L.cap + cur.slot) * H;
+          else overflow = true;
+        }
+        const uint32_t m = __ballot_sync(0xffffffffu, src >= 0);
+        const int pos = __popc(m & lanemask_lt());
+        const int n = __popc(m);
+        for (int64_t c0 = 0; c0 < H; c0 += g.cw) {
+          const uint32_t bytes = (uint32_t)(min(g.cw, H - c0) * 2);
+          if (i >= S) {
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(empty0 + 8 * s, par ^ 1u, L.status);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) {
+              stop = true;
+              break;
+            }
+          }
+          if (kWeighted && src >= 0) meta[s].w[pos] = cur.w;
+          if (lane == 0) meta[s].n = n;
+          __syncwarp();
+          const uint32_t stage = base + g.data + (uint32_t)s * g.stage_bytes;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(full0 + 8 * s, bytes * (uint32_t)(n + (kBias ? 1 : 0)));
+            if (kBias && dbg_ok(t * H + c0 + bytes / 2 <= L.T * H, L.status, 101, t))
+              bulk_load(stage + (uint32_t)L.k * slot_bytes, bias + t * H + c0, bytes, full0 + 8 * s);
+          }
+          __syncwarp();
+          if (src >= 0 && dbg_ok(src + c0 + bytes / 2 <= L.R * L.cap * H && pos < L.k &&
+                                     g.data + (uint32_t)s * g.stage_bytes + (uint32_t)pos * slot_bytes + bytes <= g.total,
+                                 L.status, 102, src))
+            bulk_load(stage + (uint32_t)pos * slot_bytes, y + src + c0, bytes, full0 + 8 * s);
+          __syncwarp();
+          ++i;
+          if (++s == S) {
+            s = 0;
+            par ^= 1u;
           }
         }
+      }
+      cur = nxt;
+    }
+    // no load of this CTA may still be in flight when it exits: wait for the last S items
+    if (lane == 0) {
+      int ss = s;
+      uint32_t pp = par;
+      for (int64_t j = 0; j < min(i, (int64_t)S); ++j) {
+        if (--ss < 0) {
+          ss = S - 1;
+          pp ^= 1u;
+        }
+        mbar_wait(full0 + 8 * ss, pp, L.status);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- consumer groups
+    const int cwarp = warp - 1;
+    const int grp = cwarp / kCombGroupWarps;
+    const int gtid = tid - 32 - grp * kCombGroupThreads;
+    const uint32_t slot_bytes = (uint32_t)(g.cw * 2);
+    // item i = (t - t_begin) * nch + chunk; this group takes i = grp, grp + G, ...
+    int64_t i = grp, t = t_begin, c = grp;
+    while (c >= g.nch) {
+      c -= g.nch;
+      ++t;
+    }
+    int s = grp % S;
+    uint32_t par = (uint32_t)((grp / S) & 1);
+    for (; i < n_items; i += kCombGroups) {
+      const int64_t c0 = c * g.cw;
+      const int64_t width = min(g.cw, H - c0);
+      if (!mbar_wait_warp(full0 + 8 * s, par, L.status)) break;
+      const int n = meta[s].n;
+      if (!dbg_ok(n >= 0 && n <= L.k, L.status, 104, n)) break;
+      const uint32_t stage = base + g.data + (uint32_t)s * g.stage_bytes;
+      for (int64_t e = gtid * 8; e < width; e += kCombGroupThreads * 8) {
+        float acc[8];
 #pragma unroll
-        for (int g = 0; g < kGroup; ++g) {
-          if (g < n) {
-            const uint32_t u[4] = {d[g].x, d[g].y, d[g].z, d[g].w};
+        for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+        int j = 0;
+        for (; j + 4 <= n; j += 4) {
+          uint4 d[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+          for (int u = 0; u < 4; ++u) d[u] = lds_v4(stage + (uint32_t)(j + u) * slot_bytes + (uint32_t)e * 2);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t wd[4] = {d[u].x, d[u].y, d[u].z, d[u].w};
+            const float wj = kWeighted ? meta[s].w[j + u] : 1.0f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
               if (kWeighted) {
-                acc[2 * i] = __fmaf_rn(wg[g], bf16lo(u[i]), acc[2 * i]);
-                acc[2 * i + 1] = __fmaf_rn(wg[g], bf16hi(u[i]), acc[2 * i + 1]);
+                acc[2 * q] = __fmaf_rn(wj, bf16lo(wd[q]), acc[2 * q]);
+                acc[2 * q + 1] = __fmaf_rn(wj, bf16hi(wd[q]), acc[2 * q + 1]);
               } else {
-                acc[2 * i] = __fadd_rn(acc[2 * i], bf16lo(u[i]));
-                acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], bf16hi(u[i]));
+                acc[2 * q] = __fadd_rn(acc[2 * q], bf16lo(wd[q]));
+                acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16hi(wd[q]));
               }
             }
           }
         }
-      }
-      if (kBias) {
-        const uint4 b = ld_stream_v4(bias + t * H + c);
-        const uint32_t u[4] = {b.x, b.y, b.z, b.w};
+        for (; j < n; ++j) {
+          const uint4 d = lds_v4(stage + (uint32_t)j * slot_bytes + (uint32_t)e * 2);
+          const uint32_t wd[4] = {d.x, d.y, d.z, d.w};
+          const float wj = kWeighted ? meta[s].w[j] : 1.0f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[2 * i] = __fadd_rn(acc[2 * i], bf16lo(u[i]));
-          acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], bf16hi(u[i]));
+          for (int q = 0; q < 4; ++q) {
+            if (kWeighted) {
+              acc[2 * q] = __fmaf_rn(wj, bf16lo(wd[q]), acc[2 * q]);
+              acc[2 * q + 1] = __fmaf_rn(wj, bf16hi(wd[q]), acc[2 * q + 1]);
+            } else {
+              acc[2 * q] = __fadd_rn(acc[2 * q], bf16lo(wd[q]));
+              acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16hi(wd[q]));
+            }
+          }
         }
+        if (kBias) {
+          const uint4 b = lds_v4(stage + (uint32_t)L.k * slot_bytes + (uint32_t)e * 2);
+          const uint32_t wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[2 * q] = __fadd_rn(acc[2 * q], bf16lo(wb[q]));
+            acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16hi(wb[q]));
+          }
+        }
+        if (!dbg_ok(t >= t_begin && t < t_end && c0 + e + 8 <= H && n <= L.k &&
+                        g.data + (uint32_t)s * g.stage_bytes + (uint32_t)(n > 0 ? n - 1 : 0) * slot_bytes +
+                                (uint32_t)e * 2 + 16 <= g.total,
+                    L.status, 103, t * 65536 + e))
+          continue;
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        st_stream_v4(out + t * H + c0 + e, o);
       }
-      uint4 o;
-      o.x = pack_bf16x2(acc[0], acc[1]);
-      o.y = pack_bf16x2(acc[2], acc[3]);
-      o.z = pack_bf16x2(acc[4], acc[5]);
-      o.w = pack_bf16x2(acc[6], acc[7]);
-      st_stream_v4(out + t * H + c, o);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * s);
+      // advance to item i + G
+      c += kCombGroups;
+      while (c >= g.nch) {
+        c -= g.nch;
+        ++t;
+      }
+      s += kCombGroups;
+      while (s >= S) {
+        s -= S;
+        par ^= 1u;
+      }
     }
-    __syncwarp();
   }
   if (overflow) atomicOr(L.status, kStatusCapacity);
 }
 
-cudaError_t launch_combine(const CombineLaunch& L, cudaStream_t s) {
-  const bool wgt = L.w != nullptr, bias = L.bias != nullptr;
-  if (wgt && bias) k_combine<true, true><<<L.grid, kMoveThreads, 0, s>>>(L);
-  else if (wgt) k_combine<true, false><<<L.grid, kMoveThreads, 0, s>>>(L);
-  else if (bias) k_combine<false, true><<<L.grid, kMoveThreads, 0, s>>>(L);
-  else k_combine<false, false><<<L.grid, kMoveThreads, 0, s>>>(L);
+cudaError_t launch_combine(const CombineLaunch& L, cudaStream_t st) {
+  const bool wgt = L.w != nullptr, has_bias = L.bias != nullptr;
+  const CombGeom g = combine_geometry(L.H, L.k, has_bias);
+  if (g.stages < kCombGroups || g.stages % kCombGroups != 0) return cudaErrorInvalidValue;
+  auto kern = wgt ? (has_bias ? k_combine<true, true> : k_combine<true, false>)
+                  : (has_bias ? k_combine<false, true> : k_combine<false, false>);
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCombSmemBudget);
+  if (err != cudaSuccess) return err;
+  kern<<<L.grid, kCombThreads, g.total, st>>>(L, g);
   note_launch();
   return cudaGetLastError();
 }

@@ -7,6 +7,7 @@
 // dispatch-combine" (phantomic12.github.io): with it, the counts are copied to the host and
 // the call waits; without it, nothing waits and consumers read the device-side psum.
 #include <atomic>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -297,6 +298,7 @@ int moe_dispatch(const moe_handle_t* h, const void* x, int out_dtype, void* recv
   L.E = p.num_experts;
   L.E_loc = p.num_experts / p.num_logical_ranks;
   L.zero_padding = do_zero_padding;
+  L.R = p.num_logical_ranks;
   L.grid = grid_for(num_sms, h->device);
   L.pair_rank = h->d.pair_rank;
   L.slot = h->d.slot;
@@ -328,6 +330,7 @@ int moe_combine(const moe_handle_t* h, const void* y, const float* topk_weights,
   L.cap = cap;
   L.H = p.hidden;
   L.k = p.topk;
+  L.R = p.num_logical_ranks;
   L.grid = grid_for(num_sms, h->device);
   L.pair_rank = h->d.pair_rank;
   L.slot = h->d.slot;
@@ -340,8 +343,14 @@ int moe_handle_status(const moe_handle_t* h, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* stage = static_cast<int32_t*>(g_stage.get(16));
   if (!stage) return MOE_ERR_CUDA;
-  if (cudaMemcpyAsync(stage, h->d.status, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpyAsync(stage, h->d.status, 16, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (stage[0] & kStatusBounds) {
+    std::fprintf(stderr, "moe: index check %d failed, detail %lld\n", stage[1],
+                 (long long)(((uint64_t)(uint32_t)stage[3] << 32) | (uint32_t)stage[2]));
+    return MOE_ERR_CUDA;
+  }
+  if (stage[0] & kStatusTimeout) return MOE_ERR_TIMEOUT;
   if (stage[0] & kStatusBadExpert) return MOE_ERR_BAD_EXPERT;
   if (stage[0] & kStatusCapacity) return MOE_ERR_CAPACITY;
   return MOE_OK;
@@ -375,6 +384,7 @@ const char* moe_status_string(int status) {
     case MOE_ERR_CUDA: return "CUDA runtime error";
     case MOE_ERR_OOM: return "device memory allocation failed";
     case MOE_ERR_UNSUPPORTED: return "unsupported by this build";
+    case MOE_ERR_TIMEOUT: return "a kernel gave up waiting on a shared-memory barrier (internal error)";
     case MOE_ERR_SCRATCH_LIMIT: return "problem needs more scratch than MOE_STATIC_SCRATCH_BYTES";
     default: return "unknown status";
   }

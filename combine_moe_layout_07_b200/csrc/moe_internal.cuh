@@ -13,6 +13,13 @@ namespace moe {
 // Device status word bits (the handle's status[0]).
 constexpr int32_t kStatusBadExpert = 1;
 constexpr int32_t kStatusCapacity = 2;
+constexpr int32_t kStatusBounds = 8;  // MOE_DEBUG builds: an index check failed (details in status[1..3])
+
+#ifdef MOE_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
 
 // Layout tiling: a chunk of tokens per CTA; 8 warps per layout CTA.
 constexpr int kChunkTokens = 512;
@@ -81,6 +88,7 @@ struct DispatchLaunch {
   float* recv_scales;
   float* recv_w;
   int64_t T, cap, H;
+  int64_t R;  // logical ranks (receive buffers hold R * cap rows)
   int k, E, E_loc;
   int zero_padding;
   int grid;
@@ -100,6 +108,7 @@ struct CombineLaunch {
   const void* bias;
   void* out;
   int64_t T, cap, H;
+  int64_t R;  // logical ranks (y holds R * cap rows)
   int k;
   int grid;
   const int32_t* pair_rank;
@@ -146,10 +155,163 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
   return (uint32_t)r;
 }
 
+// MOE_DEBUG builds: returns `cond`; on the first failure records (code, detail) in status[1..3]
+// so the host can report it, and the caller skips the access.  Release builds: always true.
+__device__ __forceinline__ bool dbg_ok(bool cond, int32_t* status, int32_t code, int64_t detail) {
+  if (!kDebugChecks || cond) return true;
+  if ((atomicOr(status, kStatusBounds) & kStatusBounds) == 0) {
+    status[1] = code;
+    status[2] = (int32_t)(detail & 0xffffffff);
+    status[3] = (int32_t)(detail >> 32);
+  }
+  return false;
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
   return m;
+}
+
+}  // namespace moe
+
+// ------------------------------------------------------------------------------ TMA bulk copies
+// 1-D bulk copies (cp.async.bulk) between global and shared memory, completed on an mbarrier
+// (loads) or a bulk-group (stores).  Every address is 16-byte aligned and every size a multiple
+// of 16 bytes; no multicast.
+namespace moe {
+
+constexpr int32_t kStatusTimeout = 4;                  // a bounded wait on an mbarrier gave up
+constexpr uint64_t kWaitLimitNs = 2000000000ull;        // 2 s of wall-clock time per wait
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase of `bar` with the given parity to complete.  Bounded by wall-clock time:
+// after kWaitLimitNs it records kStatusTimeout and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 63) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) break;
+  }
+  atomicOr(status, kStatusTimeout);
+  return false;
+}
+
+// Warp-wide wait: lane 0 waits (bounded), the result is broadcast, and every lane then observes
+// the completed phase itself (acquire).  Call with the whole warp.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, int32_t* status) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status);
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) mbar_try_wait(bar, parity);
+  return ok;
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst_smem),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src_smem), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+}  // namespace moe
+
+// ------------------------------------------------------------------------------ pair metadata
+namespace moe {
+
+// One warp-wide load of the (rank, slot, weight) of up to 32 consecutive (token, j) pairs:
+// lane l holds pair p0 + l (p0 = first token of the batch * k), if it lies before p_end.
+struct PairBatch {
+  int32_t rank, slot;
+  float w;
+};
+
+__device__ __forceinline__ PairBatch load_pair_batch(const int32_t* pair_rank, const int32_t* slot,
+                                                     const float* w, int64_t p0, int64_t p_end, int lane,
+                                                     int lanes_used) {
+  PairBatch b{-1, -1, 0.0f};
+  const int64_t p = p0 + lane;
+  if (lane < lanes_used && p < p_end) {
+    b.rank = __ldg(pair_rank + p);
+    b.slot = __ldg(slot + p);
+    if (w) b.w = __ldg(w + p);
+  }
+  return b;
+}
+
+// The contiguous token range [begin, end) of CTA b out of G (balanced split of T tokens).
+__device__ __forceinline__ void cta_token_range(int64_t T, int64_t& begin, int64_t& end) {
+  begin = T * blockIdx.x / gridDim.x;
+  end = T * (blockIdx.x + 1) / gridDim.x;
 }
 
 }  // namespace moe

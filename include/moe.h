@@ -55,8 +55,10 @@ enum moe_status_code {
   MOE_ERR_CUDA = -4,        /* a CUDA runtime call failed */
   MOE_ERR_OOM = -5,         /* the handle's device memory could not be allocated */
   MOE_ERR_UNSUPPORTED = -6, /* a valid request outside what this build implements */
-  MOE_ERR_SCRATCH_LIMIT = -7 /* moe_layout_static_scratch: the problem needs more scratch than
-                                MOE_STATIC_SCRATCH_BYTES */
+  MOE_ERR_SCRATCH_LIMIT = -7, /* moe_layout_static_scratch: the problem needs more scratch than
+                                 MOE_STATIC_SCRATCH_BYTES */
+  MOE_ERR_TIMEOUT = -8        /* a kernel's bounded wait on one of its own shared-memory barriers
+                                 expired (2 s); reported by moe_handle_status; internal error */
 };
 
 enum moe_dtype { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_E4M3 = 1 };
@@ -134,8 +136,9 @@ int moe_dispatch(const moe_handle_t* handle, const void* x, int out_dtype, void*
 int moe_combine(const moe_handle_t* handle, const void* y, const float* topk_weights,
                 const void* bias, void* out, int64_t cap, int num_sms, void* stream);
 
-/* Waits for `stream`, then returns the handle's device status (MOE_OK, MOE_ERR_BAD_EXPERT or
- * MOE_ERR_CAPACITY) as left by every layout / dispatch / combine ordered before it. */
+/* Waits for `stream`, then returns the handle's device status (MOE_OK, MOE_ERR_BAD_EXPERT,
+ * MOE_ERR_CAPACITY or MOE_ERR_TIMEOUT) as left by every layout / dispatch / combine ordered
+ * before it. */
 int moe_handle_status(const moe_handle_t* handle, void* stream);
 
 /* Device arrays owned by the handle (valid until moe_handle_free). */

@@ -83,5 +83,5 @@ def test_null_and_misaligned_arguments():
 
 
 def test_status_strings():
-    for code in range(-6, 1):
+    for code in range(-8, 1):
         assert moe.status_string(code) and moe.status_string(code) != "unknown status"

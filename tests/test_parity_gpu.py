@@ -72,6 +72,7 @@ def _roundtrip_small(wl, idx, w, x, cap_extra=3, zero_padding=True, weighted=Fal
     got = bits(out)
     assert_bf16_close(got, ref)
     assert (got == ref).all(), f"{(got != ref).sum()} elements differ in the last bit"
+    assert moe.moe_handle_status(h) == moe.MOE_OK
     moe.moe_handle_free(h)
     return lay
 
@@ -87,7 +88,7 @@ def test_tiny_bf16_roundtrip(zero_padding, mask, weighted, with_bias):
     _roundtrip_small(wl, idx, w, x, zero_padding=zero_padding, weighted=weighted, with_bias=with_bias)
 
 
-@pytest.mark.parametrize("hidden", [128, 640, 1024, 2048])
+@pytest.mark.parametrize("hidden", [128, 640, 1024, 2048, 7168])
 @pytest.mark.parametrize("zero_padding", [True, False])
 def test_small_fp8_roundtrip(hidden, zero_padding):
     wl = W.WORKLOADS["tiny"].with_(hidden=hidden, fp8=True, tokens_per_rank=300, experts=16, topk=4)
@@ -107,6 +108,8 @@ def test_small_fp8_roundtrip(hidden, zero_padding):
     dict(hidden=8),                                      # one 16-byte vector per row
     dict(hidden=136),                                    # ragged vector tail in the warp loop
     dict(experts=512, ranks=8, topk=8, tokens_per_rank=700, alignment=128),
+    dict(hidden=7168, tokens_per_rank=300, experts=32, ranks=4, topk=8),   # several column chunks
+    dict(hidden=4104, tokens_per_rank=200, experts=16, ranks=2, topk=3),   # ragged last chunk
 ])
 def test_shapes_and_edges(kw):
     wl = W.WORKLOADS["tiny"].with_(**kw)
@@ -369,3 +372,16 @@ def test_workload_full_size(name):
 
 def test_deepseek_weighted_with_bias():
     _sampled_roundtrip(W.WORKLOADS["deepseek"].with_(weighted_combine=True, bias=True), n_sample=64)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(hidden=7168, topk=8, experts=64, ranks=8, tokens_per_rank=64),    # DeepSeek row shape
+    dict(hidden=7168, topk=8, experts=64, ranks=8, tokens_per_rank=64, fp8=True),
+    dict(hidden=4096, topk=8, experts=128, ranks=16, tokens_per_rank=32),  # skewed row shape
+])
+def test_multi_chunk_rows_plain_combine(kw):
+    """Row shapes whose combine stages hold several column chunks, unweighted and without bias
+    (the stage-ring geometry of the full-size workloads)."""
+    wl = W.WORKLOADS["tiny"].with_(**kw)
+    idx, w, x = inputs(wl)
+    _roundtrip_small(wl, idx, w, x)
