@@ -22,43 +22,73 @@ namespace moe {
 
 __device__ __forceinline__ int32_t align_up_dev(int32_t n, int32_t a) { return ((n + a - 1) / a) * a; }
 
+// Expert id of a routing entry as int32: the id if in [0, E), -1 when masked, -2 when the
+// entry lies outside [-1, E) (an error the count kernel reports).
+__device__ __forceinline__ int32_t expert_of(int64_t e, int E) {
+  return (e >= 0 && e < E) ? (int32_t)e : (e == -1 ? -1 : -2);
+}
+
 // ------------------------------------------------------------------------------------ count
+// A thread per token: its k ids are loaded together, counted into the chunk's shared-memory
+// histogram (atomicAdd_block), and its rank membership is written and counted.
 __global__ void __launch_bounds__(kLayoutThreads) k_layout_count(LayoutLaunch L) {
   extern __shared__ int32_t sm[];
-  int32_t* hist = sm;          // [E]
-  int32_t* tok = sm + L.E;     // [R]
+  int32_t* hist = sm;       // [E]
+  int32_t* tok = sm + L.E;  // [R]
   const int tid = threadIdx.x;
+  bool bad = false;
   for (int c = blockIdx.x; c < L.num_chunks; c += gridDim.x) {
     for (int i = tid; i < L.E + L.R; i += blockDim.x) sm[i] = 0;
     __syncthreads();
     const int64_t t0 = (int64_t)c * kChunkTokens;
     const int64_t t1 = min(L.T, t0 + kChunkTokens);
-    bool bad = false;
-    for (int64_t p = t0 * L.k + tid; p < t1 * L.k; p += blockDim.x) {
-      const int64_t e = L.idx[p];
-      if (e >= 0 && e < L.E) atomicAdd_block(&hist[e], 1);
-      else if (e != -1) bad = true;
-    }
-    // membership: rank r holds token t if one of its k experts lives on r
     for (int64_t t = t0 + tid; t < t1; t += blockDim.x) {
-      uint8_t* row = L.d.token_in_rank + t * L.R;
-      for (int r = 0; r < L.R; ++r) row[r] = 0;
-      for (int j = 0; j < L.k; ++j) {
-        const int64_t e = L.idx[t * L.k + j];
-        if (e < 0 || e >= L.E) continue;
-        const int r = (int)(e / L.E_loc);
-        if (!row[r]) {
-          row[r] = 1;
-          atomicAdd_block(&tok[r], 1);
+      const int64_t* ids = L.idx + t * L.k;
+      int32_t ev[kMaxTopk];
+#pragma unroll
+      for (int j = 0; j < kMaxTopk; ++j) {
+        ev[j] = j < L.k ? expert_of(__ldg(ids + j), L.E) : -1;
+        if (ev[j] == -2) {
+          bad = true;
+          ev[j] = -1;
         }
       }
+      uint8_t* member = L.d.token_in_rank + t * L.R;
+      if (L.R <= 64) {
+        uint64_t mask = 0;
+#pragma unroll
+        for (int j = 0; j < kMaxTopk; ++j)
+          if (ev[j] >= 0) {
+            atomicAdd_block(&hist[ev[j]], 1);
+            mask |= 1ull << (ev[j] / L.E_loc);
+          }
+        for (int r = 0; r < L.R; ++r) member[r] = (uint8_t)((mask >> r) & 1);
+        for (uint64_t m = mask; m; m &= m - 1) atomicAdd_block(&tok[__ffsll((long long)m) - 1], 1);
+      } else {
+        for (int r = 0; r < L.R; ++r) member[r] = 0;
+#pragma unroll
+        for (int j = 0; j < kMaxTopk; ++j)
+          if (ev[j] >= 0) {
+            atomicAdd_block(&hist[ev[j]], 1);
+            const int r = ev[j] / L.E_loc;
+            bool first = true;
+#pragma unroll
+            for (int j2 = 0; j2 < j; ++j2)
+              if (ev[j2] >= 0 && ev[j2] / L.E_loc == r) first = false;
+            if (first) {
+              member[r] = 1;
+              atomicAdd_block(&tok[r], 1);
+            }
+          }
+      }
     }
-    if (bad) atomicOr(L.d.status, kStatusBadExpert);
     __syncthreads();
     for (int e = tid; e < L.E; e += blockDim.x) L.d.chunk_cnt[(int64_t)c * L.E + e] = hist[e];
-    for (int r = tid; r < L.R; r += blockDim.x) L.d.chunk_tok[(int64_t)c * L.R + r] = tok[r];
+    for (int r = tid; r < L.R; r += blockDim.x)
+      if (tok[r]) atomicAdd(L.d.tokens_per_rank + r, tok[r]);  // integer sum: order-free
     __syncthreads();
   }
+  if (bad) atomicOr(L.d.status, kStatusBadExpert);
 }
 
 // Block-wide exclusive scan of one value per thread (warp shuffles + one smem pass).
@@ -90,36 +120,57 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
 }
 
 // ------------------------------------------------------------------------------------ scan
+// One CTA.  (1) per expert, exclusive scan of the chunk counts over chunks, staged through
+// shared memory a tile of rows at a time (coalesced loads and stores); (2) block-wide scans of
+// align_up(cnt, A) and of the padding rows over all experts; (3) psum restarted at every rank.
 __global__ void __launch_bounds__(kScanThreads) k_layout_scan(LayoutLaunch L, int64_t cap_check) {
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t totals[2];
   extern __shared__ int32_t sm[];
-  int32_t* al = sm;              // [E] align_up(cnt, A)
-  int32_t* pad = sm + L.E;       // [E] align_up(cnt, A) - cnt
-  int32_t* gincl = sm + 2 * L.E; // [E] inclusive prefix of al over all experts
-  const int tid = threadIdx.x;
   const int E = L.E;
+  int32_t* al = sm;              // [E] align_up(cnt, A)
+  int32_t* pad = sm + E;         // [E] align_up(cnt, A) - cnt
+  int32_t* gincl = sm + 2 * E;   // [E] inclusive prefix of al over all experts
+  int32_t* run = sm + 3 * E;     // [E] running chunk offset
+  int32_t* tile = sm + 4 * E;    // [rows][E]
+  const int rows = kScanTileInts / E;
+  const int tid = threadIdx.x;
 
-  // 1. per expert: exclusive scan over chunks (in place), total count
-  for (int e = tid; e < E; e += blockDim.x) {
-    int32_t run = 0;
-    for (int c = 0; c < L.num_chunks; ++c) {
-      int32_t* q = L.d.chunk_cnt + (int64_t)c * E + e;
-      const int32_t v = *q;
-      *q = run;
-      run += v;
+  for (int e = tid; e < E; e += blockDim.x) run[e] = 0;
+  __syncthreads();
+  for (int c0 = 0; c0 < L.num_chunks; c0 += rows) {
+    const int nr = min(rows, L.num_chunks - c0);
+    int32_t* g = L.d.chunk_cnt + (int64_t)c0 * E;
+    for (int i = tid; i < nr * E; i += blockDim.x) tile[i] = g[i];
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) {
+      int32_t r = run[e];
+      for (int c = 0; c < nr; ++c) {
+        const int32_t v = tile[c * E + e];
+        tile[c * E + e] = r;
+        r += v;
+      }
+      run[e] = r;
     }
-    L.d.cnt[e] = run;
-    al[e] = align_up_dev(run, L.A);
-    pad[e] = al[e] - run;
+    __syncthreads();
+    for (int i = tid; i < nr * E; i += blockDim.x) g[i] = tile[i];
+    __syncthreads();
+  }
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int32_t n = run[e];
+    L.d.cnt[e] = n;
+    al[e] = align_up_dev(n, L.A);
+    pad[e] = al[e] - n;
   }
   __syncthreads();
 
-  // 2. each thread owns a contiguous run of experts; block scan of the run sums
   const int per = (E + blockDim.x - 1) / blockDim.x;
   const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
   int32_t sa = 0, sp = 0;
-  for (int e = e0; e < e1; ++e) { sa += al[e]; sp += pad[e]; }
+  for (int e = e0; e < e1; ++e) {
+    sa += al[e];
+    sp += pad[e];
+  }
   int32_t ra = block_exclusive_scan(sa, warp_tot, &totals[0]);
   int32_t rp = block_exclusive_scan(sp, warp_tot, &totals[1]);
   for (int e = e0; e < e1; ++e) {
@@ -131,23 +182,27 @@ __global__ void __launch_bounds__(kScanThreads) k_layout_scan(LayoutLaunch L, in
   if (tid == 0) L.d.pad_excl[E] = totals[1];
   __syncthreads();
 
-  // 3. restart at every rank: psum[e] = gincl[e] - (exclusive prefix at the rank's first expert)
   for (int e = tid; e < E; e += blockDim.x) {
     const int first = (e / L.E_loc) * L.E_loc;
     L.d.psum[e] = gincl[e] - (gincl[first] - al[first]);
   }
   for (int r = tid; r < L.R; r += blockDim.x) {
     const int first = r * L.E_loc, last = first + L.E_loc - 1;
-    const int32_t rows = gincl[last] - (gincl[first] - al[first]);
-    L.d.rows_per_rank[r] = rows;
-    if (cap_check > 0 && rows > cap_check) atomicOr(L.d.status, kStatusCapacity);
-    int32_t tk = 0;
-    for (int c = 0; c < L.num_chunks; ++c) tk += L.d.chunk_tok[(int64_t)c * L.R + r];
-    L.d.tokens_per_rank[r] = tk;
+    const int32_t nrows = gincl[last] - (gincl[first] - al[first]);
+    L.d.rows_per_rank[r] = nrows;
+    if (cap_check > 0 && nrows > cap_check) atomicOr(L.d.status, kStatusCapacity);
   }
 }
 
 // ------------------------------------------------------------------------------------ assign
+// A CTA per chunk of tokens, 8 warps; warp w takes a contiguous run of the chunk's (t, j) pairs
+// and loads its expert ids kAssignBatch rounds of 32 at a time.  Phase 1: per-warp histogram
+// (__match_any_sync groups equal ids inside a round; the group leader adds its size).  Phase 2:
+// per expert, exclusive scan across warps based at the expert's first row for this chunk.
+// Phase 3: walk the pairs again; a pair's row = its warp's running base + its rank among equal
+// ids of lower lanes in the round.
+constexpr int kAssignBatch = 8;
+
 __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L) {
   extern __shared__ int32_t whist[];  // [kLayoutWarps][E]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -166,18 +221,23 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L
     // phase 1: this warp's histogram of its pairs
     for (int e = lane; e < E; e += 32) h[e] = 0;
     __syncwarp();
-    for (int64_t base = wp0; base < wp1; base += 32) {
-      const int64_t p = base + lane;
-      const int64_t e = p < wp1 ? L.idx[p] : -1;
-      const bool valid = e >= 0 && e < E;
-      const uint32_t peers = __match_any_sync(0xffffffffu, valid ? (int)e : -1);
-      if (valid && lane == __ffs(peers) - 1) h[e] += __popc(peers);
-      __syncwarp();
+    for (int64_t base = wp0; base < wp1; base += 32 * kAssignBatch) {
+      int32_t ev[kAssignBatch];
+#pragma unroll
+      for (int r = 0; r < kAssignBatch; ++r) {
+        const int64_t p = base + r * 32 + lane;
+        ev[r] = p < wp1 ? max(expert_of(__ldg(L.idx + p), E), -1) : -1;
+      }
+#pragma unroll
+      for (int r = 0; r < kAssignBatch; ++r) {
+        const uint32_t peers = __match_any_sync(0xffffffffu, ev[r]);
+        if (ev[r] >= 0 && lane == __ffs(peers) - 1) h[ev[r]] += __popc(peers);
+        __syncwarp();
+      }
     }
     __syncthreads();
 
-    // phase 2: per expert, exclusive scan across warps, based at the expert's first row for
-    // this chunk (segment start + chunk offset)
+    // phase 2: per expert, exclusive scan across warps
     for (int e = tid; e < E; e += blockDim.x) {
       int32_t base = L.d.psum[e] - align_up_dev(L.d.cnt[e], L.A) + L.d.chunk_cnt[(int64_t)c * E + e];
       for (int w = 0; w < kLayoutWarps; ++w) {
@@ -188,30 +248,38 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L
     }
     __syncthreads();
 
-    // phase 3: walk the pairs again in order; equal experts inside a round are ranked by lane
-    for (int64_t base = wp0; base < wp1; base += 32) {
-      const int64_t p = base + lane;
-      const bool in = p < wp1;
-      const int64_t e = in ? L.idx[p] : -1;
-      const bool valid = in && e >= 0 && e < E;
-      const uint32_t peers = __match_any_sync(0xffffffffu, valid ? (int)e : -1);
-      int32_t row = -1;
-      if (valid) row = h[e] + __popc(peers & lt);
-      __syncwarp();
-      if (valid && lane == __ffs(peers) - 1) h[e] += __popc(peers);
-      __syncwarp();
-      if (in) {
-        const float wv = L.w ? L.w[p] : 0.0f;
-        L.d.slot[p] = row;
-        L.d.pair_rank[p] = valid ? (int32_t)(e / L.E_loc) : -1;
-        L.d.pair_w[p] = wv;
-        if (valid) {
-          const int r = (int)(e / L.E_loc);
-          if (row < L.row_cap) {
-            L.d.row_src[(int64_t)r * L.row_cap + row] = (int32_t)(p / L.k);
-            L.d.row_w[(int64_t)r * L.row_cap + row] = wv;
-          } else {
-            overflow = true;
+    // phase 3: rows in (t, j) order
+    for (int64_t base = wp0; base < wp1; base += 32 * kAssignBatch) {
+      int32_t ev[kAssignBatch];
+      float wv[kAssignBatch];
+#pragma unroll
+      for (int r = 0; r < kAssignBatch; ++r) {
+        const int64_t p = base + r * 32 + lane;
+        ev[r] = p < wp1 ? max(expert_of(__ldg(L.idx + p), E), -1) : -1;
+        wv[r] = (p < wp1 && L.w) ? __ldg(L.w + p) : 0.0f;
+      }
+#pragma unroll
+      for (int r = 0; r < kAssignBatch; ++r) {
+        const int64_t p = base + r * 32 + lane;
+        const int32_t e = ev[r];
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        int32_t row = -1;
+        if (e >= 0) row = h[e] + __popc(peers & lt);
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) h[e] += __popc(peers);
+        __syncwarp();
+        if (p < wp1) {
+          L.d.slot[p] = row;
+          L.d.pair_rank[p] = e >= 0 ? e / L.E_loc : -1;
+          L.d.pair_w[p] = wv[r];
+          if (e >= 0) {
+            const int rk = e / L.E_loc;
+            if (row < L.row_cap) {
+              L.d.row_src[(int64_t)rk * L.row_cap + row] = (int32_t)(p / L.k);
+              L.d.row_w[(int64_t)rk * L.row_cap + row] = wv[r];
+            } else {
+              overflow = true;
+            }
           }
         }
       }
@@ -225,7 +293,8 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L
     int lo = 0, hi = E;  // largest e with pad_excl[e] <= i
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (L.d.pad_excl[mid] <= i) lo = mid; else hi = mid;
+      if (L.d.pad_excl[mid] <= i) lo = mid;
+      else hi = mid;
     }
     const int e = lo;
     const int32_t pad_e = L.d.pad_excl[e + 1] - L.d.pad_excl[e];
@@ -250,7 +319,7 @@ static cudaError_t ensure_smem_attrs() {
   if (err != cudaSuccess) return err;
   if (dev < 64 && (done >> dev) & 1ull) return cudaSuccess;
   err = cudaFuncSetAttribute(k_layout_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(sizeof(int32_t) * 3 * kMaxExperts));
+                             (int)(sizeof(int32_t) * (4 * kMaxExperts + kScanTileInts)));
   if (err == cudaSuccess)
     err = cudaFuncSetAttribute(k_layout_assign, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(sizeof(int32_t) * kLayoutWarps * kMaxExperts));
@@ -269,7 +338,7 @@ cudaError_t launch_layout_count(const LayoutLaunch& L, cudaStream_t s) {
 cudaError_t launch_layout_scan(const LayoutLaunch& L, int64_t cap_check, cudaStream_t s) {
   cudaError_t err = ensure_smem_attrs();
   if (err != cudaSuccess) return err;
-  const size_t smem = sizeof(int32_t) * 3 * (size_t)L.E;
+  const size_t smem = sizeof(int32_t) * (4 * (size_t)L.E + kScanTileInts);
   k_layout_scan<<<1, kScanThreads, smem, s>>>(L, cap_check);
   note_launch();
   return cudaGetLastError();

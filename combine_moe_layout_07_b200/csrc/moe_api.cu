@@ -107,7 +107,6 @@ static int check_params(const moe_params_t* p) {
 
 static void release(moe_handle_t* h) {
   if (!h) return;
-  if (h->row_block) cudaFreeAsync(h->row_block, h->stream);
   if (h->block) cudaFreeAsync(h->block, h->stream);
   delete h;
 }
@@ -148,23 +147,23 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   h->num_chunks = (int)((T + kChunkTokens - 1) / kChunkTokens);
   const int64_t C = h->num_chunks;
 
-  // one allocation for the fixed-size arrays (256-byte aligned sub-arrays)
+  // One allocation for every array (256-byte aligned sub-arrays).  Without a capacity the row
+  // maps are sized for the worst case of this batch: T * min(k, E_loc) + E_loc * (A - 1) rows.
+  const int64_t E_loc = E / R;
+  h->row_cap = p->recv_capacity_rows > 0
+                   ? p->recv_capacity_rows
+                   : T * (k < E_loc ? k : E_loc) + E_loc * (p->expert_alignment - 1);
   int64_t off = 0;
   auto take = [&](int64_t bytes) {
     const int64_t at = off;
     off = align_up64(off + bytes, 256);
     return at;
   };
-  const int64_t o_status = take(16), o_rows = take(4 * R), o_tok = take(4 * R), o_cnt = take(4 * E),
-                o_psum = take(4 * E), o_pad = take(4 * (E + 1)), o_tir = take(T * R), o_slot = take(4 * T * k),
-                o_prank = take(4 * T * k), o_pw = take(4 * T * k), o_ccnt = take(4 * C * E), o_ctok = take(4 * C * R);
-  const bool rows_now = p->recv_capacity_rows > 0;
-  int64_t o_rsrc = 0, o_rw = 0;
-  if (rows_now) {
-    h->row_cap = p->recv_capacity_rows;
-    o_rsrc = take(4 * R * h->row_cap);
-    o_rw = take(4 * R * h->row_cap);
-  }
+  // status[4] and tokens_per_rank[R] are adjacent so that one memset clears both
+  const int64_t o_status = take(16 + 4 * R), o_rows = take(4 * R), o_cnt = take(4 * E), o_psum = take(4 * E),
+                o_pad = take(4 * (E + 1)), o_tir = take(T * R), o_slot = take(4 * T * k),
+                o_prank = take(4 * T * k), o_pw = take(4 * T * k), o_ccnt = take(4 * C * E),
+                o_rsrc = take(4 * R * h->row_cap), o_rw = take(4 * R * h->row_cap);
   if (pool_alloc(&h->block, (size_t)off, h->device, s) != cudaSuccess) {
     cudaGetLastError();
     delete h;
@@ -173,8 +172,8 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   char* b = static_cast<char*>(h->block);
   DeviceArrays& d = h->d;
   d.status = reinterpret_cast<int32_t*>(b + o_status);
+  d.tokens_per_rank = d.status + 4;
   d.rows_per_rank = reinterpret_cast<int32_t*>(b + o_rows);
-  d.tokens_per_rank = reinterpret_cast<int32_t*>(b + o_tok);
   d.cnt = reinterpret_cast<int32_t*>(b + o_cnt);
   d.psum = reinterpret_cast<int32_t*>(b + o_psum);
   d.pad_excl = reinterpret_cast<int32_t*>(b + o_pad);
@@ -183,11 +182,8 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   d.pair_rank = reinterpret_cast<int32_t*>(b + o_prank);
   d.pair_w = reinterpret_cast<float*>(b + o_pw);
   d.chunk_cnt = reinterpret_cast<int32_t*>(b + o_ccnt);
-  d.chunk_tok = reinterpret_cast<int32_t*>(b + o_ctok);
-  if (rows_now) {
-    d.row_src = reinterpret_cast<int32_t*>(b + o_rsrc);
-    d.row_w = reinterpret_cast<float*>(b + o_rw);
-  }
+  d.row_src = reinterpret_cast<int32_t*>(b + o_rsrc);
+  d.row_w = reinterpret_cast<float*>(b + o_rw);
 
   LayoutLaunch L{};
   L.idx = topk_idx;
@@ -196,7 +192,7 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   L.k = (int)k;
   L.E = (int)E;
   L.R = (int)R;
-  L.E_loc = (int)(E / R);
+  L.E_loc = (int)E_loc;
   L.A = p->expert_alignment;
   L.num_chunks = h->num_chunks;
   L.grid_chunks = h->num_chunks;
@@ -204,24 +200,25 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   L.row_cap = h->row_cap;
   L.d = d;
 
-  cudaError_t err = cudaMemsetAsync(d.status, 0, 16, s);
+  // count -> scan -> assign back to back; with do_cpu_sync one host wait at the end
+  cudaError_t err = cudaMemsetAsync(d.status, 0, (size_t)(16 + 4 * R), s);
   if (err == cudaSuccess) err = launch_layout_count(L, s);
   if (err == cudaSuccess) err = launch_layout_scan(L, p->recv_capacity_rows, s);
+  if (err == cudaSuccess) err = launch_layout_assign(L, s);
   if (err != cudaSuccess) {
     release(h);
     return MOE_ERR_CUDA;
   }
 
   if (p->do_cpu_sync) {
-    // counts to the host: [status flags, rows_per_rank[R], padding total]
-    int32_t* stage = static_cast<int32_t*>(g_stage.get(sizeof(int32_t) * (size_t)(R + 2)));
+    // [status flags, rows_per_rank[R]] to the host
+    int32_t* stage = static_cast<int32_t*>(g_stage.get(sizeof(int32_t) * (size_t)(R + 1)));
     if (!stage) {
       release(h);
       return MOE_ERR_CUDA;
     }
     err = cudaMemcpyAsync(stage, d.status, 4, cudaMemcpyDeviceToHost, s);
     if (err == cudaSuccess) err = cudaMemcpyAsync(stage + 1, d.rows_per_rank, 4 * R, cudaMemcpyDeviceToHost, s);
-    if (err == cudaSuccess) err = cudaMemcpyAsync(stage + 1 + R, d.pad_excl + E, 4, cudaMemcpyDeviceToHost, s);
     if (err == cudaSuccess) err = cudaStreamSynchronize(s);
     if (err != cudaSuccess) {
       release(h);
@@ -236,32 +233,8 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
       return MOE_ERR_CAPACITY;
     }
     h->host_rows.assign(stage + 1, stage + 1 + R);
-    h->host_total_pad = stage[1 + R];
     h->counts_on_host = true;
     if (host_rows_per_rank) std::memcpy(host_rows_per_rank, stage + 1, sizeof(int32_t) * (size_t)R);
-    if (!rows_now) {
-      int32_t mx = 0;
-      for (int32_t v : h->host_rows) mx = v > mx ? v : mx;
-      h->row_cap = mx;
-      if (mx > 0) {
-        const int64_t bytes = align_up64(4 * R * (int64_t)mx, 256);
-        if (pool_alloc(&h->row_block, (size_t)(2 * bytes), h->device, s) != cudaSuccess) {
-          cudaGetLastError();
-          release(h);
-          return MOE_ERR_OOM;
-        }
-        d.row_src = static_cast<int32_t*>(h->row_block);
-        d.row_w = reinterpret_cast<float*>(static_cast<char*>(h->row_block) + bytes);
-      }
-      L.row_cap = h->row_cap;
-      L.d = d;
-    }
-  }
-
-  err = launch_layout_assign(L, s);
-  if (err != cudaSuccess) {
-    release(h);
-    return MOE_ERR_CUDA;
   }
   *out_handle = h;
   return MOE_OK;
@@ -369,7 +342,6 @@ int64_t moe_handle_row_capacity(const moe_handle_t* h) { return h ? h->row_cap :
 int moe_handle_free(moe_handle_t* h) {
   if (!h) return MOE_OK;
   int rc = MOE_OK;
-  if (h->row_block && cudaFreeAsync(h->row_block, h->stream) != cudaSuccess) rc = MOE_ERR_CUDA;
   if (h->block && cudaFreeAsync(h->block, h->stream) != cudaSuccess) rc = MOE_ERR_CUDA;
   delete h;
   return rc;

@@ -26,6 +26,7 @@ constexpr int kChunkTokens = 512;
 constexpr int kLayoutThreads = 256;
 constexpr int kLayoutWarps = kLayoutThreads / 32;
 constexpr int kScanThreads = 1024;
+constexpr int kScanTileInts = 8192;  // chunk-count tile staged in shared memory by the scan
 constexpr int kMaxExperts = 4096;
 constexpr int kMaxTopk = 32;
 
@@ -44,7 +45,6 @@ struct DeviceArrays {
   int32_t* pair_rank = nullptr;       // [T * k]  destination logical rank, -1 if masked
   float* pair_w = nullptr;            // [T * k]
   int32_t* chunk_cnt = nullptr;       // [C * E]  counts, then exclusive offsets
-  int32_t* chunk_tok = nullptr;       // [C * R]
   int32_t* row_src = nullptr;         // [R * row_cap]
   float* row_w = nullptr;             // [R * row_cap]
 };
@@ -55,13 +55,11 @@ struct moe_handle {
   moe_params_t p{};
   cudaStream_t stream = nullptr;
   int device = 0;
-  void* block = nullptr;       // one stream-ordered allocation for the fixed-size arrays
-  void* row_block = nullptr;   // row_src / row_w
+  void* block = nullptr;       // one stream-ordered allocation for every device array
   int64_t row_cap = 0;
   int num_chunks = 0;
   bool counts_on_host = false;
   std::vector<int32_t> host_rows;  // rows_per_rank, when do_cpu_sync
-  int32_t host_total_pad = -1;     // padding rows over all experts, when do_cpu_sync
   moe::DeviceArrays d;
 };
 

@@ -164,7 +164,9 @@ def test_row_capacity_from_counts():
     idx, w, x = inputs(wl)
     h = gpu_layout(wl, idx, w, cap=0, cpu_sync=True)
     lay = oracle.layout(idx.numpy(), w.numpy(), wl.experts, wl.ranks, wl.alignment)
-    assert h.row_capacity() == int(lay.rows_per_rank.max())
+    e_loc = wl.experts_per_rank          # without a capacity the row maps take the worst case
+    assert h.row_capacity() == wl.tokens * min(wl.topk, e_loc) + e_loc * (wl.alignment - 1)
+    assert h.row_capacity() >= int(lay.rows_per_rank.max())
     assert (h.host_rows_per_rank == lay.rows_per_rank).all()
     compare_layout(h, oracle.layout(idx.numpy(), w.numpy(), wl.experts, wl.ranks, wl.alignment,
                                     cap=h.row_capacity()), wl)
