@@ -9,10 +9,10 @@
 //
 // The pages place rows with atomicAdd on the psum counter, whose order is undefined; here the
 // placement is a stable counting sort so the handle is deterministic:
-//   count  : per chunk of 512 tokens, a shared-memory histogram (atomicAdd_block) of expert ids
+//   count  : per chunk of 256 tokens, a shared-memory histogram (atomicAdd_block) of expert ids
 //            and of token->rank membership;
-//   scan   : one CTA; per expert an exclusive scan of the chunk counts (chunk offsets), then a
-//            block-wide warp-shuffle scan of align_up(cnt, A), restarted at every rank;
+//   scan   : a CTA per 32 experts scans the chunk counts of its experts over chunks (chunk
+//            offsets); the last CTA to finish scans align_up(cnt, A), restarted at every rank;
 //   assign : per chunk, each warp takes a contiguous run of (t, j) pairs; per-warp histograms
 //            are scanned across warps, and inside a warp __match_any_sync + popc give each pair
 //            its rank among equal experts -- so rows keep ascending (t, j) order.
@@ -120,71 +120,93 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
 }
 
 // ------------------------------------------------------------------------------------ scan
-// One CTA.  (1) per expert, exclusive scan of the chunk counts over chunks, staged through
-// shared memory a tile of rows at a time (coalesced loads and stores); (2) block-wide scans of
-// align_up(cnt, A) and of the padding rows over all experts; (3) psum restarted at every rank.
+// ceil(E/32) CTAs of 32 x 32 threads.  CTA b owns experts [32b, 32b + 32): lane = expert (so
+// every load of a chunk row is one 128-byte segment), warp w = a contiguous group of chunks.
+// (1) each thread sums its chunk group; (2) warp-shuffle exclusive scan of the 32 group sums of
+// each expert; (3) each thread rewrites its chunk counts as exclusive offsets; the expert total
+// is cnt[e].  The CTA that finishes last (an atomic ticket after a fence; nothing waits) then
+// (4) scans align_up(cnt, A) and the padding rows over all experts and (5) restarts psum at
+// every rank.
 __global__ void __launch_bounds__(kScanThreads) k_layout_scan(LayoutLaunch L, int64_t cap_check) {
+  __shared__ int32_t gsum[32][33];
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t totals[2];
+  __shared__ int32_t is_last;
   extern __shared__ int32_t sm[];
   const int E = L.E;
-  int32_t* al = sm;              // [E] align_up(cnt, A)
-  int32_t* pad = sm + E;         // [E] align_up(cnt, A) - cnt
-  int32_t* gincl = sm + 2 * E;   // [E] inclusive prefix of al over all experts
-  int32_t* run = sm + 3 * E;     // [E] running chunk offset
-  int32_t* tile = sm + 4 * E;    // [rows][E]
-  const int rows = kScanTileInts / E;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int e = blockIdx.x * 32 + lane;
+  const int C = L.num_chunks;
+  const int cpw = (C + 31) / 32;  // chunks per warp
+  const int c0 = min(C, warp * cpw), c1 = min(C, c0 + cpw);
 
-  for (int e = tid; e < E; e += blockDim.x) run[e] = 0;
+  int32_t sum = 0;
+  if (e < E)
+    for (int c = c0; c < c1; ++c) sum += L.d.chunk_cnt[(int64_t)c * E + e];
+  gsum[warp][lane] = sum;
   __syncthreads();
-  for (int c0 = 0; c0 < L.num_chunks; c0 += rows) {
-    const int nr = min(rows, L.num_chunks - c0);
-    int32_t* g = L.d.chunk_cnt + (int64_t)c0 * E;
-    for (int i = tid; i < nr * E; i += blockDim.x) tile[i] = g[i];
-    __syncthreads();
-    for (int e = tid; e < E; e += blockDim.x) {
-      int32_t r = run[e];
-      for (int c = 0; c < nr; ++c) {
-        const int32_t v = tile[c * E + e];
-        tile[c * E + e] = r;
-        r += v;
-      }
-      run[e] = r;
+  {  // warp x scans the 32 group sums of expert blockIdx.x*32 + x
+    const int32_t v = gsum[lane][warp];
+    int32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
     }
-    __syncthreads();
-    for (int i = tid; i < nr * E; i += blockDim.x) g[i] = tile[i];
-    __syncthreads();
-  }
-  for (int e = tid; e < E; e += blockDim.x) {
-    const int32_t n = run[e];
-    L.d.cnt[e] = n;
-    al[e] = align_up_dev(n, L.A);
-    pad[e] = al[e] - n;
+    __syncwarp();
+    gsum[lane][warp] = incl - v;
+    const int ex = blockIdx.x * 32 + warp;
+    if (lane == 31 && ex < E) L.d.cnt[ex] = incl;
   }
   __syncthreads();
+  if (e < E) {
+    int32_t off = gsum[warp][lane];
+    for (int c = c0; c < c1; ++c) {
+      int32_t* q = L.d.chunk_cnt + (int64_t)c * E + e;
+      const int32_t v = *q;
+      *q = off;
+      off += v;
+    }
+  }
 
+  // the last CTA to finish sees every cnt[e]
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) is_last = atomicAdd(L.d.ticket, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  if (tid == 0) *L.d.ticket = 0;  // ready for the next layout on this scratch
+
+  int32_t* al = sm;             // [E] align_up(cnt, A)
+  int32_t* pad = sm + E;        // [E] align_up(cnt, A) - cnt
+  int32_t* gincl = sm + 2 * E;  // [E] inclusive prefix of al over all experts
+  for (int x = tid; x < E; x += blockDim.x) {
+    const int32_t n = __ldcg(L.d.cnt + x);
+    al[x] = align_up_dev(n, L.A);
+    pad[x] = al[x] - n;
+  }
+  __syncthreads();
   const int per = (E + blockDim.x - 1) / blockDim.x;
   const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
   int32_t sa = 0, sp = 0;
-  for (int e = e0; e < e1; ++e) {
-    sa += al[e];
-    sp += pad[e];
+  for (int x = e0; x < e1; ++x) {
+    sa += al[x];
+    sp += pad[x];
   }
   int32_t ra = block_exclusive_scan(sa, warp_tot, &totals[0]);
   int32_t rp = block_exclusive_scan(sp, warp_tot, &totals[1]);
-  for (int e = e0; e < e1; ++e) {
-    L.d.pad_excl[e] = rp;
-    rp += pad[e];
-    ra += al[e];
-    gincl[e] = ra;
+  for (int x = e0; x < e1; ++x) {
+    L.d.pad_excl[x] = rp;
+    rp += pad[x];
+    ra += al[x];
+    gincl[x] = ra;
   }
   if (tid == 0) L.d.pad_excl[E] = totals[1];
   __syncthreads();
-
-  for (int e = tid; e < E; e += blockDim.x) {
-    const int first = (e / L.E_loc) * L.E_loc;
-    L.d.psum[e] = gincl[e] - (gincl[first] - al[first]);
+  for (int x = tid; x < E; x += blockDim.x) {
+    const int first = (x / L.E_loc) * L.E_loc;
+    L.d.psum[x] = gincl[x] - (gincl[first] - al[first]);
   }
   for (int r = tid; r < L.R; r += blockDim.x) {
     const int first = r * L.E_loc, last = first + L.E_loc - 1;
@@ -319,7 +341,7 @@ static cudaError_t ensure_smem_attrs() {
   if (err != cudaSuccess) return err;
   if (dev < 64 && (done >> dev) & 1ull) return cudaSuccess;
   err = cudaFuncSetAttribute(k_layout_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(sizeof(int32_t) * (4 * kMaxExperts + kScanTileInts)));
+                             (int)(sizeof(int32_t) * 3 * kMaxExperts));
   if (err == cudaSuccess)
     err = cudaFuncSetAttribute(k_layout_assign, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(sizeof(int32_t) * kLayoutWarps * kMaxExperts));
@@ -338,8 +360,8 @@ cudaError_t launch_layout_count(const LayoutLaunch& L, cudaStream_t s) {
 cudaError_t launch_layout_scan(const LayoutLaunch& L, int64_t cap_check, cudaStream_t s) {
   cudaError_t err = ensure_smem_attrs();
   if (err != cudaSuccess) return err;
-  const size_t smem = sizeof(int32_t) * (4 * (size_t)L.E + kScanTileInts);
-  k_layout_scan<<<1, kScanThreads, smem, s>>>(L, cap_check);
+  const size_t smem = sizeof(int32_t) * 3 * (size_t)L.E;
+  k_layout_scan<<<(L.E + 31) / 32, kScanThreads, smem, s>>>(L, cap_check);
   note_launch();
   return cudaGetLastError();
 }

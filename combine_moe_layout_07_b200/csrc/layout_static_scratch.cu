@@ -9,9 +9,9 @@
 //
 // The array (MOE_STATIC_SCRATCH_BYTES) is part of the library's device image: every GPU that
 // loads the library holds it until the process exits.  All calls share it and it keeps the last
-// call's contents, so the status word is cleared at the start of every call (all other scratch
-// regions are fully rewritten before they are read; the caller's tokens_per_rank, which the
-// kernels sum into, is cleared too).  Calls whose GPU work overlaps -- on two
+// call's contents, so the status word and the scan's ticket counter are cleared at the start of
+// every call (all other scratch regions are fully rewritten before they are read; the caller's
+// tokens_per_rank, which the kernels sum into, is cleared too).  Calls whose GPU work overlaps -- on two
 // streams, or from two host threads, on the same device -- race on the array.
 //
 // Host code cannot use the array's name as a device address: the first call on each device,
@@ -75,7 +75,7 @@ extern "C" int moe_layout_static_scratch(const moe_params_t* p, const int64_t* t
       (reinterpret_cast<uintptr_t>(device_status) & 3u))
     return MOE_ERR_INVALID_ARG;
 
-  // scratch regions: status | pad prefix | chunk counts | pair rank | pair weight
+  // scratch regions: status and scan ticket | pad prefix | chunk counts | pair rank | pair weight
   const int64_t C = (T + kChunkTokens - 1) / kChunkTokens;
   const int64_t o_status = 0, o_pad = o_status + 256, o_ccnt = o_pad + round256(4 * (E + 1)),
                 o_prank = o_ccnt + round256(4 * C * E), o_pw = o_prank + round256(4 * T * k),
@@ -90,6 +90,7 @@ extern "C" int moe_layout_static_scratch(const moe_params_t* p, const int64_t* t
 
   DeviceArrays d{};
   d.status = device_status ? device_status : reinterpret_cast<int32_t*>(b + o_status);
+  d.ticket = reinterpret_cast<int32_t*>(b + o_status + 64);
   d.cnt = counts;
   d.psum = psum;
   d.pad_excl = reinterpret_cast<int32_t*>(b + o_pad);
@@ -120,6 +121,7 @@ extern "C" int moe_layout_static_scratch(const moe_params_t* p, const int64_t* t
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t err = cudaMemsetAsync(d.status, 0, sizeof(int32_t), s);
+  if (err == cudaSuccess) err = cudaMemsetAsync(d.ticket, 0, sizeof(int32_t), s);
   if (err == cudaSuccess) err = cudaMemsetAsync(tokens_per_rank, 0, sizeof(int32_t) * (size_t)R, s);  // summed atomically
   if (err == cudaSuccess) err = launch_layout_count(L, s);
   if (err == cudaSuccess) err = launch_layout_scan(L, p->recv_capacity_rows, s);

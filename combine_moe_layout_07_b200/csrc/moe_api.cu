@@ -159,8 +159,8 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
     off = align_up64(off + bytes, 256);
     return at;
   };
-  // status[4] and tokens_per_rank[R] are adjacent so that one memset clears both
-  const int64_t o_status = take(16 + 4 * R), o_rows = take(4 * R), o_cnt = take(4 * E), o_psum = take(4 * E),
+  // status[4], the scan ticket and tokens_per_rank[R] are adjacent: one memset clears them
+  const int64_t o_status = take(32 + 4 * R), o_rows = take(4 * R), o_cnt = take(4 * E), o_psum = take(4 * E),
                 o_pad = take(4 * (E + 1)), o_tir = take(T * R), o_slot = take(4 * T * k),
                 o_prank = take(4 * T * k), o_pw = take(4 * T * k), o_ccnt = take(4 * C * E),
                 o_rsrc = take(4 * R * h->row_cap), o_rw = take(4 * R * h->row_cap);
@@ -172,7 +172,8 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   char* b = static_cast<char*>(h->block);
   DeviceArrays& d = h->d;
   d.status = reinterpret_cast<int32_t*>(b + o_status);
-  d.tokens_per_rank = d.status + 4;
+  d.ticket = d.status + 4;
+  d.tokens_per_rank = d.status + 8;
   d.rows_per_rank = reinterpret_cast<int32_t*>(b + o_rows);
   d.cnt = reinterpret_cast<int32_t*>(b + o_cnt);
   d.psum = reinterpret_cast<int32_t*>(b + o_psum);
@@ -201,7 +202,7 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   L.d = d;
 
   // count -> scan -> assign back to back; with do_cpu_sync one host wait at the end
-  cudaError_t err = cudaMemsetAsync(d.status, 0, (size_t)(16 + 4 * R), s);
+  cudaError_t err = cudaMemsetAsync(d.status, 0, (size_t)(32 + 4 * R), s);
   if (err == cudaSuccess) err = launch_layout_count(L, s);
   if (err == cudaSuccess) err = launch_layout_scan(L, p->recv_capacity_rows, s);
   if (err == cudaSuccess) err = launch_layout_assign(L, s);

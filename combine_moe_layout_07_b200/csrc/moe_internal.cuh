@@ -21,12 +21,12 @@ constexpr bool kDebugChecks = true;
 constexpr bool kDebugChecks = false;
 #endif
 
-// Layout tiling: a chunk of tokens per CTA; 8 warps per layout CTA.
-constexpr int kChunkTokens = 512;
+// Layout tiling: a chunk of tokens per CTA (a thread per token in the count kernel); 8 warps per
+// layout CTA.
+constexpr int kChunkTokens = 256;
 constexpr int kLayoutThreads = 256;
 constexpr int kLayoutWarps = kLayoutThreads / 32;
 constexpr int kScanThreads = 1024;
-constexpr int kScanTileInts = 8192;  // chunk-count tile staged in shared memory by the scan
 constexpr int kMaxExperts = 4096;
 constexpr int kMaxTopk = 32;
 
@@ -34,7 +34,8 @@ constexpr int kMaxTopk = 32;
 constexpr int kMoveThreads = 1024;
 
 struct DeviceArrays {
-  int32_t* status = nullptr;          // [4]
+  int32_t* status = nullptr;          // [4]  flags, then MOE_DEBUG details
+  int32_t* ticket = nullptr;          // [1]  CTAs of the scan that have finished (0 between launches)
   int32_t* cnt = nullptr;             // [E]
   int32_t* psum = nullptr;            // [E]
   int32_t* pad_excl = nullptr;        // [E + 1]  exclusive prefix of padding rows, all experts

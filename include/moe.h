@@ -173,7 +173,7 @@ const char* moe_status_string(int status);
  * Its temporaries (status word, padding prefix, per-chunk counts, per-pair rank and weight)
  * live in one file-scope device array of MOE_STATIC_SCRATCH_BYTES, which every GPU that loads
  * the library holds until the process exits.  It needs
- *   256 + r(4(E+1)) + r(4*C*E) + 2*r(4*T*k) bytes, C = ceil(T/512), r = round up to 256;
+ *   256 + r(4(E+1)) + r(4*C*E) + 2*r(4*T*k) bytes, C = ceil(T/256), r = round up to 256;
  * larger problems return MOE_ERR_SCRATCH_LIMIT before any GPU work.
  *   device_status  int32, device, nullable: receives the device status flags of this call
  *                  (bit 0: an expert id outside [-1, E); bit 1: a rank needs more than cap rows);
