@@ -286,6 +286,109 @@ def run_e2e(args, world, dev, stream, step, step_bytes, x, idx, w, y, bias, out,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n}
 
 
+# --------------------------------------------------------------------------- workload extras
+def decode_latency(step_parts, stream, dev, n: int = 50) -> dict:
+    """Per-call latency of layout, dispatch and combine, median over n steps, warm (back to back)
+    and cold (L2 flushed by writing a buffer of twice the L2 size before every step)."""
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+    def run(cold: bool) -> dict:
+        rec = {"layout": [], "dispatch": [], "combine": [], "total": []}
+        for _ in range(n):
+            if cold:
+                flush.fill_(1)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            step_parts(ev, stream)
+            torch.cuda.synchronize()
+            rec["layout"].append(ev[0].elapsed_time(ev[1]) * 1e3)
+            rec["dispatch"].append(ev[1].elapsed_time(ev[2]) * 1e3)
+            rec["combine"].append(ev[2].elapsed_time(ev[3]) * 1e3)
+            rec["total"].append(ev[0].elapsed_time(ev[3]) * 1e3)
+        return {k: round(statistics.median(v), 2) for k, v in rec.items()}
+
+    res = {"unit": "us", "warm": run(False), "cold_l2_flushed": run(True), "samples": n}
+    # the same round trip captured once in a CUDA graph (do_cpu_sync=0 path), replayed warm
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step_parts([torch.cuda.Event() for _ in range(4)], torch.cuda.current_stream())
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    res["graph_replay_total"] = round(e0.elapsed_time(e1) * 1e3 / n, 2)
+    del g
+    return res
+
+
+def skewed_overlap(step, stream, dev, n_steps: int = 50) -> dict:
+    """MoE round trips capped at the workload's num_sms on one stream while a second stream runs
+    bf16 4096^3 matmuls: serial vs concurrent device time, and each side's slowdown."""
+    a = torch.randn(4096, 4096, device=dev, dtype=torch.bfloat16)
+    b = torch.randn(4096, 4096, device=dev, dtype=torch.bfloat16)
+    side = torch.cuda.Stream(device=dev)
+
+    def timed(fn, st):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        fn()
+        e1.record(st)
+        return e0, e1
+
+    def moe_loop():
+        for _ in range(n_steps):
+            step(False)
+
+    # size the GEMM loop to last about as long as the MoE loop (after cuBLAS warm-up)
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            torch.matmul(a, b)
+    torch.cuda.synchronize()
+    m0, m1 = timed(moe_loop, stream)
+    torch.cuda.synchronize()
+    moe_ms = m0.elapsed_time(m1)
+    per_gemm = float("inf")
+    for _ in range(2):  # twice; the faster run sets the per-call time
+        with torch.cuda.stream(side):
+            g0, g1 = timed(lambda: [torch.matmul(a, b) for _ in range(20)], side)
+        torch.cuda.synchronize()
+        per_gemm = min(per_gemm, g0.elapsed_time(g1) / 20)
+    n_gemm = max(1, int(round(moe_ms / max(per_gemm, 1e-3))))
+
+    def gemm_loop():
+        for _ in range(n_gemm):
+            torch.matmul(a, b)
+
+    with torch.cuda.stream(side):
+        g0, g1 = timed(gemm_loop, side)
+    torch.cuda.synchronize()
+    gemm_ms = g0.elapsed_time(g1)
+    # concurrent: both streams start after one event
+    start = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    side.wait_event(start)
+    with torch.cuda.stream(side):
+        ge = torch.cuda.Event(enable_timing=True)
+        gemm_loop()
+        ge.record(side)
+    me = torch.cuda.Event(enable_timing=True)
+    moe_loop()
+    me.record(stream)
+    torch.cuda.synchronize()
+    moe_c, gemm_c = start.elapsed_time(me), start.elapsed_time(ge)
+    wall = max(moe_c, gemm_c)
+    return {"unit": "ms", "moe_steps": n_steps, "gemm_calls": n_gemm, "moe_alone": round(moe_ms, 3),
+            "gemm_alone": round(gemm_ms, 3), "serial": round(moe_ms + gemm_ms, 3),
+            "concurrent_wall": round(wall, 3), "moe_concurrent": round(moe_c, 3), "gemm_concurrent": round(gemm_c, 3),
+            "moe_slowdown": round(moe_c / moe_ms, 3), "gemm_slowdown": round(gemm_c / gemm_ms, 3),
+            "overlap_saving": round(1 - wall / (moe_ms + gemm_ms), 3)}
+
+
 # --------------------------------------------------------------------------- our arm
 def run_ours(args) -> int:
     world, rank, local = dist_setup("nccl")
@@ -357,6 +460,18 @@ def run_ours(args) -> int:
         moe.moe_handle_free(h)
 
     clk = ClockSampler(local).start()
+    def step_parts(ev, st):
+        ev[0].record(st)
+        h = moe.moe_layout(make_params(p_cap), idx, w, stream=st)
+        ev[1].record(st)
+        moe.moe_dispatch(h, x, dtype_out, recv, scales, None, cap=cap, do_zero_padding=wl.zero_padding,
+                         num_sms=wl.num_sms, stream=st)
+        ev[2].record(st)
+        moe.moe_combine(h, y, out, topk_weights=weights_for_combine, bias=bias, cap=cap, num_sms=wl.num_sms,
+                        stream=st)
+        ev[3].record(st)
+        moe.moe_handle_free(h)
+
     for _ in range(args.warmup):
         step(False)
     torch.cuda.synchronize()
@@ -385,6 +500,12 @@ def run_ours(args) -> int:
     # end to end through the public API: pinned host inputs -> device, round trip, result -> host
     e2e = None if args.no_e2e else run_e2e(args, world, dev, stream, step, step_bytes, x, idx, w, y, bias, out,
                                            x_c, idx_c, w_c, bias_c)
+    extras = {}
+    if wl.name == "decode":
+        extras["latency"] = decode_latency(step_parts, stream, dev)
+    if wl.name == "skewed":
+        extras["overlap"] = skewed_overlap(step, stream, dev)
+        extras["rows_per_rank"] = {"max": int(rows.max()), "mean": float(rows.mean()), "min": int(rows.min())}
     peak, peak_kind = hbm_peak()
     kern = {"dispatch": (dispatch_ms, nb["dispatch"]), "combine": (combine_ms, nb["combine"])}
     dom = max(kern, key=lambda k: kern[k][0])
@@ -417,7 +538,7 @@ def run_ours(args) -> int:
                 "roofline": roofline, "cpu_baseline": cpu,
                 "e2e": e2e,
                 "gpu_launches": launches, "clocks": clk.summary(),
-                "library": os.path.relpath(moe.library_path(), ROOT)}
+                "library": os.path.relpath(moe.library_path(), ROOT), **extras}
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized():

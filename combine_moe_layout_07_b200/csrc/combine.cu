@@ -112,6 +112,8 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
     fence_mbar_init();
   }
   __syncthreads();
+  grid_dependents_launch();
+  grid_dependency_wait();  // the expert outputs and the handle written by earlier kernels
 
   int64_t t_begin, t_end;
   cta_token_range(L.T, t_begin, t_end);
@@ -293,13 +295,15 @@ cudaError_t launch_combine(const CombineLaunch& L, cudaStream_t st) {
   const bool wgt = L.w != nullptr, has_bias = L.bias != nullptr;
   const CombGeom g = combine_geometry(L.H, L.k, has_bias);
   if (g.stages < kCombGroups || g.stages % kCombGroups != 0) return cudaErrorInvalidValue;
+  static unsigned long long done[4] = {0, 0, 0, 0};
+  const int variant = (wgt ? 2 : 0) + (has_bias ? 1 : 0);
   auto kern = wgt ? (has_bias ? k_combine<true, true> : k_combine<true, false>)
                   : (has_bias ? k_combine<false, true> : k_combine<false, false>);
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCombSmemBudget);
+  cudaError_t err = set_smem_limit_once(kern, (int)kCombSmemBudget, &done[variant]);
   if (err != cudaSuccess) return err;
-  kern<<<L.grid, kCombThreads, g.total, st>>>(L, g);
+  err = launch_pdl(kern, dim3(L.grid), dim3(kCombThreads), (size_t)g.total, st, L, g);
   note_launch();
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace moe

@@ -94,6 +94,8 @@ __global__ void __launch_bounds__(kDispThreads, 1) k_dispatch(DispatchLaunch L, 
     fence_mbar_init();
   }
   __syncthreads();
+  grid_dependents_launch();
+  grid_dependency_wait();  // the handle written by the layout kernels
 
   int64_t t_begin, t_end;
   cta_token_range(L.T, t_begin, t_end);
@@ -278,12 +280,13 @@ cudaError_t launch_dispatch(const DispatchLaunch& L, bool fp8, cudaStream_t st) 
   const int S = dispatch_stages(L.H);
   if (S < kDispGroups) return cudaErrorInvalidValue;
   const uint32_t smem = disp_smem(L.H, S).total;
+  static unsigned long long done[2] = {0, 0};
   auto kern = fp8 ? k_dispatch<true> : k_dispatch<false>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBudget);
+  cudaError_t err = set_smem_limit_once(kern, (int)kSmemBudget, &done[fp8 ? 1 : 0]);
   if (err != cudaSuccess) return err;
-  kern<<<L.grid, kDispThreads, smem, st>>>(L, S);
+  err = launch_pdl(kern, dim3(L.grid), dim3(kDispThreads), smem, st, L, S);
   note_launch();
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace moe

@@ -28,67 +28,149 @@ __device__ __forceinline__ int32_t expert_of(int64_t e, int E) {
   return (e >= 0 && e < E) ? (int32_t)e : (e == -1 ? -1 : -2);
 }
 
-// ------------------------------------------------------------------------------------ count
-// A thread per token: its k ids are loaded together, counted into the chunk's shared-memory
-// histogram (atomicAdd_block), and its rank membership is written and counted.
-__global__ void __launch_bounds__(kLayoutThreads) k_layout_count(LayoutLaunch L) {
-  extern __shared__ int32_t sm[];
-  int32_t* hist = sm;       // [E]
-  int32_t* tok = sm + L.E;  // [R]
-  const int tid = threadIdx.x;
+// ------------------------------------------------------------------------------------ helpers
+// Membership of token t (when `valid`): writes token_in_rank[t, :] and counts the token for every
+// rank holding one of its experts into tok[r] (shared memory).  Called by whole warps: with R <= 64
+// the per-rank counts are aggregated over the warp (one ballot per rank, one atomic from lane 0),
+// which keeps shared-memory atomics off a handful of hot addresses.  When `hist` is given, every
+// valid id is also counted into it.  Returns false if one of the token's ids lies outside [-1, E).
+__device__ __forceinline__ bool token_membership(const LayoutLaunch& L, int64_t t, bool valid, int32_t* hist,
+                                                 int32_t* tok) {
   bool bad = false;
-  for (int c = blockIdx.x; c < L.num_chunks; c += gridDim.x) {
-    for (int i = tid; i < L.E + L.R; i += blockDim.x) sm[i] = 0;
-    __syncthreads();
-    const int64_t t0 = (int64_t)c * kChunkTokens;
-    const int64_t t1 = min(L.T, t0 + kChunkTokens);
-    for (int64_t t = t0 + tid; t < t1; t += blockDim.x) {
-      const int64_t* ids = L.idx + t * L.k;
-      int32_t ev[kMaxTopk];
+  int32_t ev[kMaxTopk];
+  const int64_t* ids = L.idx + t * L.k;
 #pragma unroll
-      for (int j = 0; j < kMaxTopk; ++j) {
-        ev[j] = j < L.k ? expert_of(__ldg(ids + j), L.E) : -1;
-        if (ev[j] == -2) {
-          bad = true;
-          ev[j] = -1;
+  for (int j = 0; j < kMaxTopk; ++j) {
+    ev[j] = (valid && j < L.k) ? expert_of(__ldg(ids + j), L.E) : -1;
+    if (ev[j] == -2) {
+      bad = true;
+      ev[j] = -1;
+    }
+  }
+  uint8_t* member = L.d.token_in_rank + t * L.R;
+  if (L.R <= 64) {
+    uint64_t mask = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxTopk; ++j)
+      if (ev[j] >= 0) {
+        if (hist) atomicAdd_block(&hist[ev[j]], 1);
+        mask |= 1ull << ((uint32_t)ev[j] / (uint32_t)L.E_loc);
+      }
+    if (valid)
+      for (int r = 0; r < L.R; ++r) member[r] = (uint8_t)((mask >> r) & 1);
+    const int lane = threadIdx.x & 31;
+    for (int r = 0; r < L.R; ++r) {
+      const int c = __popc(__ballot_sync(0xffffffffu, (mask >> r) & 1));
+      if (lane == 0 && c) atomicAdd_block(&tok[r], c);
+    }
+  } else if (valid) {
+    for (int r = 0; r < L.R; ++r) member[r] = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxTopk; ++j)
+      if (ev[j] >= 0) {
+        if (hist) atomicAdd_block(&hist[ev[j]], 1);
+        const int r = (int)((uint32_t)ev[j] / (uint32_t)L.E_loc);
+        bool first = true;
+#pragma unroll
+        for (int j2 = 0; j2 < j; ++j2)
+          if (ev[j2] >= 0 && (int)((uint32_t)ev[j2] / (uint32_t)L.E_loc) == r) first = false;
+        if (first) {
+          member[r] = 1;
+          atomicAdd_block(&tok[r], 1);
         }
       }
-      uint8_t* member = L.d.token_in_rank + t * L.R;
-      if (L.R <= 64) {
-        uint64_t mask = 0;
+  }
+  return !bad;
+}
+
+constexpr int kAssignBatch = 8;  // rounds of 32 pairs a warp loads before it works on them
+
+// Phase 1 of the slot assignment: histogram h[E] of the warp's pairs [wp0, wp1) (h zeroed).
+__device__ __forceinline__ void warp_histogram(const LayoutLaunch& L, int64_t wp0, int64_t wp1, int32_t* h) {
+  const int lane = threadIdx.x & 31;
+  for (int64_t base = wp0; base < wp1; base += 32 * kAssignBatch) {
+    int32_t ev[kAssignBatch];
 #pragma unroll
-        for (int j = 0; j < kMaxTopk; ++j)
-          if (ev[j] >= 0) {
-            atomicAdd_block(&hist[ev[j]], 1);
-            mask |= 1ull << (ev[j] / L.E_loc);
+    for (int r = 0; r < kAssignBatch; ++r) {
+      const int64_t p = base + r * 32 + lane;
+      ev[r] = p < wp1 ? max(expert_of(__ldg(L.idx + p), L.E), -1) : -1;
+    }
+#pragma unroll
+    for (int r = 0; r < kAssignBatch; ++r) {
+      const uint32_t peers = __match_any_sync(0xffffffffu, ev[r]);
+      if (ev[r] >= 0 && lane == __ffs(peers) - 1) h[ev[r]] += __popc(peers);
+      __syncwarp();
+    }
+  }
+}
+
+// Phase 3: walk the warp's pairs in (t, j) order; h[e] holds the warp's next row of expert e.
+// Writes slot, pair rank, pair weight and the row maps.  Returns true on a row >= row_cap.
+__device__ __forceinline__ bool warp_assign(const LayoutLaunch& L, int64_t wp0, int64_t wp1, int32_t* h) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = lanemask_lt();
+  bool overflow = false;
+  for (int64_t base = wp0; base < wp1; base += 32 * kAssignBatch) {
+    int32_t ev[kAssignBatch];
+    float wv[kAssignBatch];
+#pragma unroll
+    for (int r = 0; r < kAssignBatch; ++r) {
+      const int64_t p = base + r * 32 + lane;
+      ev[r] = p < wp1 ? max(expert_of(__ldg(L.idx + p), L.E), -1) : -1;
+      wv[r] = (p < wp1 && L.w) ? __ldg(L.w + p) : 0.0f;
+    }
+#pragma unroll
+    for (int r = 0; r < kAssignBatch; ++r) {
+      const int64_t p = base + r * 32 + lane;
+      const int32_t e = ev[r];
+      const uint32_t peers = __match_any_sync(0xffffffffu, e);
+      int32_t row = -1;
+      if (e >= 0) row = h[e] + __popc(peers & lt);
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) h[e] += __popc(peers);
+      __syncwarp();
+      if (p < wp1) {
+        // 32-bit divisions: e < E and p < T * k < 2^31
+        const int rk = e >= 0 ? (int)((uint32_t)e / (uint32_t)L.E_loc) : -1;
+        L.d.slot[p] = row;
+        L.d.pair_rank[p] = rk;
+        L.d.pair_w[p] = wv[r];
+        if (e >= 0) {
+          if (row < L.row_cap) {
+            L.d.row_src[(int64_t)rk * L.row_cap + row] = (int32_t)((uint32_t)p / (uint32_t)L.k);
+            L.d.row_w[(int64_t)rk * L.row_cap + row] = wv[r];
+          } else {
+            overflow = true;
           }
-        for (int r = 0; r < L.R; ++r) member[r] = (uint8_t)((mask >> r) & 1);
-        for (uint64_t m = mask; m; m &= m - 1) atomicAdd_block(&tok[__ffsll((long long)m) - 1], 1);
-      } else {
-        for (int r = 0; r < L.R; ++r) member[r] = 0;
-#pragma unroll
-        for (int j = 0; j < kMaxTopk; ++j)
-          if (ev[j] >= 0) {
-            atomicAdd_block(&hist[ev[j]], 1);
-            const int r = ev[j] / L.E_loc;
-            bool first = true;
-#pragma unroll
-            for (int j2 = 0; j2 < j; ++j2)
-              if (ev[j2] >= 0 && ev[j2] / L.E_loc == r) first = false;
-            if (first) {
-              member[r] = 1;
-              atomicAdd_block(&tok[r], 1);
-            }
-          }
+        }
       }
     }
-    __syncthreads();
-    for (int e = tid; e < L.E; e += blockDim.x) L.d.chunk_cnt[(int64_t)c * L.E + e] = hist[e];
-    for (int r = tid; r < L.R; r += blockDim.x)
-      if (tok[r]) atomicAdd(L.d.tokens_per_rank + r, tok[r]);  // integer sum: order-free
-    __syncthreads();
   }
-  if (bad) atomicOr(L.d.status, kStatusBadExpert);
+  return overflow;
+}
+
+// Padding rows of the row maps: warp w0, w0 + wstride, ... takes experts in turn and its lanes
+// stride over the expert's padding rows [psum - pad, psum) (pad from pad_excl, psum and pad_excl
+// in global or shared memory).  Returns true on a row >= row_cap.
+__device__ __forceinline__ bool row_map_padding(const LayoutLaunch& L, const int32_t* pad_excl, const int32_t* psum,
+                                                int64_t w0, int64_t wstride) {
+  const int lane = threadIdx.x & 31;
+  bool overflow = false;
+  for (int64_t e = w0; e < L.E; e += wstride) {
+    const int32_t pad_e = pad_excl[e + 1] - pad_excl[e];
+    if (pad_e == 0) continue;
+    const int32_t end = psum[e];
+    const int64_t base = (int64_t)((uint32_t)e / (uint32_t)L.E_loc) * L.row_cap;
+    for (int32_t row = end - pad_e + lane; row < end; row += 32) {
+      if (row < L.row_cap) {
+        L.d.row_src[base + row] = -1;
+        L.d.row_w[base + row] = 0.0f;
+      } else {
+        overflow = true;
+      }
+    }
+  }
+  return overflow;
 }
 
 // Block-wide exclusive scan of one value per thread (warp shuffles + one smem pass).
@@ -119,18 +201,95 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
   return r;
 }
 
+// Given cnt[] (global memory written by other CTAs when kCntGlobal, else this CTA's shared
+// memory), one CTA computes, with al / pad / gincl / pad_s as [E] or [E + 1] shared arrays:
+// align_up(cnt, A), the padding prefix over all experts (to pad_excl and pad_s), psum restarted
+// at every rank (to psum and psum_s), rows_per_rank and the capacity flag.
+template <bool kCntGlobal>
+__device__ __forceinline__ void block_psum(const LayoutLaunch& L, const int32_t* cnt, int64_t cap_check, int32_t* al,
+                                           int32_t* pad, int32_t* gincl, int32_t* pad_s, int32_t* psum_s) {
+  __shared__ int32_t warp_tot[32];
+  __shared__ int32_t totals[2];
+  const int E = L.E, tid = threadIdx.x;
+  for (int x = tid; x < E; x += blockDim.x) {
+    const int32_t n = kCntGlobal ? __ldcg(cnt + x) : cnt[x];  // L2: values other CTAs wrote
+    al[x] = align_up_dev(n, L.A);
+    pad[x] = al[x] - n;
+  }
+  __syncthreads();
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
+  int32_t sa = 0, sp = 0;
+  for (int x = e0; x < e1; ++x) {
+    sa += al[x];
+    sp += pad[x];
+  }
+  int32_t ra = block_exclusive_scan(sa, warp_tot, &totals[0]);
+  int32_t rp = block_exclusive_scan(sp, warp_tot, &totals[1]);
+  for (int x = e0; x < e1; ++x) {
+    L.d.pad_excl[x] = rp;
+    if (pad_s) pad_s[x] = rp;
+    rp += pad[x];
+    ra += al[x];
+    gincl[x] = ra;
+  }
+  if (tid == 0) {
+    L.d.pad_excl[E] = totals[1];
+    if (pad_s) pad_s[E] = totals[1];
+  }
+  __syncthreads();
+  for (int x = tid; x < E; x += blockDim.x) {
+    const int first = (x / L.E_loc) * L.E_loc;
+    const int32_t v = gincl[x] - (gincl[first] - al[first]);
+    L.d.psum[x] = v;
+    if (psum_s) psum_s[x] = v;
+  }
+  for (int r = tid; r < L.R; r += blockDim.x) {
+    const int first = r * L.E_loc, last = first + L.E_loc - 1;
+    const int32_t nrows = gincl[last] - (gincl[first] - al[first]);
+    L.d.rows_per_rank[r] = nrows;
+    if (cap_check > 0 && nrows > cap_check) atomicOr(L.d.status, kStatusCapacity);
+  }
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------------------------ count
+// A thread per token: its k ids are loaded together, counted into the chunk's shared-memory
+// histogram (atomicAdd_block), and its rank membership is written and counted.
+__global__ void __launch_bounds__(kLayoutThreads) k_layout_count(LayoutLaunch L) {
+  extern __shared__ int32_t sm[];
+  int32_t* hist = sm;       // [E]
+  int32_t* tok = sm + L.E;  // [R]
+  const int tid = threadIdx.x;
+  bool ok = true;
+  grid_dependents_launch();
+  for (int c = blockIdx.x; c < L.num_chunks; c += gridDim.x) {
+    for (int i = tid; i < L.E + L.R; i += blockDim.x) sm[i] = 0;
+    __syncthreads();
+    const int64_t t0 = (int64_t)c * kChunkTokens;
+    const int64_t t1 = min(L.T, t0 + kChunkTokens);
+    for (int64_t tb = t0; tb < t1; tb += blockDim.x) {  // same trip count for every thread
+      const int64_t t = tb + tid;
+      ok &= token_membership(L, t, t < t1, hist, tok);
+    }
+    __syncthreads();
+    for (int e = tid; e < L.E; e += blockDim.x) L.d.chunk_cnt[(int64_t)c * L.E + e] = hist[e];
+    for (int r = tid; r < L.R; r += blockDim.x)
+      if (tok[r]) atomicAdd(L.d.tokens_per_rank + r, tok[r]);  // integer sum: order-free
+    __syncthreads();
+  }
+  if (!ok) atomicOr(L.d.status, kStatusBadExpert);
+}
+
 // ------------------------------------------------------------------------------------ scan
 // ceil(E/32) CTAs of 32 x 32 threads.  CTA b owns experts [32b, 32b + 32): lane = expert (so
 // every load of a chunk row is one 128-byte segment), warp w = a contiguous group of chunks.
 // (1) each thread sums its chunk group; (2) warp-shuffle exclusive scan of the 32 group sums of
 // each expert; (3) each thread rewrites its chunk counts as exclusive offsets; the expert total
 // is cnt[e].  The CTA that finishes last (an atomic ticket after a fence; nothing waits) then
-// (4) scans align_up(cnt, A) and the padding rows over all experts and (5) restarts psum at
-// every rank.
+// scans align_up(cnt, A) and the padding rows over all experts and restarts psum at every rank.
 __global__ void __launch_bounds__(kScanThreads) k_layout_scan(LayoutLaunch L, int64_t cap_check) {
   __shared__ int32_t gsum[32][33];
-  __shared__ int32_t warp_tot[32];
-  __shared__ int32_t totals[2];
   __shared__ int32_t is_last;
   extern __shared__ int32_t sm[];
   const int E = L.E;
@@ -139,6 +298,8 @@ __global__ void __launch_bounds__(kScanThreads) k_layout_scan(LayoutLaunch L, in
   const int C = L.num_chunks;
   const int cpw = (C + 31) / 32;  // chunks per warp
   const int c0 = min(C, warp * cpw), c1 = min(C, c0 + cpw);
+  grid_dependents_launch();
+  grid_dependency_wait();  // chunk counts of the count kernel
 
   int32_t sum = 0;
   if (e < E)
@@ -177,61 +338,23 @@ __global__ void __launch_bounds__(kScanThreads) k_layout_scan(LayoutLaunch L, in
   if (!is_last) return;
   __threadfence();
   if (tid == 0) *L.d.ticket = 0;  // ready for the next layout on this scratch
-
-  int32_t* al = sm;             // [E] align_up(cnt, A)
-  int32_t* pad = sm + E;        // [E] align_up(cnt, A) - cnt
-  int32_t* gincl = sm + 2 * E;  // [E] inclusive prefix of al over all experts
-  for (int x = tid; x < E; x += blockDim.x) {
-    const int32_t n = __ldcg(L.d.cnt + x);
-    al[x] = align_up_dev(n, L.A);
-    pad[x] = al[x] - n;
-  }
-  __syncthreads();
-  const int per = (E + blockDim.x - 1) / blockDim.x;
-  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
-  int32_t sa = 0, sp = 0;
-  for (int x = e0; x < e1; ++x) {
-    sa += al[x];
-    sp += pad[x];
-  }
-  int32_t ra = block_exclusive_scan(sa, warp_tot, &totals[0]);
-  int32_t rp = block_exclusive_scan(sp, warp_tot, &totals[1]);
-  for (int x = e0; x < e1; ++x) {
-    L.d.pad_excl[x] = rp;
-    rp += pad[x];
-    ra += al[x];
-    gincl[x] = ra;
-  }
-  if (tid == 0) L.d.pad_excl[E] = totals[1];
-  __syncthreads();
-  for (int x = tid; x < E; x += blockDim.x) {
-    const int first = (x / L.E_loc) * L.E_loc;
-    L.d.psum[x] = gincl[x] - (gincl[first] - al[first]);
-  }
-  for (int r = tid; r < L.R; r += blockDim.x) {
-    const int first = r * L.E_loc, last = first + L.E_loc - 1;
-    const int32_t nrows = gincl[last] - (gincl[first] - al[first]);
-    L.d.rows_per_rank[r] = nrows;
-    if (cap_check > 0 && nrows > cap_check) atomicOr(L.d.status, kStatusCapacity);
-  }
+  block_psum<true>(L, L.d.cnt, cap_check, sm, sm + E, sm + 2 * E, nullptr, nullptr);
 }
 
 // ------------------------------------------------------------------------------------ assign
-// A CTA per chunk of tokens, 8 warps; warp w takes a contiguous run of the chunk's (t, j) pairs
-// and loads its expert ids kAssignBatch rounds of 32 at a time.  Phase 1: per-warp histogram
-// (__match_any_sync groups equal ids inside a round; the group leader adds its size).  Phase 2:
-// per expert, exclusive scan across warps based at the expert's first row for this chunk.
-// Phase 3: walk the pairs again; a pair's row = its warp's running base + its rank among equal
-// ids of lower lanes in the round.
-constexpr int kAssignBatch = 8;
-
+// A CTA per chunk of tokens, 8 warps; warp w takes a contiguous run of the chunk's (t, j) pairs.
+// Phase 1: per-warp histogram (__match_any_sync groups equal ids inside a round; the group
+// leader adds its size).  Phase 2: per expert, exclusive scan across warps based at the
+// expert's first row for this chunk.  Phase 3: a pair's row = its warp's running base + its rank
+// among equal ids of lower lanes in the round.
 __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L) {
   extern __shared__ int32_t whist[];  // [kLayoutWarps][E]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = L.E;
   int32_t* h = whist + warp * E;
-  const uint32_t lt = lanemask_lt();
   bool overflow = false;
+  grid_dependents_launch();
+  grid_dependency_wait();  // offsets, counts and psum of the scan kernel
 
   for (int c = blockIdx.x; c < L.num_chunks; c += gridDim.x) {
     const int64_t t0 = (int64_t)c * kChunkTokens;
@@ -240,26 +363,10 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L
     const int64_t per = (np + kLayoutWarps - 1) / kLayoutWarps;
     const int64_t wp0 = p0 + min(np, warp * per), wp1 = p0 + min(np, (warp + 1) * per);
 
-    // phase 1: this warp's histogram of its pairs
     for (int e = lane; e < E; e += 32) h[e] = 0;
     __syncwarp();
-    for (int64_t base = wp0; base < wp1; base += 32 * kAssignBatch) {
-      int32_t ev[kAssignBatch];
-#pragma unroll
-      for (int r = 0; r < kAssignBatch; ++r) {
-        const int64_t p = base + r * 32 + lane;
-        ev[r] = p < wp1 ? max(expert_of(__ldg(L.idx + p), E), -1) : -1;
-      }
-#pragma unroll
-      for (int r = 0; r < kAssignBatch; ++r) {
-        const uint32_t peers = __match_any_sync(0xffffffffu, ev[r]);
-        if (ev[r] >= 0 && lane == __ffs(peers) - 1) h[ev[r]] += __popc(peers);
-        __syncwarp();
-      }
-    }
+    warp_histogram(L, wp0, wp1, h);
     __syncthreads();
-
-    // phase 2: per expert, exclusive scan across warps
     for (int e = tid; e < E; e += blockDim.x) {
       int32_t base = L.d.psum[e] - align_up_dev(L.d.cnt[e], L.A) + L.d.chunk_cnt[(int64_t)c * E + e];
       for (int w = 0; w < kLayoutWarps; ++w) {
@@ -269,67 +376,81 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L
       }
     }
     __syncthreads();
-
-    // phase 3: rows in (t, j) order
-    for (int64_t base = wp0; base < wp1; base += 32 * kAssignBatch) {
-      int32_t ev[kAssignBatch];
-      float wv[kAssignBatch];
-#pragma unroll
-      for (int r = 0; r < kAssignBatch; ++r) {
-        const int64_t p = base + r * 32 + lane;
-        ev[r] = p < wp1 ? max(expert_of(__ldg(L.idx + p), E), -1) : -1;
-        wv[r] = (p < wp1 && L.w) ? __ldg(L.w + p) : 0.0f;
-      }
-#pragma unroll
-      for (int r = 0; r < kAssignBatch; ++r) {
-        const int64_t p = base + r * 32 + lane;
-        const int32_t e = ev[r];
-        const uint32_t peers = __match_any_sync(0xffffffffu, e);
-        int32_t row = -1;
-        if (e >= 0) row = h[e] + __popc(peers & lt);
-        __syncwarp();
-        if (e >= 0 && lane == __ffs(peers) - 1) h[e] += __popc(peers);
-        __syncwarp();
-        if (p < wp1) {
-          L.d.slot[p] = row;
-          L.d.pair_rank[p] = e >= 0 ? e / L.E_loc : -1;
-          L.d.pair_w[p] = wv[r];
-          if (e >= 0) {
-            const int rk = e / L.E_loc;
-            if (row < L.row_cap) {
-              L.d.row_src[(int64_t)rk * L.row_cap + row] = (int32_t)(p / L.k);
-              L.d.row_w[(int64_t)rk * L.row_cap + row] = wv[r];
-            } else {
-              overflow = true;
-            }
-          }
-        }
-      }
-    }
+    overflow |= warp_assign(L, wp0, wp1, h);
     __syncthreads();
   }
-
-  // padding rows of the row maps: global padding index i -> expert by binary search
-  const int32_t total_pad = L.d.pad_excl[E];
-  for (int32_t i = blockIdx.x * blockDim.x + tid; i < total_pad; i += gridDim.x * blockDim.x) {
-    int lo = 0, hi = E;  // largest e with pad_excl[e] <= i
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (L.d.pad_excl[mid] <= i) lo = mid;
-      else hi = mid;
-    }
-    const int e = lo;
-    const int32_t pad_e = L.d.pad_excl[e + 1] - L.d.pad_excl[e];
-    const int32_t row = L.d.psum[e] - pad_e + (i - L.d.pad_excl[e]);
-    const int r = e / L.E_loc;
-    if (row < L.row_cap) {
-      L.d.row_src[(int64_t)r * L.row_cap + row] = -1;
-      L.d.row_w[(int64_t)r * L.row_cap + row] = 0.0f;
-    } else {
-      overflow = true;
-    }
-  }
+  overflow |= row_map_padding(L, L.d.pad_excl, L.d.psum, (int64_t)blockIdx.x * kLayoutWarps + warp,
+                              (int64_t)gridDim.x * kLayoutWarps);
   if (overflow) atomicOr(L.d.status, kStatusCapacity);
+}
+
+// ------------------------------------------------------------------------------------ small
+// The whole layout in one CTA of 32 warps, for small batches (T * k <= kSmallPairs and
+// E <= kSmallMaxExperts, e.g. decode): membership and id checks, per-warp histograms of
+// token-aligned pair ranges, cross-warp scan, psum, slots and row maps, all through shared
+// memory, in one launch.  The results equal those of count -> scan -> assign.
+__global__ void __launch_bounds__(kSmallThreads) k_layout_small(LayoutLaunch L, int64_t cap_check) {
+  extern __shared__ int32_t sm[];
+  const int E = L.E, tid = threadIdx.x, warp = tid >> 5;
+  constexpr int W = kSmallThreads / 32;
+  int32_t* whist = sm;                  // [W][E]
+  int32_t* al = whist + W * E;          // [E]
+  int32_t* pad = al + E;                // [E]
+  int32_t* gincl = pad + E;             // [E]
+  int32_t* psum_s = gincl + E;          // [E]
+  int32_t* pad_s = psum_s + E;          // [E + 1]
+  int32_t* cnt_s = pad_s + E + 1;       // [E]
+  int32_t* tok = cnt_s + E;             // [R]
+  grid_dependents_launch();
+
+  for (int i = tid; i < W * E; i += blockDim.x) whist[i] = 0;
+  for (int r = tid; r < L.R; r += blockDim.x) tok[r] = 0;
+  __syncthreads();
+
+  bool ok = true;
+  for (int64_t tb = 0; tb < L.T; tb += blockDim.x) {  // same trip count for every thread
+    const int64_t t = tb + tid;
+    ok &= token_membership(L, t, t < L.T, nullptr, tok);
+  }
+  if (!ok) atomicOr(L.d.status, kStatusBadExpert);
+
+  // token-aligned pair range of this warp
+  const int64_t tpw = (L.T + W - 1) / W;
+  const int64_t wp0 = min(L.T, warp * tpw) * L.k, wp1 = min(L.T, (warp + 1) * tpw) * L.k;
+  int32_t* h = whist + warp * E;
+  warp_histogram(L, wp0, wp1, h);
+  __syncthreads();
+
+  for (int e = tid; e < E; e += blockDim.x) {  // exclusive scan across warps; cnt = total
+    int32_t run = 0;
+    for (int w = 0; w < W; ++w) {
+      const int32_t v = whist[w * E + e];
+      whist[w * E + e] = run;
+      run += v;
+    }
+    cnt_s[e] = run;
+    L.d.cnt[e] = run;
+  }
+  for (int r = tid; r < L.R; r += blockDim.x) L.d.tokens_per_rank[r] = tok[r];
+  __syncthreads();
+  block_psum<false>(L, cnt_s, cap_check, al, pad, gincl, pad_s, psum_s);
+
+  for (int e = tid; e < E; e += blockDim.x) {  // base every warp's rows at the segment start
+    const int32_t seg = psum_s[e] - al[e];
+    for (int w = 0; w < W; ++w) whist[w * E + e] += seg;
+  }
+  __syncthreads();
+  bool overflow = warp_assign(L, wp0, wp1, h);
+  overflow |= row_map_padding(L, pad_s, psum_s, warp, W);
+  if (overflow) atomicOr(L.d.status, kStatusCapacity);
+}
+
+bool layout_fits_one_cta(int64_t T, int k, int E) {
+  return T * k <= kSmallPairs && E <= kSmallMaxExperts;
+}
+
+size_t small_layout_smem(int E, int R) {
+  return sizeof(int32_t) * ((size_t)(kSmallThreads / 32) * E + 6 * (size_t)E + 1 + R);
 }
 
 // ------------------------------------------------------------------------------------ launch
@@ -342,6 +463,9 @@ static cudaError_t ensure_smem_attrs() {
   if (dev < 64 && (done >> dev) & 1ull) return cudaSuccess;
   err = cudaFuncSetAttribute(k_layout_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(sizeof(int32_t) * 3 * kMaxExperts));
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(k_layout_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)small_layout_smem(kSmallMaxExperts, kSmallMaxExperts));
   if (err == cudaSuccess)
     err = cudaFuncSetAttribute(k_layout_assign, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(sizeof(int32_t) * kLayoutWarps * kMaxExperts));
@@ -357,13 +481,21 @@ cudaError_t launch_layout_count(const LayoutLaunch& L, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+cudaError_t launch_layout_small(const LayoutLaunch& L, int64_t cap_check, cudaStream_t s) {
+  cudaError_t err = ensure_smem_attrs();
+  if (err != cudaSuccess) return err;
+  k_layout_small<<<1, kSmallThreads, small_layout_smem(L.E, L.R), s>>>(L, cap_check);
+  note_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_layout_scan(const LayoutLaunch& L, int64_t cap_check, cudaStream_t s) {
   cudaError_t err = ensure_smem_attrs();
   if (err != cudaSuccess) return err;
   const size_t smem = sizeof(int32_t) * 3 * (size_t)L.E;
-  k_layout_scan<<<(L.E + 31) / 32, kScanThreads, smem, s>>>(L, cap_check);
+  err = launch_pdl(k_layout_scan, dim3((L.E + 31) / 32), dim3(kScanThreads), smem, s, L, cap_check);
   note_launch();
-  return cudaGetLastError();
+  return err;
 }
 
 cudaError_t launch_layout_assign(const LayoutLaunch& L, cudaStream_t s) {
@@ -371,9 +503,9 @@ cudaError_t launch_layout_assign(const LayoutLaunch& L, cudaStream_t s) {
   if (err != cudaSuccess) return err;
   const size_t smem = sizeof(int32_t) * (size_t)kLayoutWarps * L.E;
   const int grid = L.grid_chunks > 0 ? L.grid_chunks : 1;
-  k_layout_assign<<<grid, kLayoutThreads, smem, s>>>(L);
+  err = launch_pdl(k_layout_assign, dim3(grid), dim3(kLayoutThreads), smem, s, L);
   note_launch();
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace moe

@@ -19,7 +19,7 @@
 // it.  That first call should come before any stream capture.
 //
 // Nothing here calls cudaMalloc, cudaMallocAsync, cudaMallocHost, cudaFree or any allocating
-// library routine; the three layout kernels are the ones moe_layout launches.
+// library routine; the layout kernels are the ones moe_layout launches.
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -120,11 +120,16 @@ extern "C" int moe_layout_static_scratch(const moe_params_t* p, const int64_t* t
   L.d = d;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool one_cta = layout_fits_one_cta(T, (int)k, (int)E);
   cudaError_t err = cudaMemsetAsync(d.status, 0, sizeof(int32_t), s);
   if (err == cudaSuccess) err = cudaMemsetAsync(d.ticket, 0, sizeof(int32_t), s);
   if (err == cudaSuccess) err = cudaMemsetAsync(tokens_per_rank, 0, sizeof(int32_t) * (size_t)R, s);  // summed atomically
-  if (err == cudaSuccess) err = launch_layout_count(L, s);
-  if (err == cudaSuccess) err = launch_layout_scan(L, p->recv_capacity_rows, s);
+  if (one_cta) {
+    if (err == cudaSuccess) err = launch_layout_small(L, p->recv_capacity_rows, s);
+  } else {
+    if (err == cudaSuccess) err = launch_layout_count(L, s);
+    if (err == cudaSuccess) err = launch_layout_scan(L, p->recv_capacity_rows, s);
+  }
   if (err != cudaSuccess) return MOE_ERR_CUDA;
 
   if (p->do_cpu_sync) {
@@ -138,5 +143,6 @@ extern "C" int moe_layout_static_scratch(const moe_params_t* p, const int64_t* t
     if (flags & kStatusBadExpert) return MOE_ERR_BAD_EXPERT;
     if (flags & kStatusCapacity) return MOE_ERR_CAPACITY;
   }
+  if (one_cta) return MOE_OK;
   return launch_layout_assign(L, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -203,9 +203,13 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
 
   // count -> scan -> assign back to back; with do_cpu_sync one host wait at the end
   cudaError_t err = cudaMemsetAsync(d.status, 0, (size_t)(32 + 4 * R), s);
-  if (err == cudaSuccess) err = launch_layout_count(L, s);
-  if (err == cudaSuccess) err = launch_layout_scan(L, p->recv_capacity_rows, s);
-  if (err == cudaSuccess) err = launch_layout_assign(L, s);
+  if (layout_fits_one_cta(T, (int)k, (int)E)) {
+    if (err == cudaSuccess) err = launch_layout_small(L, p->recv_capacity_rows, s);
+  } else {
+    if (err == cudaSuccess) err = launch_layout_count(L, s);
+    if (err == cudaSuccess) err = launch_layout_scan(L, p->recv_capacity_rows, s);
+    if (err == cudaSuccess) err = launch_layout_assign(L, s);
+  }
   if (err != cudaSuccess) {
     release(h);
     return MOE_ERR_CUDA;

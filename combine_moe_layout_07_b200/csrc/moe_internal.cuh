@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
 #include <vector>
 
 #include "moe.h"
@@ -27,6 +28,9 @@ constexpr int kChunkTokens = 256;
 constexpr int kLayoutThreads = 256;
 constexpr int kLayoutWarps = kLayoutThreads / 32;
 constexpr int kScanThreads = 1024;
+constexpr int kSmallThreads = 1024;     // the one-CTA layout for small batches
+constexpr int kSmallPairs = 8192;       // ... used when T * k <= kSmallPairs
+constexpr int kSmallMaxExperts = 1024;  // ... and E <= kSmallMaxExperts
 constexpr int kMaxExperts = 4096;
 constexpr int kMaxTopk = 32;
 
@@ -80,6 +84,8 @@ struct LayoutLaunch {
 cudaError_t launch_layout_count(const LayoutLaunch& L, cudaStream_t s);
 cudaError_t launch_layout_scan(const LayoutLaunch& L, int64_t cap_check, cudaStream_t s);
 cudaError_t launch_layout_assign(const LayoutLaunch& L, cudaStream_t s);
+cudaError_t launch_layout_small(const LayoutLaunch& L, int64_t cap_check, cudaStream_t s);
+bool layout_fits_one_cta(int64_t T, int k, int E);
 
 struct DispatchLaunch {
   const void* x;
@@ -119,6 +125,37 @@ cudaError_t launch_combine(const CombineLaunch& L, cudaStream_t s);
 
 void note_launch(int n = 1);
 int sm_count(int device);
+
+// Raise a kernel's dynamic shared-memory limit once per device (the attribute is per function).
+template <typename Kernel>
+cudaError_t set_smem_limit_once(Kernel kernel, int bytes, unsigned long long* done_mask) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 64 && ((*done_mask >> dev) & 1ull)) return cudaSuccess;
+  err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err == cudaSuccess && dev < 64) *done_mask |= 1ull << dev;
+  return err;
+}
+
+// Launch with programmatic stream serialization: the kernel may be scheduled while the
+// previous kernel in the stream finishes; it calls grid_dependency_wait() before it reads
+// anything that kernel wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ------------------------------------------------------------------------------ device helpers
 
@@ -164,6 +201,16 @@ __device__ __forceinline__ bool dbg_ok(bool cond, int32_t* status, int32_t code,
     status[3] = (int32_t)(detail >> 32);
   }
   return false;
+}
+
+// Wait until the previous kernel in the stream has completed and its writes are visible (a no-op
+// when the kernel was not launched as a programmatic dependent).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next kernel in the stream to be scheduled (it still waits for this one to finish
+// before reading its results).
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t lanemask_lt() {

@@ -109,6 +109,10 @@ def test_small_fp8_roundtrip(hidden, zero_padding):
     dict(hidden=136),                                    # ragged vector tail in the warp loop
     dict(experts=512, ranks=8, topk=8, tokens_per_rank=700, alignment=128),
     dict(hidden=7168, tokens_per_rank=300, experts=32, ranks=4, topk=8),   # several column chunks
+    dict(tokens_per_rank=1024, ranks=1, experts=8, topk=8),   # 8192 pairs: one-CTA layout
+    dict(tokens_per_rank=1025, ranks=1, experts=8, topk=8),   # 8200 pairs: three-kernel layout
+    dict(experts=128, ranks=128, topk=4, tokens_per_rank=2),  # more than 64 ranks (membership)
+    dict(experts=128, ranks=128, topk=4, tokens_per_rank=70), # ... on the three-kernel layout
     dict(hidden=4104, tokens_per_rank=200, experts=16, ranks=2, topk=3),   # ragged last chunk
 ])
 def test_shapes_and_edges(kw):
