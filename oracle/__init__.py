@@ -50,6 +50,9 @@ def lib() -> ctypes.CDLL:
         L.oracle_bf16_to_float.restype = ctypes.c_float
         L.oracle_quantize_block.argtypes = [_P, _I32, _P, _P]
         L.oracle_quantize_block.restype = None
+        L.oracle_combine_backward.argtypes = [_I64, _I32, _I32, _I32, _I32, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I32]
+        L.oracle_grad_weights_f64.argtypes = [_I64, _I32, _I32, _I32, _I64, _I64, _P, _P, _P, _P, _P]
+        L.oracle_grad_weights_f64.restype = None
         _lib = L
     return _lib
 
@@ -192,3 +195,31 @@ def float_to_bf16(v: float) -> int:
 
 def bf16_to_float(b: int) -> float:
     return float(lib().oracle_bf16_to_float(int(b)))
+
+
+def combine_backward(lay: Layout, idx, grad_out_bits, E: int, R: int, A: int, cap: int, w=None,
+                     zero_padding: bool = True, fill: int = 0xA5A5):
+    """Backward of combine: (status, grad_y uint16 [R, cap, H]) -- grad_out scattered to every
+    routed row, scaled by the pair weight (one fp32 multiply, bf16 rounding) when w is given."""
+    idx = _c(idx, np.int64)
+    g = _c(grad_out_bits, np.uint16)
+    w = _c(w, np.float32)
+    T, k = idx.shape
+    H = g.shape[1]
+    gy = np.full((R, cap, H), fill, np.uint16)
+    st = lib().oracle_combine_backward(T, k, E, R, A, H, cap, _p(idx), _p(lay.cnt), _p(lay.psum), _p(lay.slot),
+                                       _p(g), _p(w), _p(gy), int(zero_padding))
+    return st, gy
+
+
+def grad_weights_f64(idx, slot, grad_out_bits, y_bits, E: int, R: int) -> np.ndarray:
+    """grad_w[t, j] = <grad_out[t], y[row(t, j)]> in binary64 (0 for masked pairs)."""
+    idx = _c(idx, np.int64)
+    slot = _c(slot, np.int32)
+    g = _c(grad_out_bits, np.uint16)
+    y = _c(y_bits, np.uint16)
+    T, k = idx.shape
+    _, cap, H = y.shape
+    gw = np.zeros((T, k), np.float64)
+    lib().oracle_grad_weights_f64(T, k, E, R, H, cap, _p(idx), _p(slot), _p(g), _p(y), _p(gw))
+    return gw

@@ -404,3 +404,57 @@ void oracle_combine_f64(int64_t T, int k, int E, int R, int64_t H, int64_t cap,
             out64[t * H + h] = acc;
         }
 }
+
+/* ---------------------------------------------------------------------------------------
+ * Backward of combine  ["Why MoE gets stuck on communication" s1 and s2: the handle records one
+ * dispatch's grouping and counts and training reuses it in the backward pass]
+ * For out[t] = sum_j w[t,j] * y[slot(t,j)] (+ bias[t]):
+ *   grad_y[slot(t,j)] = bf16(w[t,j] * grad_out[t])   (one fp32 multiply, then bf16 RNE);
+ *                     = grad_out[t]                   when the rows were pre-weighted (w NULL);
+ *   padding rows of grad_y are zero when do_zero_padding, other rows untouched.
+ * grad_y is [R, cap, H] bf16.
+ * ------------------------------------------------------------------------------------- */
+int oracle_combine_backward(int64_t T, int k, int E, int R, int A, int64_t H, int64_t cap,
+                            const int64_t* idx, const int32_t* cnt, const int32_t* psum,
+                            const int32_t* slot, const uint16_t* grad_out, const float* w,
+                            uint16_t* grad_y, int do_zero_padding) {
+    const int E_loc = E / R;
+    int status = ORC_OK;
+    for (int64_t t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            int32_t row = slot[t * k + j];
+            if (row < 0) continue;
+            if (row >= cap) { status = ORC_ERR_CAPACITY; continue; }
+            int r = (int)(idx[t * k + j] / E_loc);
+            uint16_t* dst = grad_y + ((int64_t)r * cap + row) * H;
+            for (int64_t h = 0; h < H; ++h) {
+                uint16_t g = grad_out[t * H + h];
+                dst[h] = w ? oracle_float_to_bf16(w[t * k + j] * oracle_bf16_to_float(g)) : g;
+            }
+        }
+    if (do_zero_padding) {
+        pad_ctx c = { (uint8_t*)grad_y, cap, H * 2, NULL, cap };
+        for_each_padding_row(E, R, A, cnt, psum, zero_row, &c);
+    }
+    return status;
+}
+
+/* Gradient of the combine with respect to the pair weights: grad_w[t,j] = sum_h grad_out[t,h] *
+ * y[slot(t,j), h] in binary64 (0 for masked pairs). */
+void oracle_grad_weights_f64(int64_t T, int k, int E, int R, int64_t H, int64_t cap,
+                             const int64_t* idx, const int32_t* slot, const uint16_t* grad_out,
+                             const uint16_t* y, double* grad_w) {
+    const int E_loc = E / R;
+    for (int64_t t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            int32_t row = slot[t * k + j];
+            double acc = 0.0;
+            if (row >= 0 && row < cap) {
+                int r = (int)(idx[t * k + j] / E_loc);
+                const uint16_t* yr = y + ((int64_t)r * cap + row) * H;
+                for (int64_t h = 0; h < H; ++h)
+                    acc += (double)oracle_bf16_to_float(grad_out[t * H + h]) * (double)oracle_bf16_to_float(yr[h]);
+            }
+            grad_w[t * k + j] = acc;
+        }
+}

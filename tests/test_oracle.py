@@ -377,3 +377,69 @@ def test_bf16_rounding_definition():
     assert oracle.float_to_bf16(float("nan")) == 0x7FC0
     # ties: 1 + 2^-8 is halfway between 1 and 1 + 2^-7 -> even (1.0)
     assert oracle.float_to_bf16(1.00390625) == 0x3F80
+
+
+# ----------------------------------------------------------------------------- backward of combine
+
+def _bwd_case(mask=0.1, topk=4):
+    wl, idx, w, x = _tiny(mask, topk=topk)
+    E, R, A = wl.experts, wl.ranks, wl.alignment
+    lay = oracle.layout(idx, w, E, R, A)
+    cap = int(lay.rows_per_rank.max())
+    y = W.gen_y(wl, cap)
+    g = W.gen_bias(wl)          # any bf16 [T, H] tensor serves as grad_out
+    return wl, idx, w, lay, cap, bits(y), bits(g)
+
+
+def test_combine_backward_unweighted_is_the_bf16_dispatch_of_grad_out():
+    wl, idx, w, lay, cap, y, g = _bwd_case()
+    E, R, A = wl.experts, wl.ranks, wl.alignment
+    st, gy = oracle.combine_backward(lay, idx, g, E, R, A, cap, w=None)
+    st2, ref, _ = oracle.dispatch_bf16(lay, idx, w, g, E, R, A, cap, True)
+    assert st == st2 == oracle.OK
+    assert (gy == ref).all()
+
+
+def test_combine_backward_is_the_adjoint_of_combine():
+    """<g, C(y)> == <C^T(g), y> in binary64, up to the bf16 rounding of grad_y (weighted case)."""
+    wl, idx, w, lay, cap, y, g = _bwd_case()
+    E, R = wl.experts, wl.ranks
+    out64 = oracle.combine_f64(idx, lay.slot, y, E, R, w=w)
+    lhs = float(((g.astype(np.uint32) << 16).view(np.float32).astype(np.float64) * out64).sum())
+    st, gy = oracle.combine_backward(lay, idx, g, E, R, wl.alignment, cap, w=w, fill=0)
+    gyf = (gy.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    yf = (y.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    rhs = float((gyf * yf).sum())
+    scale = float(np.abs(gyf * yf).sum())
+    assert abs(lhs - rhs) <= 2.0 ** -8 * scale
+    # and exactly: each grad_y row is the bf16 rounding of w * g for its (t, j)
+    e_loc = E // R
+    gf = (g.astype(np.uint32) << 16).view(np.float32)
+    for t in range(wl.tokens):
+        for j in range(wl.topk):
+            if idx[t, j] >= 0:
+                row = gy[idx[t, j] // e_loc, lay.slot[t, j]]
+                expect = bits(torch.from_numpy((np.float32(w[t, j]) * gf[t]).astype(np.float32)).to(torch.bfloat16))
+                assert (row == expect).all()
+
+
+def test_grad_weights_is_the_derivative_of_combine():
+    """Central finite difference of L(w) = <g, combine_f64(y; w)> reproduces grad_w (L is
+    linear in each weight, so the difference quotient is exact up to binary64 rounding)."""
+    wl, idx, w, lay, cap, y, g = _bwd_case()
+    E, R = wl.experts, wl.ranks
+    gw = oracle.grad_weights_f64(idx, lay.slot, g, y, E, R)
+    gf = (g.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    rng = np.random.default_rng(3)
+    for _ in range(12):
+        t, j = int(rng.integers(wl.tokens)), int(rng.integers(wl.topk))
+        h = 0.25
+        wp, wm = w.copy(), w.copy()
+        wp[t, j] += h
+        wm[t, j] -= h
+        lp = float((gf * oracle.combine_f64(idx, lay.slot, y, E, R, w=wp)).sum())
+        lm = float((gf * oracle.combine_f64(idx, lay.slot, y, E, R, w=wm)).sum())
+        fd = (lp - lm) / (float(wp[t, j]) - float(wm[t, j]))  # the weights are fp32: use the real step
+        assert abs(fd - gw[t, j]) <= 1e-9 * max(1.0, abs(gw[t, j])), (t, j, fd, gw[t, j])
+        if idx[t, j] < 0:
+            assert gw[t, j] == 0.0
