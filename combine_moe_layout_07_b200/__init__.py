@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
         L.moe_dispatch.argtypes = [_P, _P, _I32, _P, _P, _P, _I64, _I32, _I32, _I32, _P]
         L.moe_combine.argtypes = [_P, _P, _P, _P, _P, _I64, _I32, _P]
         L.moe_handle_status.argtypes = [_P, _P]
+        L.moe_combine_backward.argtypes = [_P, _P, _P, _P, _I64, _I32, _P, _P, _I32, _P]
         for name in ("counts", "psum", "rows_per_rank", "tokens_per_rank", "token_in_rank", "slots",
                      "row_src", "row_weights"):
             f = getattr(L, f"moe_handle_{name}")
@@ -207,6 +208,17 @@ def moe_combine(handle: Handle, y: torch.Tensor, out: torch.Tensor, topk_weights
     rc = lib().moe_combine(handle.ptr, _ptr(y), _ptr(topk_weights), _ptr(bias), _ptr(out), cap, num_sms,
                            _stream(stream))
     _check(rc, "moe_combine")
+
+
+def moe_combine_backward(handle: Handle, grad_out: torch.Tensor, grad_y: torch.Tensor,
+                         topk_weights: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                         grad_weights: Optional[torch.Tensor] = None, cap: Optional[int] = None,
+                         do_zero_padding: bool = True, num_sms: int = 0, stream=None) -> None:
+    """Backward of moe_combine: grad_y (and grad_weights when given, which needs y)."""
+    cap = grad_y.shape[1] if cap is None else cap
+    rc = lib().moe_combine_backward(handle.ptr, _ptr(grad_out), _ptr(topk_weights), _ptr(grad_y), cap,
+                                    int(do_zero_padding), _ptr(y), _ptr(grad_weights), num_sms, _stream(stream))
+    _check(rc, "moe_combine_backward")
 
 
 def moe_handle_status(handle: Handle, stream=None) -> int:

@@ -107,13 +107,14 @@ __global__ void __launch_bounds__(kDispThreads, 1) k_dispatch(DispatchLaunch L, 
     // pair metadata for tpb tokens per warp-wide load, prefetched one batch ahead
     const int tpb = 32 / L.k, lanes_used = tpb * L.k;
     const int64_t p_end = t_end * L.k;
-    PairBatch cur = load_pair_batch(L.pair_rank, L.slot, L.pair_w, t_begin * L.k, p_end, lane, lanes_used);
+    const float* wsrc = L.scale_w ? L.scale_w : L.pair_w;
+    PairBatch cur = load_pair_batch(L.pair_rank, L.slot, wsrc, t_begin * L.k, p_end, lane, lanes_used);
     int64_t i = 0;
     int s = 0;
     uint32_t par = 0;  // (i / S) & 1
     bool stop = false;
     for (int64_t tb = t_begin; tb < t_end && !stop; tb += tpb) {
-      const PairBatch nxt = load_pair_batch(L.pair_rank, L.slot, L.pair_w, (tb + tpb) * L.k, p_end, lane, lanes_used);
+      const PairBatch nxt = load_pair_batch(L.pair_rank, L.slot, wsrc, (tb + tpb) * L.k, p_end, lane, lanes_used);
       const int nt = (int)min((int64_t)tpb, t_end - tb);
       for (int q = 0; q < nt; ++q) {
         const int64_t t = tb + q;
@@ -223,9 +224,18 @@ __global__ void __launch_bounds__(kDispThreads, 1) k_dispatch(DispatchLaunch L, 
         const int64_t nvec = H / 8;  // 16-byte vectors per bf16 row
         for (int64_t v = gtid; v < nvec; v += kDispGroupThreads) {
           const uint4 d = lds_v4(in_s + (uint32_t)v * 16);
-          for (int j = 0; j < n; ++j)
-            if (dbg_ok(M.row[j] >= 0 && M.row[j] < L.R * L.cap, L.status, 203, M.row[j]))
-              st_stream_v4(static_cast<uint16_t*>(L.recv_x) + M.row[j] * H + v * 8, d);
+          for (int j = 0; j < n; ++j) {
+            if (!dbg_ok(M.row[j] >= 0 && M.row[j] < L.R * L.cap, L.status, 203, M.row[j])) continue;
+            uint4 o = d;
+            if (L.scale_w) {  // backward of a weighted combine: bf16(w * g), one fp32 multiply
+              const float wj = M.w[j];
+              o.x = pack_bf16x2(__fmul_rn(wj, bf16lo(d.x)), __fmul_rn(wj, bf16hi(d.x)));
+              o.y = pack_bf16x2(__fmul_rn(wj, bf16lo(d.y)), __fmul_rn(wj, bf16hi(d.y)));
+              o.z = pack_bf16x2(__fmul_rn(wj, bf16lo(d.z)), __fmul_rn(wj, bf16hi(d.z)));
+              o.w = pack_bf16x2(__fmul_rn(wj, bf16lo(d.w)), __fmul_rn(wj, bf16hi(d.w)));
+            }
+            st_stream_v4(static_cast<uint16_t*>(L.recv_x) + M.row[j] * H + v * 8, o);
+          }
         }
       }
       if (L.recv_w && gtid < n) L.recv_w[M.row[gtid]] = M.w[gtid];

@@ -316,6 +316,62 @@ int moe_combine(const moe_handle_t* h, const void* y, const float* topk_weights,
   return launch_combine(L, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+int moe_combine_backward(const moe_handle_t* h, const void* grad_out, const float* topk_weights, void* grad_y,
+                         int64_t cap, int do_zero_padding, const void* y, float* grad_weights, int num_sms,
+                         void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (cap < 0 || cap >= (int64_t)1 << 31 || num_sms < 0) return MOE_ERR_INVALID_ARG;
+  if (do_zero_padding != 0 && do_zero_padding != 1) return MOE_ERR_INVALID_ARG;
+  const moe_params_t& p = h->p;
+  if (p.num_tokens > 0 && (!grad_out || !grad_y)) return MOE_ERR_INVALID_ARG;
+  if (grad_weights && !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(grad_out) || !aligned16(grad_y) || !aligned16(y) || !aligned4(topk_weights) ||
+      !aligned4(grad_weights))
+    return MOE_ERR_INVALID_ARG;
+  if (h->counts_on_host) {
+    for (int32_t v : h->host_rows)
+      if (v > cap) return MOE_ERR_CAPACITY;
+  }
+  if (p.num_tokens == 0) return MOE_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DispatchLaunch D{};
+  D.x = grad_out;
+  D.recv_x = grad_y;
+  D.T = p.num_tokens;
+  D.cap = cap;
+  D.H = p.hidden;
+  D.R = p.num_logical_ranks;
+  D.k = p.topk;
+  D.E = p.num_experts;
+  D.E_loc = p.num_experts / p.num_logical_ranks;
+  D.zero_padding = do_zero_padding;
+  D.grid = grid_for(num_sms, h->device);
+  D.pair_rank = h->d.pair_rank;
+  D.slot = h->d.slot;
+  D.pair_w = h->d.pair_w;
+  D.scale_w = topk_weights;
+  D.psum = h->d.psum;
+  D.pad_excl = h->d.pad_excl;
+  D.status = h->d.status;
+  if (launch_dispatch(D, false, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (grad_weights) {
+    GradWeightsLaunch G{};
+    G.grad_out = grad_out;
+    G.y = y;
+    G.grad_w = grad_weights;
+    G.T = p.num_tokens;
+    G.cap = cap;
+    G.H = p.hidden;
+    G.k = p.topk;
+    G.grid = 4 * grid_for(num_sms, h->device);
+    G.pair_rank = h->d.pair_rank;
+    G.slot = h->d.slot;
+    G.status = h->d.status;
+    if (launch_grad_weights(G, s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
 int moe_handle_status(const moe_handle_t* h, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -100,6 +100,7 @@ struct DispatchLaunch {
   const int32_t* pair_rank;
   const int32_t* slot;
   const float* pair_w;
+  const float* scale_w;  // BF16 rows only, nullable: each destination row is bf16(w[t,j] * x[t])
   const int32_t* psum;
   const int32_t* pad_excl;
   int32_t* status;
@@ -122,6 +123,20 @@ struct CombineLaunch {
 };
 
 cudaError_t launch_combine(const CombineLaunch& L, cudaStream_t s);
+
+struct GradWeightsLaunch {
+  const void* grad_out;  // bf16 [T, H]
+  const void* y;         // bf16 [R, cap, H]
+  float* grad_w;         // [T, k]
+  int64_t T, cap, H;
+  int k;
+  int grid;
+  const int32_t* pair_rank;
+  const int32_t* slot;
+  int32_t* status;
+};
+
+cudaError_t launch_grad_weights(const GradWeightsLaunch& L, cudaStream_t s);
 
 void note_launch(int n = 1);
 int sm_count(int device);

@@ -136,6 +136,24 @@ int moe_dispatch(const moe_handle_t* handle, const void* x, int out_dtype, void*
 int moe_combine(const moe_handle_t* handle, const void* y, const float* topk_weights,
                 const void* bias, void* out, int64_t cap, int num_sms, void* stream);
 
+/*
+ * Backward of combine ("Why MoE gets stuck on communication" 1 and 2: the handle of a dispatch is
+ * reused by the backward pass).  For out[t] = sum_j w[t,j] * y[row(t,j)] (+ bias[t]):
+ *   grad_out      bf16 [T, H], device.
+ *   topk_weights  fp32 [T, k], nullable: the weights the combine applied (NULL: pre-weighted rows).
+ *   grad_y        bf16 [R, cap, H]: grad_y[row(t,j)] = bf16(w[t,j] * grad_out[t]) (one fp32 multiply)
+ *                 or grad_out[t] when topk_weights is NULL; padding rows are zeroed when
+ *                 do_zero_padding, other rows beyond rows_per_rank are not written.
+ *   y             bf16 [R, cap, H], nullable: the combine's input, needed for grad_weights.
+ *   grad_weights  fp32 [T, k], nullable: grad_w[t,j] = <grad_out[t], y[row(t,j)]> (0 if masked),
+ *                 fp32 FMA per lane over columns in ascending order, then a fixed 32-lane tree.
+ * The gradient of the bias is grad_out itself.  The backward of dispatch is moe_combine with
+ * topk_weights = NULL applied to the gradient of the received rows.
+ */
+int moe_combine_backward(const moe_handle_t* handle, const void* grad_out, const float* topk_weights,
+                         void* grad_y, int64_t cap, int do_zero_padding, const void* y,
+                         float* grad_weights, int num_sms, void* stream);
+
 /* Waits for `stream`, then returns the handle's device status (MOE_OK, MOE_ERR_BAD_EXPERT,
  * MOE_ERR_CAPACITY or MOE_ERR_TIMEOUT) as left by every layout / dispatch / combine ordered
  * before it. */
