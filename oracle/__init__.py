@@ -53,6 +53,9 @@ def lib() -> ctypes.CDLL:
         L.oracle_combine_backward.argtypes = [_I64, _I32, _I32, _I32, _I32, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I32]
         L.oracle_grad_weights_f64.argtypes = [_I64, _I32, _I32, _I32, _I64, _I64, _P, _P, _P, _P, _P]
         L.oracle_grad_weights_f64.restype = None
+        L.oracle_layout_by_rank.argtypes = [_I64, _I32, _I32, _I32, _P, _P, _P]
+        L.oracle_dispatch_by_rank.argtypes = [_I64, _I32, _I32, _I32, _I64, _I64, _P, _P, _P, _P, _I32, _P, _P, _P, _P]
+        L.oracle_combine_by_rank.argtypes = [_I64, _I32, _I32, _I32, _I64, _I64, _P, _P, _P, _P, _P]
         _lib = L
     return _lib
 
@@ -223,3 +226,49 @@ def grad_weights_f64(idx, slot, grad_out_bits, y_bits, E: int, R: int) -> np.nda
     gw = np.zeros((T, k), np.float64)
     lib().oracle_grad_weights_f64(T, k, E, R, H, cap, _p(idx), _p(slot), _p(g), _p(y), _p(gw))
     return gw
+
+
+def layout_by_rank(idx, E: int, R: int):
+    """(status, token_row int32 [T, R], rows_per_rank int32 [R]) of the non-expanded layout."""
+    idx = _c(idx, np.int64)
+    T, k = idx.shape
+    tr = np.zeros((T, R), np.int32)
+    rows = np.zeros(R, np.int32)
+    st = lib().oracle_layout_by_rank(T, k, E, R, _p(idx), _p(tr), _p(rows))
+    return st, tr, rows
+
+
+def dispatch_by_rank(idx, w, token_row, x_bits, E: int, R: int, cap: int, fp8: bool, fill: int = 0xA5):
+    """By-rank dispatch: (status, recv [R, cap, H] (uint8 codes or uint16 bf16), scales or None,
+    recv_topk_idx int32 [R, cap, k], recv_topk_w fp32 [R, cap, k]); untouched entries keep fill /
+    -7 / NaN."""
+    idx = _c(idx, np.int64)
+    w = _c(w, np.float32)
+    tr = _c(token_row, np.int32)
+    x_bits = _c(x_bits, np.uint16)
+    T, k = idx.shape
+    H = x_bits.shape[1]
+    if fp8:
+        recv = np.full((R, cap, H), fill, np.uint8)
+        scales = np.full((R, cap, H // 128), np.nan, np.float32)
+    else:
+        recv = np.full((R, cap, H), fill | (fill << 8), np.uint16)
+        scales = None
+    ti = np.full((R, cap, k), -7, np.int32)
+    tw = np.full((R, cap, k), np.nan, np.float32)
+    st = lib().oracle_dispatch_by_rank(T, k, E, R, H, cap, _p(idx), _p(w), _p(tr), _p(x_bits), int(fp8), _p(recv),
+                                       _p(scales), _p(ti), _p(tw))
+    return st, recv, scales, ti, tw
+
+
+def combine_by_rank(idx, token_row, y_bits, E: int, R: int, bias_bits=None):
+    """By-rank combine: (status, out uint16 [T, H])."""
+    idx = _c(idx, np.int64)
+    tr = _c(token_row, np.int32)
+    y_bits = _c(y_bits, np.uint16)
+    bias_bits = _c(bias_bits, np.uint16)
+    T, k = idx.shape
+    _, cap, H = y_bits.shape
+    out = np.zeros((T, H), np.uint16)
+    st = lib().oracle_combine_by_rank(T, k, E, R, H, cap, _p(idx), _p(tr), _p(y_bits), _p(bias_bits), _p(out))
+    return st, out

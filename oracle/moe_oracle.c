@@ -458,3 +458,99 @@ void oracle_grad_weights_f64(int64_t T, int k, int E, int R, int64_t H, int64_t 
             grad_w[t * k + j] = acc;
         }
 }
+
+/* ---------------------------------------------------------------------------------------
+ * Non-expanded (by rank) round trip  ["Why MoE gets stuck on communication" s1: do_expand
+ * selects the expert-side expanded layout; without it every destination rank receives a token
+ * once; "Chapter 2: repository map" s2.1: layout.cu produces the token -> rank membership]
+ *
+ * token_row[t*R + r] = row of token t in rank r's buffer (tokens of rank r in ascending token
+ * order), -1 when none of t's experts lives on r.  rows_per_rank[r] = number of such tokens.
+ * ------------------------------------------------------------------------------------- */
+int oracle_layout_by_rank(int64_t T, int k, int E, int R, const int64_t* idx, int32_t* token_row,
+                          int32_t* rows_per_rank) {
+    if (T < 0 || k < 1 || E < 1 || R < 1 || E % R != 0) return ORC_ERR_INVALID_ARG;
+    const int E_loc = E / R;
+    int status = ORC_OK;
+    for (int r = 0; r < R; ++r) rows_per_rank[r] = 0;
+    for (int64_t t = 0; t < T; ++t)
+        for (int r = 0; r < R; ++r) {
+            int member = 0;
+            for (int j = 0; j < k; ++j) {
+                int64_t e = idx[t * k + j];
+                if (e < -1 || e >= E) status = ORC_ERR_BAD_EXPERT;
+                else if (e >= 0 && e / E_loc == r) member = 1;
+            }
+            token_row[t * R + r] = member ? rows_per_rank[r]++ : -1;
+        }
+    return status;
+}
+
+/* By-rank dispatch: recv[r, token_row[t,r]] = x[t] (BF16 copy, or FP8 codes + 1x128 scales with
+ * the block recipe of oracle_quantize_block).  recv_topk_idx[r, row, j] = e_j - r*E_loc when
+ * expert e_j lives on r, else -1; recv_topk_w[r, row, j] = w[t,j] or 0.  Either is nullable.
+ * fp8 == 0: recv is uint16 [R, cap, H]; fp8 == 1: recv is uint8 [R, cap, H] and scales
+ * [R, cap, H/128]. */
+int oracle_dispatch_by_rank(int64_t T, int k, int E, int R, int64_t H, int64_t cap, const int64_t* idx,
+                            const float* w, const int32_t* token_row, const uint16_t* x, int fp8, void* recv,
+                            float* recv_scales, int32_t* recv_topk_idx, float* recv_topk_w) {
+    const int E_loc = E / R;
+    const int64_t nb = H / 128;
+    int status = ORC_OK;
+    uint8_t* codes = (uint8_t*)malloc((size_t)(H > 0 ? H : 1));
+    float* scales = (float*)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    for (int64_t t = 0; t < T; ++t) {
+        if (fp8)
+            for (int64_t b = 0; b < nb; ++b) oracle_quantize_block(x + t * H + b * 128, 128, codes + b * 128, scales + b);
+        for (int r = 0; r < R; ++r) {
+            int32_t row = token_row[t * R + r];
+            if (row < 0) continue;
+            if (row >= cap) { status = ORC_ERR_CAPACITY; continue; }
+            int64_t g = (int64_t)r * cap + row;
+            if (fp8) {
+                memcpy((uint8_t*)recv + g * H, codes, (size_t)H);
+                memcpy(recv_scales + g * nb, scales, sizeof(float) * (size_t)nb);
+            } else {
+                memcpy((uint16_t*)recv + g * H, x + t * H, (size_t)H * 2);
+            }
+            for (int j = 0; j < k; ++j) {
+                int64_t e = idx[t * k + j];
+                int on_r = e >= 0 && e < E && e / E_loc == r;
+                if (recv_topk_idx) recv_topk_idx[g * k + j] = on_r ? (int32_t)(e - (int64_t)r * E_loc) : -1;
+                if (recv_topk_w) recv_topk_w[g * k + j] = on_r && w ? w[t * k + j] : 0.0f;
+            }
+        }
+    }
+    free(codes);
+    free(scales);
+    return status;
+}
+
+/* By-rank combine: y holds, per (token, rank), the rank's already-weighted partial sum.  For
+ * each element: acc = 0 (fp32); for every rank of the token, in the order in which the ranks
+ * first appear in topk_idx[t, :], acc += y[r, token_row[t,r]]; then acc + bias; bf16 RNE. */
+int oracle_combine_by_rank(int64_t T, int k, int E, int R, int64_t H, int64_t cap, const int64_t* idx,
+                           const int32_t* token_row, const uint16_t* y, const uint16_t* bias, uint16_t* out) {
+    const int E_loc = E / R;
+    int status = ORC_OK;
+    int* seen = (int*)malloc(sizeof(int) * (size_t)R);
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t h = 0; h < H; ++h) {
+            for (int r = 0; r < R; ++r) seen[r] = 0;
+            float acc = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                int64_t e = idx[t * k + j];
+                if (e < 0 || e >= E) continue;
+                int r = (int)(e / E_loc);
+                if (seen[r]) continue;
+                seen[r] = 1;
+                int32_t row = token_row[t * R + r];
+                if (row >= cap) { status = ORC_ERR_CAPACITY; continue; }
+                acc = acc + oracle_bf16_to_float(y[((int64_t)r * cap + row) * H + h]);
+            }
+            if (bias) acc = acc + oracle_bf16_to_float(bias[t * H + h]);
+            out[t * H + h] = oracle_float_to_bf16(acc);
+        }
+    free(seen);
+    return status;
+}

@@ -443,3 +443,68 @@ def test_grad_weights_is_the_derivative_of_combine():
         assert abs(fd - gw[t, j]) <= 1e-9 * max(1.0, abs(gw[t, j])), (t, j, fd, gw[t, j])
         if idx[t, j] < 0:
             assert gw[t, j] == 0.0
+
+
+# ----------------------------------------------------------------------------- non-expanded (by rank)
+
+def test_layout_by_rank_invariants():
+    wl, idx, w, x = _tiny(0.2, topk=4, experts=16, ranks=4)
+    st, tr, rows = oracle.layout_by_rank(idx, wl.experts, wl.ranks)
+    assert st == oracle.OK
+    e_loc = wl.experts // wl.ranks
+    lay = oracle.layout(idx, w, wl.experts, wl.ranks, wl.alignment)
+    assert (rows == lay.tokens_per_rank).all()          # one row per member token
+    for r in range(wl.ranks):
+        members = [t for t in range(wl.tokens) if any(e >= 0 and e // e_loc == r for e in idx[t])]
+        assert [int(tr[t, r]) for t in members] == list(range(len(members)))   # ascending tokens
+        assert all(tr[t, r] == -1 for t in range(wl.tokens) if t not in members)
+
+
+def test_by_rank_round_trip_equals_the_expanded_one():
+    """Two-level reduction: with per-(token, rank) partial sums built from an expanded expert
+    output, the by-rank combine equals the expanded combine in binary64 (then within one bf16
+    rounding of each other)."""
+    wl, idx, w, x = _tiny(0.15, topk=4, experts=16, ranks=4)
+    E, R, A = wl.experts, wl.ranks, wl.alignment
+    lay = oracle.layout(idx, w, E, R, A)
+    cap = int(lay.rows_per_rank.max())
+    y = bits(W.gen_y(wl, cap))
+    e_loc = E // R
+    st, tr, rows = oracle.layout_by_rank(idx, E, R)
+    yf = (y.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    part = np.zeros((R, int(rows.max()), wl.hidden))
+    for t in range(wl.tokens):
+        for j in range(wl.topk):
+            e = idx[t, j]
+            if e >= 0:
+                part[e // e_loc, tr[t, e // e_loc]] += w[t, j] * yf[e // e_loc, lay.slot[t, j]]
+    part_bits = bits(torch.from_numpy(part.astype(np.float32)).to(torch.bfloat16))
+    st, out_rank = oracle.combine_by_rank(idx, tr, part_bits, E, R)
+    ref = oracle.combine_f64(idx, lay.slot, y, E, R, w=w)
+    got = (out_rank.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    # each partial sum was rounded to bf16 once, the final sum once more
+    assert (np.abs(got - ref) <= 2.0 ** -7 * (np.abs(ref) + np.abs(part).max(axis=(0, 1)).max()) + 1e-6).all()
+
+
+def test_by_rank_dispatch_copies_and_topk_views():
+    wl, idx, w, x = _tiny(0.1, topk=4, experts=16, ranks=4, hidden=256)
+    E, R = wl.experts, wl.ranks
+    st, tr, rows = oracle.layout_by_rank(idx, E, R)
+    cap = int(rows.max())
+    st, recv, _, ti, tw = oracle.dispatch_by_rank(idx, w, tr, bits(x), E, R, cap, fp8=False)
+    e_loc = E // R
+    xb = bits(x)
+    for t in range(wl.tokens):
+        for r in range(R):
+            if tr[t, r] >= 0:
+                assert (recv[r, tr[t, r]] == xb[t]).all()
+                for j in range(wl.topk):
+                    e = idx[t, j]
+                    on = e >= 0 and e // e_loc == r
+                    assert ti[r, tr[t, r], j] == (e - r * e_loc if on else -1)
+                    assert tw[r, tr[t, r], j] == (w[t, j] if on else 0.0)
+    # identity expert: the by-rank combine of the received copies gives (#member ranks) * x
+    st, out = oracle.combine_by_rank(idx, tr, recv, E, R)
+    members = np.array([[tr[t, r] >= 0 for r in range(R)] for t in range(wl.tokens)]).sum(1)
+    expect = bits((x.float() * torch.from_numpy(members).float()[:, None]).to(torch.bfloat16))
+    assert (out == expect).all()
