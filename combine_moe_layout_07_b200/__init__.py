@@ -27,6 +27,7 @@ MOE_ERR_SCRATCH_LIMIT = -7
 MOE_ERR_TIMEOUT = -8
 MOE_DTYPE_BF16 = 0
 MOE_DTYPE_FP8_E4M3 = 1
+MOE_LAYOUT_BY_RANK = 1
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -47,16 +48,16 @@ class MoeParams(ctypes.Structure):
         ("expert_alignment", ctypes.c_int32),
         ("num_sms", ctypes.c_int32),
         ("do_cpu_sync", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("flags", ctypes.c_int32),
         ("recv_capacity_rows", ctypes.c_int64),
     ]
 
 
 def params(num_tokens: int, num_logical_ranks: int, num_experts: int, topk: int, hidden: int,
            expert_alignment: int, recv_capacity_rows: int = 0, num_sms: int = 0,
-           do_cpu_sync: bool = True) -> MoeParams:
+           do_cpu_sync: bool = True, by_rank: bool = False) -> MoeParams:
     return MoeParams(num_tokens, num_logical_ranks, num_experts, topk, hidden, expert_alignment,
-                     num_sms, int(do_cpu_sync), 0, recv_capacity_rows)
+                     num_sms, int(do_cpu_sync), MOE_LAYOUT_BY_RANK if by_rank else 0, recv_capacity_rows)
 
 
 _P, _I64, _I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
@@ -76,8 +77,10 @@ def lib() -> ctypes.CDLL:
         L.moe_combine.argtypes = [_P, _P, _P, _P, _P, _I64, _I32, _P]
         L.moe_handle_status.argtypes = [_P, _P]
         L.moe_combine_backward.argtypes = [_P, _P, _P, _P, _I64, _I32, _P, _P, _I32, _P]
+        L.moe_dispatch_by_rank.argtypes = [_P, _P, _P, _I32, _P, _P, _P, _P, _I64, _I32, _P]
+        L.moe_combine_by_rank.argtypes = [_P, _P, _P, _P, _I64, _I32, _P]
         for name in ("counts", "psum", "rows_per_rank", "tokens_per_rank", "token_in_rank", "slots",
-                     "row_src", "row_weights"):
+                     "row_src", "row_weights", "token_rows"):
             f = getattr(L, f"moe_handle_{name}")
             f.argtypes = [_P]
             f.restype = _P
@@ -157,6 +160,9 @@ class Handle:
     def slots(self):
         return self._view("slots", (self.params.num_tokens, self.params.topk), "<i4").clone()
 
+    def token_rows(self):
+        return self._view("token_rows", (self.params.num_tokens, self.params.num_logical_ranks), "<i4").clone()
+
     def row_capacity(self) -> int:
         return int(lib().moe_handle_row_capacity(self.ptr))
 
@@ -208,6 +214,26 @@ def moe_combine(handle: Handle, y: torch.Tensor, out: torch.Tensor, topk_weights
     rc = lib().moe_combine(handle.ptr, _ptr(y), _ptr(topk_weights), _ptr(bias), _ptr(out), cap, num_sms,
                            _stream(stream))
     _check(rc, "moe_combine")
+
+
+def moe_dispatch_by_rank(handle: Handle, x: torch.Tensor, out_dtype: int, recv_x: torch.Tensor,
+                         recv_scales: Optional[torch.Tensor] = None, topk_idx: Optional[torch.Tensor] = None,
+                         recv_topk_idx: Optional[torch.Tensor] = None,
+                         recv_topk_weights: Optional[torch.Tensor] = None, cap: Optional[int] = None,
+                         num_sms: int = 0, stream=None) -> None:
+    """Non-expanded dispatch: one row per (token, rank) with the token's per-rank top-k views."""
+    cap = recv_x.shape[1] if cap is None else cap
+    rc = lib().moe_dispatch_by_rank(handle.ptr, _ptr(x), _ptr(topk_idx), out_dtype, _ptr(recv_x), _ptr(recv_scales),
+                                    _ptr(recv_topk_idx), _ptr(recv_topk_weights), cap, num_sms, _stream(stream))
+    _check(rc, "moe_dispatch_by_rank")
+
+
+def moe_combine_by_rank(handle: Handle, y: torch.Tensor, out: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                        cap: Optional[int] = None, num_sms: int = 0, stream=None) -> None:
+    """Non-expanded combine: sum of the token's per-rank partial sums (+ bias)."""
+    cap = y.shape[1] if cap is None else cap
+    rc = lib().moe_combine_by_rank(handle.ptr, _ptr(y), _ptr(bias), _ptr(out), cap, num_sms, _stream(stream))
+    _check(rc, "moe_combine_by_rank")
 
 
 def moe_combine_backward(handle: Handle, grad_out: torch.Tensor, grad_y: torch.Tensor,

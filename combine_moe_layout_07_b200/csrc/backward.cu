@@ -27,7 +27,7 @@ __global__ void __launch_bounds__(32 * kGradWarps) k_grad_weights(GradWeightsLau
   for (int64_t p = gw; p < L.T * L.k; p += nw) {
     const int32_t r = __ldg(L.pair_rank + p), s = __ldg(L.slot + p);
     float acc = 0.0f;
-    if (r >= 0 && s < L.cap) {
+    if (r >= 0 && s >= 0 && s < L.cap) {
       const uint16_t* yr = y + ((int64_t)r * L.cap + s) * H;
       const uint16_t* gr = go + (int64_t)((uint32_t)p / (uint32_t)L.k) * H;
       constexpr int U = 4;
@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(32 * kGradWarps) k_grad_weights(GradWeightsLau
           }
         }
       }
-    } else if (r >= 0) {
+    } else if (r >= 0 && s >= 0) {
       atomicOr(L.status, kStatusCapacity);
     }
 #pragma unroll

@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
       for (int q = 0; q < nt && !stop; ++q) {
         const int64_t t = tb + q;
         int64_t src = -1;
-        if (lane >= q * L.k && lane < (q + 1) * L.k && cur.rank >= 0) {
+        if (lane >= q * L.k && lane < (q + 1) * L.k && cur.rank >= 0 && cur.slot >= 0) {  // by-rank rows: -1 on repeats
           if (cur.slot < L.cap) src = ((int64_t)cur.rank * L.cap + cur.slot) * H;
           else overflow = true;
         }

@@ -34,8 +34,9 @@ constexpr int kDispMaxStages = 8;
 constexpr uint32_t kSmemBudget = 200 * 1024;
 
 struct DispMeta {
-  int64_t row[kMaxTopk];  // destination rows (rank * cap + slot) of the valid pairs, in j order
-  float w[kMaxTopk];      // their topk weights
+  int64_t row[kMaxTopk];   // destination rows (rank * cap + slot) of the valid pairs, in j order
+  float w[kMaxTopk];       // their topk weights
+  int32_t rank[kMaxTopk];  // their logical ranks
   int32_t n;
   int32_t pad_[3];
 };
@@ -108,13 +109,16 @@ __global__ void __launch_bounds__(kDispThreads, 1) k_dispatch(DispatchLaunch L, 
     const int tpb = 32 / L.k, lanes_used = tpb * L.k;
     const int64_t p_end = t_end * L.k;
     const float* wsrc = L.scale_w ? L.scale_w : L.pair_w;
-    PairBatch cur = load_pair_batch(L.pair_rank, L.slot, wsrc, t_begin * L.k, p_end, lane, lanes_used);
+    const bool views = L.recv_topk_idx || L.recv_topk_w;  // by-rank per-row top-k views
+    const int64_t* ids = views ? L.topk_idx : nullptr;
+    PairBatch cur = load_pair_batch(L.pair_rank, L.slot, wsrc, t_begin * L.k, p_end, lane, lanes_used, ids);
     int64_t i = 0;
     int s = 0;
     uint32_t par = 0;  // (i / S) & 1
     bool stop = false;
     for (int64_t tb = t_begin; tb < t_end && !stop; tb += tpb) {
-      const PairBatch nxt = load_pair_batch(L.pair_rank, L.slot, wsrc, (tb + tpb) * L.k, p_end, lane, lanes_used);
+      const PairBatch nxt =
+          load_pair_batch(L.pair_rank, L.slot, wsrc, (tb + tpb) * L.k, p_end, lane, lanes_used, ids);
       const int nt = (int)min((int64_t)tpb, t_end - tb);
       for (int q = 0; q < nt; ++q) {
         const int64_t t = tb + q;
@@ -127,7 +131,7 @@ __global__ void __launch_bounds__(kDispThreads, 1) k_dispatch(DispatchLaunch L, 
           }
         }
         int64_t row = -1;
-        if (lane >= q * L.k && lane < (q + 1) * L.k && cur.rank >= 0) {
+        if (lane >= q * L.k && lane < (q + 1) * L.k && cur.rank >= 0 && cur.slot >= 0) {  // by-rank rows: -1 on repeats
           if (cur.slot < L.cap) row = (int64_t)cur.rank * L.cap + cur.slot;
           else overflow = true;
         }
@@ -136,9 +140,24 @@ __global__ void __launch_bounds__(kDispThreads, 1) k_dispatch(DispatchLaunch L, 
           const int pos = __popc(m & lanemask_lt());
           meta[s].row[pos] = row;
           meta[s].w[pos] = cur.w;
+          meta[s].rank[pos] = cur.rank;
         }
         if (lane == 0) meta[s].n = __popc(m);
         __syncwarp();
+        if (views) {  // by-rank: each destination row gets the token's k ids / weights for its rank
+          const bool mine = lane >= q * L.k && lane < (q + 1) * L.k;
+          const int jj = lane - q * L.k;
+          const int n = __popc(m);
+          for (int d = 0; d < n; ++d) {
+            const int64_t row_d = meta[s].row[d];
+            const int r_d = meta[s].rank[d];
+            if (mine) {
+              const bool on = cur.rank == r_d;  // this choice of the token lives on rank r_d
+              if (L.recv_topk_idx) L.recv_topk_idx[row_d * L.k + jj] = on ? cur.e - r_d * L.E_loc : -1;
+              if (L.recv_topk_w) L.recv_topk_w[row_d * L.k + jj] = on ? cur.w : 0.0f;
+            }
+          }
+        }
         if (lane == 0) {
           mbar_arrive_expect_tx(full0 + 8 * s, in_bytes);
           if (dbg_ok(t < L.T && lay.in + (uint32_t)(s + 1) * in_bytes <= lay.total, L.status, 201, t))

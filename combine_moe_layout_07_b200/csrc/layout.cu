@@ -173,6 +173,60 @@ __device__ __forceinline__ bool row_map_padding(const LayoutLaunch& L, const int
   return overflow;
 }
 
+// Non-expanded (by-rank) layout for the block-sized group of tokens [t0, t0 + blockDim):
+// token_row[t, r] = base_r[r] + (member tokens of rank r before t in the group), -1 when t has
+// no expert on r; base_r[r] (shared) advances by the group's count.  tslot[t, j] = the token's
+// row on rank(e_j) for the first j of the token on that rank, else -1.  R <= 64 (rank bitmasks);
+// wcnt is shared scratch of [blockDim / 32][kMaxByRankRanks].  Called by the whole block.
+__device__ __forceinline__ void token_rows_group(const LayoutLaunch& L, int64_t t0, int64_t t_end, int32_t* base_r,
+                                                 int32_t* wcnt) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, W = blockDim.x >> 5;
+  const int64_t t = t0 + tid;
+  const bool valid = t < t_end;
+  const uint32_t lt = lanemask_lt();
+  uint64_t mask = 0;
+  if (valid)
+    for (int j = 0; j < L.k; ++j) {
+      const int32_t e = expert_of(__ldg(L.idx + t * L.k + j), L.E);
+      if (e >= 0) mask |= 1ull << ((uint32_t)e / (uint32_t)L.E_loc);
+    }
+  for (int r = 0; r < L.R; ++r) {
+    const uint32_t b = __ballot_sync(0xffffffffu, (mask >> r) & 1);
+    if (lane == 0) wcnt[warp * kMaxByRankRanks + r] = __popc(b);
+  }
+  __syncthreads();
+  for (int r = tid; r < L.R; r += blockDim.x) {
+    int32_t run = base_r[r];
+    for (int w = 0; w < W; ++w) {
+      const int32_t v = wcnt[w * kMaxByRankRanks + r];
+      wcnt[w * kMaxByRankRanks + r] = run;
+      run += v;
+    }
+    base_r[r] = run;
+  }
+  __syncthreads();
+  for (int r = 0; r < L.R; ++r) {
+    const uint32_t b = __ballot_sync(0xffffffffu, (mask >> r) & 1);
+    if (valid) L.d.token_row[t * L.R + r] = ((mask >> r) & 1) ? wcnt[warp * kMaxByRankRanks + r] + __popc(b & lt) : -1;
+  }
+  if (valid) {
+    uint64_t seen = 0;
+    for (int j = 0; j < L.k; ++j) {
+      const int32_t e = expert_of(__ldg(L.idx + t * L.k + j), L.E);
+      int32_t v = -1;
+      if (e >= 0) {
+        const int r = (int)((uint32_t)e / (uint32_t)L.E_loc);
+        if (!((seen >> r) & 1)) {
+          seen |= 1ull << r;
+          v = L.d.token_row[t * L.R + r];  // written above by this thread
+        }
+      }
+      L.d.tslot[t * L.k + j] = v;
+    }
+  }
+  __syncthreads();
+}
+
 // Block-wide exclusive scan of one value per thread (warp shuffles + one smem pass).
 __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_tot, int32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
@@ -274,8 +328,10 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_count(LayoutLaunch L)
     }
     __syncthreads();
     for (int e = tid; e < L.E; e += blockDim.x) L.d.chunk_cnt[(int64_t)c * L.E + e] = hist[e];
-    for (int r = tid; r < L.R; r += blockDim.x)
+    for (int r = tid; r < L.R; r += blockDim.x) {
       if (tok[r]) atomicAdd(L.d.tokens_per_rank + r, tok[r]);  // integer sum: order-free
+      if (L.by_rank) L.d.chunk_tok[(int64_t)c * L.R + r] = tok[r];
+    }
     __syncthreads();
   }
   if (!ok) atomicOr(L.d.status, kStatusBadExpert);
@@ -294,7 +350,14 @@ __global__ void __launch_bounds__(kScanThreads) k_layout_scan(LayoutLaunch L, in
   extern __shared__ int32_t sm[];
   const int E = L.E;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int e = blockIdx.x * 32 + lane;
+  // CTAs [0, ceil(E/32)) scan expert columns of chunk_cnt; the rest (by-rank) rank columns of
+  // chunk_tok, the same way
+  const int n_expert_ctas = (E + 31) / 32;
+  const bool experts = (int)blockIdx.x < n_expert_ctas;
+  const int width = experts ? E : L.R;
+  int32_t* counts = experts ? L.d.chunk_cnt : L.d.chunk_tok;
+  const int col0 = (experts ? (int)blockIdx.x : (int)blockIdx.x - n_expert_ctas) * 32;
+  const int e = col0 + lane;
   const int C = L.num_chunks;
   const int cpw = (C + 31) / 32;  // chunks per warp
   const int c0 = min(C, warp * cpw), c1 = min(C, c0 + cpw);
@@ -302,8 +365,8 @@ __global__ void __launch_bounds__(kScanThreads) k_layout_scan(LayoutLaunch L, in
   grid_dependency_wait();  // chunk counts of the count kernel
 
   int32_t sum = 0;
-  if (e < E)
-    for (int c = c0; c < c1; ++c) sum += L.d.chunk_cnt[(int64_t)c * E + e];
+  if (e < width)
+    for (int c = c0; c < c1; ++c) sum += counts[(int64_t)c * width + e];
   gsum[warp][lane] = sum;
   __syncthreads();
   {  // warp x scans the 32 group sums of expert blockIdx.x*32 + x
@@ -316,14 +379,14 @@ __global__ void __launch_bounds__(kScanThreads) k_layout_scan(LayoutLaunch L, in
     }
     __syncwarp();
     gsum[lane][warp] = incl - v;
-    const int ex = blockIdx.x * 32 + warp;
-    if (lane == 31 && ex < E) L.d.cnt[ex] = incl;
+    const int ex = col0 + warp;
+    if (experts && lane == 31 && ex < E) L.d.cnt[ex] = incl;
   }
   __syncthreads();
-  if (e < E) {
+  if (e < width) {
     int32_t off = gsum[warp][lane];
     for (int c = c0; c < c1; ++c) {
-      int32_t* q = L.d.chunk_cnt + (int64_t)c * E + e;
+      int32_t* q = counts + (int64_t)c * width + e;
       const int32_t v = *q;
       *q = off;
       off += v;
@@ -349,6 +412,8 @@ __global__ void __launch_bounds__(kScanThreads) k_layout_scan(LayoutLaunch L, in
 // among equal ids of lower lanes in the round.
 __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L) {
   extern __shared__ int32_t whist[];  // [kLayoutWarps][E]
+  __shared__ int32_t base_r[kMaxByRankRanks];
+  __shared__ int32_t wcnt[kLayoutWarps * kMaxByRankRanks];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = L.E;
   int32_t* h = whist + warp * E;
@@ -378,6 +443,11 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L
     __syncthreads();
     overflow |= warp_assign(L, wp0, wp1, h);
     __syncthreads();
+    if (L.by_rank) {  // chunk = kChunkTokens = blockDim tokens: one group, based at the chunk offsets
+      for (int r = tid; r < L.R; r += blockDim.x) base_r[r] = L.d.chunk_tok[(int64_t)c * L.R + r];
+      __syncthreads();
+      token_rows_group(L, t0, t1, base_r, wcnt);
+    }
   }
   overflow |= row_map_padding(L, L.d.pad_excl, L.d.psum, (int64_t)blockIdx.x * kLayoutWarps + warp,
                               (int64_t)gridDim.x * kLayoutWarps);
@@ -443,6 +513,13 @@ __global__ void __launch_bounds__(kSmallThreads) k_layout_small(LayoutLaunch L, 
   bool overflow = warp_assign(L, wp0, wp1, h);
   overflow |= row_map_padding(L, pad_s, psum_s, warp, W);
   if (overflow) atomicOr(L.d.status, kStatusCapacity);
+  if (L.by_rank) {
+    __shared__ int32_t base_r[kMaxByRankRanks];
+    __shared__ int32_t wcnt[W * kMaxByRankRanks];
+    for (int r = tid; r < L.R; r += blockDim.x) base_r[r] = 0;
+    __syncthreads();
+    for (int64_t t0 = 0; t0 < L.T; t0 += blockDim.x) token_rows_group(L, t0, L.T, base_r, wcnt);
+  }
 }
 
 bool layout_fits_one_cta(int64_t T, int k, int E) {
@@ -493,7 +570,8 @@ cudaError_t launch_layout_scan(const LayoutLaunch& L, int64_t cap_check, cudaStr
   cudaError_t err = ensure_smem_attrs();
   if (err != cudaSuccess) return err;
   const size_t smem = sizeof(int32_t) * 3 * (size_t)L.E;
-  err = launch_pdl(k_layout_scan, dim3((L.E + 31) / 32), dim3(kScanThreads), smem, s, L, cap_check);
+  const int grid = (L.E + 31) / 32 + (L.by_rank ? (L.R + 31) / 32 : 0);
+  err = launch_pdl(k_layout_scan, dim3(grid), dim3(kScanThreads), smem, s, L, cap_check);
   note_launch();
   return err;
 }

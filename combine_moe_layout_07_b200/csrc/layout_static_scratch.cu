@@ -60,7 +60,7 @@ extern "C" int moe_layout_static_scratch(const moe_params_t* p, const int64_t* t
   // argument checks: the same limits as moe_layout, plus caller-owned row maps
   if (!p) return MOE_ERR_INVALID_ARG;
   if (p->num_tokens < 0 || p->num_logical_ranks < 1 || p->num_experts < 1 || p->topk < 1 ||
-      p->expert_alignment < 1 || p->hidden < 8 || p->hidden % 8 != 0 || p->num_sms < 0 || p->reserved != 0 ||
+      p->expert_alignment < 1 || p->hidden < 8 || p->hidden % 8 != 0 || p->num_sms < 0 || p->flags != 0 ||
       (p->do_cpu_sync != 0 && p->do_cpu_sync != 1) || p->recv_capacity_rows < 1 ||
       p->num_experts % p->num_logical_ranks != 0)
     return MOE_ERR_INVALID_ARG;

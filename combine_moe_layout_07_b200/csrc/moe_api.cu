@@ -93,7 +93,8 @@ static int check_params(const moe_params_t* p) {
   if (!p) return MOE_ERR_INVALID_ARG;
   if (p->num_tokens < 0 || p->num_logical_ranks < 1 || p->num_experts < 1 || p->topk < 1 ||
       p->expert_alignment < 1 || p->hidden < 8 || p->hidden % 8 != 0 || p->num_sms < 0 ||
-      p->reserved != 0 || (p->do_cpu_sync != 0 && p->do_cpu_sync != 1) || p->recv_capacity_rows < 0)
+      (p->flags & ~MOE_LAYOUT_BY_RANK) != 0 || (p->do_cpu_sync != 0 && p->do_cpu_sync != 1) ||
+      p->recv_capacity_rows < 0)
     return MOE_ERR_INVALID_ARG;
   if (p->num_experts % p->num_logical_ranks != 0) return MOE_ERR_INVALID_ARG;
   if (p->topk > kMaxTopk || p->num_experts > kMaxExperts) return MOE_ERR_UNSUPPORTED;
@@ -164,6 +165,10 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
                 o_pad = take(4 * (E + 1)), o_tir = take(T * R), o_slot = take(4 * T * k),
                 o_prank = take(4 * T * k), o_pw = take(4 * T * k), o_ccnt = take(4 * C * E),
                 o_rsrc = take(4 * R * h->row_cap), o_rw = take(4 * R * h->row_cap);
+  // the non-expanded (by-rank) layout, on request and for R <= kMaxByRankRanks
+  const bool by_rank = (p->flags & MOE_LAYOUT_BY_RANK) && R <= kMaxByRankRanks;
+  const int64_t o_ctok = by_rank ? take(4 * C * R) : 0, o_trow = by_rank ? take(4 * T * R) : 0,
+                o_tslot = by_rank ? take(4 * T * k) : 0;
   if (pool_alloc(&h->block, (size_t)off, h->device, s) != cudaSuccess) {
     cudaGetLastError();
     delete h;
@@ -185,6 +190,11 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   d.chunk_cnt = reinterpret_cast<int32_t*>(b + o_ccnt);
   d.row_src = reinterpret_cast<int32_t*>(b + o_rsrc);
   d.row_w = reinterpret_cast<float*>(b + o_rw);
+  if (by_rank) {
+    d.chunk_tok = reinterpret_cast<int32_t*>(b + o_ctok);
+    d.token_row = reinterpret_cast<int32_t*>(b + o_trow);
+    d.tslot = reinterpret_cast<int32_t*>(b + o_tslot);
+  }
 
   LayoutLaunch L{};
   L.idx = topk_idx;
@@ -199,6 +209,7 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   L.grid_chunks = h->num_chunks;
   if (p->num_sms > 0 && L.grid_chunks > p->num_sms) L.grid_chunks = p->num_sms;
   L.row_cap = h->row_cap;
+  L.by_rank = by_rank ? 1 : 0;
   L.d = d;
 
   // count -> scan -> assign back to back; with do_cpu_sync one host wait at the end
@@ -216,15 +227,18 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   }
 
   if (p->do_cpu_sync) {
-    // [status flags, rows_per_rank[R]] to the host
-    int32_t* stage = static_cast<int32_t*>(g_stage.get(sizeof(int32_t) * (size_t)(R + 1)));
+    // [status flags, ticket, tokens_per_rank[R]] (one adjacent block) and rows_per_rank[R]
+    // layout: [flags][rows_per_rank R][status 4, ticket, pad 3][tokens_per_rank R]
+    int32_t* stage = static_cast<int32_t*>(g_stage.get(sizeof(int32_t) * (size_t)(9 + 2 * R)));
     if (!stage) {
       release(h);
       return MOE_ERR_CUDA;
     }
-    err = cudaMemcpyAsync(stage, d.status, 4, cudaMemcpyDeviceToHost, s);
+    int32_t* tokens_stage = stage + 1 + R + 8;
+    err = cudaMemcpyAsync(tokens_stage - 8, d.status, (size_t)(32 + 4 * R), cudaMemcpyDeviceToHost, s);
     if (err == cudaSuccess) err = cudaMemcpyAsync(stage + 1, d.rows_per_rank, 4 * R, cudaMemcpyDeviceToHost, s);
     if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+    if (err == cudaSuccess) stage[0] = tokens_stage[-8];  // status flags
     if (err != cudaSuccess) {
       release(h);
       return MOE_ERR_CUDA;
@@ -238,6 +252,7 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
       return MOE_ERR_CAPACITY;
     }
     h->host_rows.assign(stage + 1, stage + 1 + R);
+    h->host_tokens.assign(tokens_stage, tokens_stage + R);
     h->counts_on_host = true;
     if (host_rows_per_rank) std::memcpy(host_rows_per_rank, stage + 1, sizeof(int32_t) * (size_t)R);
   }
@@ -258,7 +273,9 @@ int moe_dispatch(const moe_handle_t* h, const void* x, int out_dtype, void* recv
   if (fp8 && (p.hidden % 128 != 0 || !recv_scales || !aligned4(recv_scales))) return MOE_ERR_INVALID_ARG;
   if (p.num_tokens > 0 && (!x || !recv_x)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(recv_x) || !aligned4(recv_weights)) return MOE_ERR_INVALID_ARG;
-  if (!do_expand) return MOE_ERR_UNSUPPORTED;
+  if (!do_expand)  // one row per (token, rank); recv_weights then holds [R, cap, k] weights
+    return moe_dispatch_by_rank(h, x, nullptr, out_dtype, recv_x, recv_scales, nullptr, recv_weights, cap, num_sms,
+                                stream);
   if (h->counts_on_host) {
     for (int32_t v : h->host_rows)
       if (v > cap) return MOE_ERR_CAPACITY;
@@ -312,6 +329,81 @@ int moe_combine(const moe_handle_t* h, const void* y, const float* topk_weights,
   L.grid = grid_for(num_sms, h->device);
   L.pair_rank = h->d.pair_rank;
   L.slot = h->d.slot;
+  L.status = h->d.status;
+  return launch_combine(L, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_dispatch_by_rank(const moe_handle_t* h, const void* x, const int64_t* topk_idx, int out_dtype, void* recv_x,
+                         float* recv_scales, int32_t* recv_topk_idx, float* recv_topk_weights, int64_t cap,
+                         int num_sms, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (out_dtype != MOE_DTYPE_BF16 && out_dtype != MOE_DTYPE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+  if (cap < 0 || cap >= (int64_t)1 << 31 || num_sms < 0) return MOE_ERR_INVALID_ARG;
+  const bool fp8 = out_dtype == MOE_DTYPE_FP8_E4M3;
+  const moe_params_t& p = h->p;
+  if (!h->d.tslot) return MOE_ERR_UNSUPPORTED;  // more logical ranks than the by-rank layout keeps
+  if (fp8 && (p.hidden % 128 != 0 || !recv_scales || !aligned4(recv_scales))) return MOE_ERR_INVALID_ARG;
+  if (p.num_tokens > 0 && (!x || !recv_x)) return MOE_ERR_INVALID_ARG;
+  if (recv_topk_idx && !topk_idx) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(recv_x) || !aligned4(recv_topk_idx) || !aligned4(recv_topk_weights) ||
+      (reinterpret_cast<uintptr_t>(topk_idx) & 7u))
+    return MOE_ERR_INVALID_ARG;
+  if (h->counts_on_host) {
+    for (int32_t v : h->host_tokens)
+      if (v > cap) return MOE_ERR_CAPACITY;
+  }
+  if (p.num_tokens == 0) return MOE_OK;
+  DispatchLaunch L{};
+  L.x = x;
+  L.recv_x = recv_x;
+  L.recv_scales = recv_scales;
+  L.T = p.num_tokens;
+  L.cap = cap;
+  L.H = p.hidden;
+  L.R = p.num_logical_ranks;
+  L.k = p.topk;
+  L.E = p.num_experts;
+  L.E_loc = p.num_experts / p.num_logical_ranks;
+  L.zero_padding = 0;  // no alignment padding without expansion
+  L.grid = grid_for(num_sms, h->device);
+  L.pair_rank = h->d.pair_rank;
+  L.slot = h->d.tslot;
+  L.pair_w = h->d.pair_w;
+  L.topk_idx = topk_idx;
+  L.recv_topk_idx = recv_topk_idx;
+  L.recv_topk_w = recv_topk_weights;
+  L.psum = h->d.psum;
+  L.pad_excl = h->d.pad_excl;
+  L.status = h->d.status;
+  return launch_dispatch(L, fp8, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_combine_by_rank(const moe_handle_t* h, const void* y, const void* bias, void* out, int64_t cap, int num_sms,
+                        void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (cap < 0 || cap >= (int64_t)1 << 31 || num_sms < 0) return MOE_ERR_INVALID_ARG;
+  const moe_params_t& p = h->p;
+  if (!h->d.tslot) return MOE_ERR_UNSUPPORTED;
+  if (p.num_tokens > 0 && (!y || !out)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(out) || !aligned16(bias)) return MOE_ERR_INVALID_ARG;
+  if (h->counts_on_host) {
+    for (int32_t v : h->host_tokens)
+      if (v > cap) return MOE_ERR_CAPACITY;
+  }
+  if (p.num_tokens == 0) return MOE_OK;
+  CombineLaunch L{};
+  L.y = y;
+  L.w = nullptr;  // the per-rank rows are partial sums of already-weighted expert outputs
+  L.bias = bias;
+  L.out = out;
+  L.T = p.num_tokens;
+  L.cap = cap;
+  L.H = p.hidden;
+  L.k = p.topk;
+  L.R = p.num_logical_ranks;
+  L.grid = grid_for(num_sms, h->device);
+  L.pair_rank = h->d.pair_rank;
+  L.slot = h->d.tslot;
   L.status = h->d.status;
   return launch_combine(L, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -398,6 +490,7 @@ const uint8_t* moe_handle_token_in_rank(const moe_handle_t* h) { return h ? h->d
 const int32_t* moe_handle_slots(const moe_handle_t* h) { return h ? h->d.slot : nullptr; }
 const int32_t* moe_handle_row_src(const moe_handle_t* h) { return h ? h->d.row_src : nullptr; }
 const float* moe_handle_row_weights(const moe_handle_t* h) { return h ? h->d.row_w : nullptr; }
+const int32_t* moe_handle_token_rows(const moe_handle_t* h) { return h ? h->d.token_row : nullptr; }
 int64_t moe_handle_row_capacity(const moe_handle_t* h) { return h ? h->row_cap : -1; }
 
 int moe_handle_free(moe_handle_t* h) {

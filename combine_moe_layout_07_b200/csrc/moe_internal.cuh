@@ -33,6 +33,7 @@ constexpr int kSmallPairs = 8192;       // ... used when T * k <= kSmallPairs
 constexpr int kSmallMaxExperts = 1024;  // ... and E <= kSmallMaxExperts
 constexpr int kMaxExperts = 4096;
 constexpr int kMaxTopk = 32;
+constexpr int kMaxByRankRanks = 64;  // the non-expanded (by-rank) layout keeps rank bitmasks
 
 // Data-movement kernels: one 1024-thread CTA per SM, so a num_sms cap is an SM cap.
 constexpr int kMoveThreads = 1024;
@@ -50,6 +51,10 @@ struct DeviceArrays {
   int32_t* pair_rank = nullptr;       // [T * k]  destination logical rank, -1 if masked
   float* pair_w = nullptr;            // [T * k]
   int32_t* chunk_cnt = nullptr;       // [C * E]  counts, then exclusive offsets
+  int32_t* chunk_tok = nullptr;       // [C * R]  by-rank: member tokens per chunk, then offsets
+  int32_t* token_row = nullptr;       // [T * R]  by-rank: row of token t on rank r, -1 if none
+  int32_t* tslot = nullptr;           // [T * k]  by-rank: token row on the pair's rank for the
+                                      //          first pair of the token on that rank, else -1
   int32_t* row_src = nullptr;         // [R * row_cap]
   float* row_w = nullptr;             // [R * row_cap]
 };
@@ -64,7 +69,8 @@ struct moe_handle {
   int64_t row_cap = 0;
   int num_chunks = 0;
   bool counts_on_host = false;
-  std::vector<int32_t> host_rows;  // rows_per_rank, when do_cpu_sync
+  std::vector<int32_t> host_rows;    // rows_per_rank, when do_cpu_sync
+  std::vector<int32_t> host_tokens;  // tokens_per_rank, when do_cpu_sync
   moe::DeviceArrays d;
 };
 
@@ -78,6 +84,7 @@ struct LayoutLaunch {
   int num_chunks;
   int grid_chunks;  // CTAs for the per-chunk kernels (<= num_chunks)
   int64_t row_cap;  // 0 -> row maps not written (filled by a later assign launch)
+  int by_rank;      // also build the non-expanded layout (R <= kMaxByRankRanks)
   DeviceArrays d;
 };
 
@@ -101,6 +108,9 @@ struct DispatchLaunch {
   const int32_t* slot;
   const float* pair_w;
   const float* scale_w;  // BF16 rows only, nullable: each destination row is bf16(w[t,j] * x[t])
+  const int64_t* topk_idx;   // by-rank views, nullable: the routing (for local expert ids)
+  int32_t* recv_topk_idx;    // by-rank, nullable: [R, cap, k] local expert id or -1
+  float* recv_topk_w;        // by-rank, nullable: [R, cap, k] topk weight or 0
   const int32_t* psum;
   const int32_t* pad_excl;
   int32_t* status;
@@ -354,17 +364,19 @@ namespace moe {
 struct PairBatch {
   int32_t rank, slot;
   float w;
+  int32_t e;  // expert id (only when `ids` is given), else -1
 };
 
 __device__ __forceinline__ PairBatch load_pair_batch(const int32_t* pair_rank, const int32_t* slot,
                                                      const float* w, int64_t p0, int64_t p_end, int lane,
-                                                     int lanes_used) {
-  PairBatch b{-1, -1, 0.0f};
+                                                     int lanes_used, const int64_t* ids = nullptr) {
+  PairBatch b{-1, -1, 0.0f, -1};
   const int64_t p = p0 + lane;
   if (lane < lanes_used && p < p_end) {
     b.rank = __ldg(pair_rank + p);
     b.slot = __ldg(slot + p);
     if (w) b.w = __ldg(w + p);
+    if (ids && b.rank >= 0) b.e = (int32_t)__ldg(ids + p);
   }
   return b;
 }

@@ -63,6 +63,10 @@ enum moe_status_code {
 
 enum moe_dtype { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_E4M3 = 1 };
 
+/* moe_params_t.flags: also build the non-expanded (one row per token and rank) layout that
+ * moe_dispatch_by_rank / moe_combine_by_rank / moe_dispatch(do_expand = 0) need (R <= 64). */
+#define MOE_LAYOUT_BY_RANK 1
+
 /* Problem description for moe_layout.  All fields are read once; the handle keeps a copy. */
 typedef struct moe_params {
   int64_t num_tokens;         /* T >= 0 */
@@ -73,7 +77,7 @@ typedef struct moe_params {
   int32_t expert_alignment;   /* A >= 1; T*k + E*A < 2^31 */
   int32_t num_sms;            /* SMs the layout kernels may occupy; 0 = all */
   int32_t do_cpu_sync;        /* 1: moe_layout waits for the counts and copies them to host */
-  int32_t reserved;           /* must be 0 */
+  int32_t flags;              /* 0 or MOE_LAYOUT_BY_RANK */
   int64_t recv_capacity_rows; /* cap per rank for the handle's row maps; 0 only with
                                  do_cpu_sync=1 (the rows are then sized from the counts) */
 } moe_params_t;
@@ -114,7 +118,8 @@ int moe_layout(const moe_params_t* params, const int64_t* topk_idx, const float*
  *                 recv_scales[r, row, b] = a / 448 (fp32 [R, cap, H/128]).
  *   recv_weights  fp32 [R, cap], nullable: the pair's topk weight (0 on padding rows).
  *   cap           rows per logical rank in recv_x / recv_scales / recv_weights.
- *   do_expand     must be 1 (one row per (token, expert)); 0 returns MOE_ERR_UNSUPPORTED.
+ *   do_expand     1: one row per (token, expert), the layout above.  0: one row per (token,
+ *                 rank), see moe_dispatch_by_rank (recv_weights is then [R, cap, k]).
  *   do_zero_padding  1: padding rows are written as zero bytes (codes, scales and bf16).
  *   num_sms       SMs the kernel may occupy (0 = all).
  * Rows beyond rows_per_rank[r] are never written.
@@ -122,6 +127,33 @@ int moe_layout(const moe_params_t* params, const int64_t* topk_idx, const float*
 int moe_dispatch(const moe_handle_t* handle, const void* x, int out_dtype, void* recv_x,
                  float* recv_scales, float* recv_weights, int64_t cap, int do_expand,
                  int do_zero_padding, int num_sms, void* stream);
+
+/*
+ * Non-expanded dispatch ("Why MoE gets stuck on communication" 1: without do_expand a destination
+ * rank receives each token once; "Chapter 2: repository map" 2.1: token -> rank membership).
+ * Rank r receives one row per token that has at least one expert on r, in ascending token order
+ * (row = moe_handle_token_rows(handle)[t, r]); cap is the capacity in TOKENS per rank
+ * (tokens_per_rank[r] rows are used).  No alignment padding exists in this layout.
+ *   recv_x / recv_scales  as for moe_dispatch (BF16 copy or FP8 codes + 1x128 scales).
+ *   recv_topk_idx      int32 [R, cap, k], nullable (then topk_idx may be NULL): the local expert
+ *                      index (e - r*E_loc) of the token's j-th choice when it lives on r, else -1.
+ *   recv_topk_weights  fp32 [R, cap, k], nullable: the matching topk weight, else 0.
+ *   topk_idx           int64 [T, k]: the routing given to moe_layout (needed for recv_topk_idx).
+ * Needs a handle laid out with MOE_LAYOUT_BY_RANK and R <= 64 (MOE_ERR_UNSUPPORTED otherwise).
+ * moe_dispatch with do_expand = 0 calls this with
+ * recv_topk_idx = NULL and recv_topk_weights = its recv_weights, read as [R, cap, k].
+ */
+int moe_dispatch_by_rank(const moe_handle_t* handle, const void* x, const int64_t* topk_idx, int out_dtype,
+                         void* recv_x, float* recv_scales, int32_t* recv_topk_idx, float* recv_topk_weights,
+                         int64_t cap, int num_sms, void* stream);
+
+/*
+ * Non-expanded combine: y is bf16 [R, cap, H] with, for every (token, rank), the rank's
+ * already-weighted partial sum over its experts; out[t] = bf16(fp32 sum over the token's ranks in
+ * the order in which they first appear in topk_idx[t, :], then + bias[t]).  Needs R <= 64.
+ */
+int moe_combine_by_rank(const moe_handle_t* handle, const void* y, const void* bias, void* out, int64_t cap,
+                        int num_sms, void* stream);
 
 /*
  * Combine ("From DeepEP to Mega MoE" 2.3 and 2.5: element-wise top-k reduction; "Why MoE gets
@@ -168,6 +200,8 @@ const uint8_t* moe_handle_token_in_rank(const moe_handle_t* handle);   /* [T, R]
 const int32_t* moe_handle_slots(const moe_handle_t* handle);           /* [T, k] */
 const int32_t* moe_handle_row_src(const moe_handle_t* handle);         /* [R, row_cap] */
 const float* moe_handle_row_weights(const moe_handle_t* handle);       /* [R, row_cap] */
+const int32_t* moe_handle_token_rows(const moe_handle_t* handle);      /* [T, R]; NULL without
+                                                                          MOE_LAYOUT_BY_RANK */
 int64_t moe_handle_row_capacity(const moe_handle_t* handle);           /* row_cap */
 
 /* Releases the handle.  Its device memory is freed stream-ordered on the layout stream, so
@@ -185,7 +219,8 @@ const char* moe_status_string(int status);
  * allocator that has reserved the GPU, a runtime that hands out fixed arenas) and serving loops
  * that forbid allocation calls on their hot path, where a driver allocation may block.
  *
- * Computes exactly what moe_layout computes, into caller-owned device buffers:
+ * Computes exactly what moe_layout computes (params->flags must be 0: the by-rank layout is not
+ * built here), into caller-owned device buffers:
  *   counts[E], psum[E], rows_per_rank[R], tokens_per_rank[R], token_in_rank[T, R] (uint8),
  *   slots[T, k], row_src[R, cap] and row_weights[R, cap] with cap = recv_capacity_rows (>= 1).
  * Its temporaries (status word, padding prefix, per-chunk counts, per-pair rank and weight)

@@ -35,10 +35,10 @@ def inputs(wl: W.Workload, mask: float = 0.0):
 
 
 def gpu_layout(wl: W.Workload, idx: torch.Tensor, w: torch.Tensor | None, cap: int = 0,
-               cpu_sync: bool | None = None, num_sms: int = 0):
+               cpu_sync: bool | None = None, num_sms: int = 0, by_rank: bool = False):
     cpu_sync = wl.cpu_sync if cpu_sync is None else cpu_sync
     p = moe.params(wl.tokens, wl.ranks, wl.experts, wl.topk, wl.hidden, wl.alignment,
-                   recv_capacity_rows=cap, num_sms=num_sms, do_cpu_sync=cpu_sync)
+                   recv_capacity_rows=cap, num_sms=num_sms, do_cpu_sync=cpu_sync, by_rank=by_rank)
     return moe.moe_layout(p, idx.cuda(), None if w is None else w.cuda())
 
 

@@ -48,7 +48,7 @@ def test_capacity_hint_formula():
     ("hidden", 100, moe.MOE_ERR_INVALID_ARG),           # not a multiple of 8
     ("expert_alignment", 0, moe.MOE_ERR_INVALID_ARG),
     ("num_tokens", -1, moe.MOE_ERR_INVALID_ARG),
-    ("reserved", 1, moe.MOE_ERR_INVALID_ARG),
+    ("flags", 2, moe.MOE_ERR_INVALID_ARG),               # only MOE_LAYOUT_BY_RANK is defined
     ("do_cpu_sync", 2, moe.MOE_ERR_INVALID_ARG),
     ("num_tokens", 1 << 40, moe.MOE_ERR_UNSUPPORTED),   # row indices would overflow int32
 ])

@@ -255,9 +255,8 @@ def test_bad_dispatch_arguments():
     idx, w, x = inputs(wl)
     h = gpu_layout(wl, idx, w, cap=256)
     recv = torch.zeros(wl.ranks, 256, wl.hidden, dtype=torch.bfloat16, device="cuda")
-    with pytest.raises(moe.MoeError) as e:
-        moe.moe_dispatch(h, x.cuda(), moe.MOE_DTYPE_BF16, recv, do_expand=False)
-    assert e.value.status == moe.MOE_ERR_UNSUPPORTED
+    rc = moe.lib().moe_dispatch(h.ptr, x.cuda().data_ptr(), 0, recv.data_ptr(), None, None, 256, 2, 1, 0, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG          # do_expand is 0 or 1
     with pytest.raises(moe.MoeError) as e:        # FP8 needs H % 128 == 0 and scales
         moe.moe_dispatch(h, x.cuda(), moe.MOE_DTYPE_FP8_E4M3, recv.view(torch.uint8), None)
     assert e.value.status == moe.MOE_ERR_INVALID_ARG
