@@ -15,6 +15,9 @@ LIB = os.path.join(_HERE, "libmoe_oracle.so")
 
 
 def build(force: bool = False) -> str:
+    override = os.environ.get("MOE_ORACLE_LIB")  # tests: a separately built (e.g. mutated) oracle
+    if override:
+        return override
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
@@ -23,6 +26,14 @@ def build(force: bool = False) -> str:
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     return LIB
+
+
+def build_from(src: str, out: str) -> str:
+    """Compile another copy of the oracle source with the same flags (used by the tests that
+    plant mistakes in the oracle to show that its pins catch them)."""
+    subprocess.run(["gcc", "-std=c11", "-O1", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-w",
+                    "-o", out, src, "-lm"], check=True)
+    return out
 
 
 if __name__ == "__main__":

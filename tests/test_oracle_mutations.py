@@ -1,0 +1,49 @@
+"""The oracle's pins have teeth: each test plants one plausible mistake in a copy of the oracle
+(on the CPU), rebuilds it, and requires the pin suite (tests/test_oracle.py) to fail against it."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "moe_oracle.c")
+
+# (name, exact text in moe_oracle.c, replacement)
+MUTATIONS = [
+    ("psum exclusive instead of inclusive", "            run += align_up(cnt[e], A);\n            psum[e] = (int32_t)run;",
+     "            psum[e] = (int32_t)run;\n            run += align_up(cnt[e], A);"),
+    ("alignment dropped", "            run += align_up(cnt[e], A);", "            run += cnt[e];"),
+    ("slot order reversed inside a segment", "            int32_t row = seg_start + fill[e]++;",
+     "            int32_t row = seg_start + (cnt[e] - 1 - fill[e]++);"),
+    ("row_src holds the pair index", "                row_src[(int64_t)r * cap + row] = (int32_t)t;",
+     "                row_src[(int64_t)r * cap + row] = (int32_t)(t * k + j);"),
+    ("masked entries counted", "            if (e == -1) continue;\n            if (e < -1 || e >= E)",
+     "            if (e == -1) { cnt[0] += 1; continue; }\n            if (e < -1 || e >= E)"),
+    ("E4M3 rounds half away from zero", "    double m = nearbyint(ldexp(a, 3 - e));", "    double m = round(ldexp(a, 3 - e));"),
+    ("E4M3 truncates", "    double m = nearbyint(ldexp(a, 3 - e));", "    double m = floor(ldexp(a, 3 - e));"),
+    ("E4M3 saturation threshold off", "    if (a >= 448.0) return (uint8_t)(sign | 0x7E);",
+     "    if (a >= 480.0) return (uint8_t)(sign | 0x7F);"),
+    ("FP8 scale inverted", "    float inv = 448.0f / a;", "    float inv = a / 448.0f;"),
+    ("combine ignores the weights", "                acc = w ? fmaf(w[t * k + j], v, acc) : acc + v;",
+     "                acc = acc + v;"),
+    ("combine drops the bias", "            if (bias) acc = acc + oracle_bf16_to_float(bias[t * H + h]);\n            out[t * H + h] = oracle_float_to_bf16(acc);\n        }\n    return status;\n}\n\n/* The same sum",
+     "            out[t * H + h] = oracle_float_to_bf16(acc);\n        }\n    return status;\n}\n\n/* The same sum"),
+    ("bf16 rounding truncates", "    if (lo > 0x8000u || (lo == 0x8000u && (hi & 1u))) hi += 1;", "    (void)lo;"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_planted_mistake(name, old, new, tmp_path):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site not found exactly once: {name}"
+    mutated = tmp_path / "moe_oracle_mutated.c"
+    mutated.write_text(src.replace(old, new))
+    sys.path.insert(0, ROOT)
+    from oracle import build as oracle_build
+    lib = oracle_build.build_from(str(mutated), str(tmp_path / "libmutated.so"))
+    env = dict(os.environ, MOE_ORACLE_LIB=lib)
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_oracle.py"), "-x", "-q",
+                        "-p", "no:cacheprovider", "-k", "not brute_force"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"no pin caught the planted mistake '{name}'"
