@@ -74,6 +74,162 @@ __device__ __forceinline__ int find_padding_expert(const int32_t* pad_excl, int 
   return lo;
 }
 
+// The producer warp of both dispatch kernels: pair metadata for tpb tokens per warp-wide load,
+// prefetched one batch ahead; per token, waits for its stage to be free, writes the destination
+// rows into the stage's DispMeta (and, by rank, the per-row top-k views) and issues one bulk load
+// of the bf16 row.  Stage s of token i is i % S, phase (i / S) & 1.
+__device__ __forceinline__ void dispatch_producer(const DispatchLaunch& L, int S, uint32_t full0, uint32_t empty0,
+                                                  DispMeta* meta, uint32_t in_smem, int64_t t_begin,
+                                                  int64_t t_end, int lane, bool& overflow) {
+  const int64_t H = L.H;
+  const uint32_t in_bytes = (uint32_t)(2 * H);
+  const uint16_t* x = static_cast<const uint16_t*>(L.x);
+  const int tpb = 32 / L.k, lanes_used = tpb * L.k;
+  const int64_t p_end = t_end * L.k;
+  const float* wsrc = L.scale_w ? L.scale_w : L.pair_w;
+  const bool views = L.recv_topk_idx || L.recv_topk_w;  // by-rank per-row top-k views
+  const int64_t* ids = views ? L.topk_idx : nullptr;
+  PairBatch cur = load_pair_batch(L.pair_rank, L.slot, wsrc, t_begin * L.k, p_end, lane, lanes_used, ids);
+  int64_t i = 0;
+  int s = 0;
+  uint32_t par = 0;  // (i / S) & 1
+  bool stop = false;
+  for (int64_t tb = t_begin; tb < t_end && !stop; tb += tpb) {
+    const PairBatch nxt =
+        load_pair_batch(L.pair_rank, L.slot, wsrc, (tb + tpb) * L.k, p_end, lane, lanes_used, ids);
+    const int nt = (int)min((int64_t)tpb, t_end - tb);
+    for (int q = 0; q < nt; ++q) {
+      const int64_t t = tb + q;
+      if (i >= S) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(empty0 + 8 * s, par ^ 1u, L.status);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          stop = true;
+          break;
+        }
+      }
+      int64_t row = -1;
+      if (lane >= q * L.k && lane < (q + 1) * L.k && cur.rank >= 0 && cur.slot >= 0) {  // by-rank rows: -1 on repeats
+        if (cur.slot < L.cap) row = (int64_t)cur.rank * L.cap + cur.slot;
+        else overflow = true;
+      }
+      const uint32_t m = __ballot_sync(0xffffffffu, row >= 0);
+      if (row >= 0) {
+        const int pos = __popc(m & lanemask_lt());
+        meta[s].row[pos] = row;
+        meta[s].w[pos] = cur.w;
+        meta[s].rank[pos] = cur.rank;
+      }
+      if (lane == 0) meta[s].n = __popc(m);
+      __syncwarp();
+      if (views) {  // by-rank: each destination row gets the token's k ids / weights for its rank
+        const bool mine = lane >= q * L.k && lane < (q + 1) * L.k;
+        const int jj = lane - q * L.k;
+        const int n = __popc(m);
+        for (int d = 0; d < n; ++d) {
+          const int64_t row_d = meta[s].row[d];
+          const int r_d = meta[s].rank[d];
+          if (mine) {
+            const bool on = cur.rank == r_d;  // this choice of the token lives on rank r_d
+            if (L.recv_topk_idx) L.recv_topk_idx[row_d * L.k + jj] = on ? cur.e - r_d * L.E_loc : -1;
+            if (L.recv_topk_w) L.recv_topk_w[row_d * L.k + jj] = on ? cur.w : 0.0f;
+          }
+        }
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(full0 + 8 * s, in_bytes);
+        if (dbg_ok(t < L.T && s < S, L.status, 201, t))
+          bulk_load(in_smem + (uint32_t)s * in_bytes, x + t * H, in_bytes, full0 + 8 * s);
+      }
+      __syncwarp();
+      ++i;
+      if (++s == S) {
+        s = 0;
+        par ^= 1u;
+      }
+    }
+    cur = nxt;
+  }
+  // no load of this CTA may still be in flight when it exits: wait for the last S tokens
+  if (lane == 0) {
+    int ss = s;
+    uint32_t pp = par;
+    for (int64_t j = 0; j < min(i, (int64_t)S); ++j) {
+      if (--ss < 0) {
+        ss = S - 1;
+        pp ^= 1u;
+      }
+      mbar_wait(full0 + 8 * ss, pp, L.status);
+    }
+  }
+}
+
+// Padding rows (zero_padding: zero codes and scales; recv_w: weight 0), a warp per row: warp gw of
+// nw warps in the grid takes padding rows gw, gw + nw, ...
+template <bool kFp8>
+__device__ __forceinline__ void zero_padding_rows(const DispatchLaunch& L, int64_t gw, int64_t nw, int lane,
+                                                  bool& overflow) {
+  if (!L.zero_padding && !L.recv_w) return;
+  const int64_t H = L.H, nblk = H / 128;
+  const int32_t total_pad = __ldg(L.pad_excl + L.E);
+  const int64_t row_bytes = kFp8 ? H : 2 * H;
+  for (int64_t i = gw; i < total_pad; i += nw) {
+    const int e = find_padding_expert(L.pad_excl, L.E, (int32_t)i);
+    const int32_t pad_e = __ldg(L.pad_excl + e + 1) - __ldg(L.pad_excl + e);
+    const int32_t row = __ldg(L.psum + e) - pad_e + ((int32_t)i - __ldg(L.pad_excl + e));
+    if (row >= L.cap) {
+      overflow = true;
+      continue;
+    }
+    const int64_t grow = (int64_t)(e / L.E_loc) * L.cap + row;
+    if (!dbg_ok(row >= 0 && grow < L.R * L.cap, L.status, 204, grow)) continue;
+    if (L.zero_padding) {
+      uint8_t* dst = static_cast<uint8_t*>(L.recv_x) + grow * row_bytes;
+      for (int64_t o = lane * 16; o < row_bytes; o += 32 * 16) st_stream_v4(dst + o, make_uint4(0, 0, 0, 0));
+      if (kFp8)
+        for (int64_t b = lane; b < nblk; b += 32) L.recv_scales[grow * nblk + b] = 0.0f;
+    }
+    if (L.recv_w && lane == 0) L.recv_w[grow] = 0.0f;
+  }
+}
+
+// FP8 E4M3 codes of the 16 bf16 values of unit u (bytes 32u .. 32u + 31) of a staged row.  Eight
+// consecutive lanes hold one 1x128 block: amax over the block by three xor-shuffles, a =
+// max(amax, 1e-4), inv = 448 / a and scale = a / 448 as IEEE divisions, codes =
+// satfinite(v * inv) rounded to nearest even.  Call with the whole warp; a lane with act = false
+// reads nothing and adds zeros to its block's amax.
+__device__ __forceinline__ uint4 quantize_unit(uint32_t in_s, int64_t u, bool act, float& scale) {
+  uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+  if (act) {
+    a = lds_v4(in_s + (uint32_t)u * 32);
+    b = lds_v4(in_s + (uint32_t)u * 32 + 16);
+  }
+  const uint32_t wd[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  float v[16];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    v[2 * q] = bf16lo(wd[q]);
+    v[2 * q + 1] = bf16hi(wd[q]);
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+  const float am = fmaxf(amax, 1e-4f);
+  const float inv = __fdiv_rn(448.0f, am);
+  scale = __fdiv_rn(am, 448.0f);
+  uint32_t qw[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t lo = pack_e4m3x2(__fmul_rn(v[4 * q], inv), __fmul_rn(v[4 * q + 1], inv));
+    const uint32_t hi = pack_e4m3x2(__fmul_rn(v[4 * q + 2], inv), __fmul_rn(v[4 * q + 3], inv));
+    qw[q] = lo | (hi << 16);
+  }
+  return make_uint4(qw[0], qw[1], qw[2], qw[3]);
+}
+
 template <bool kFp8>
 __global__ void __launch_bounds__(kDispThreads, 1) k_dispatch(DispatchLaunch L, int S) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -85,7 +241,6 @@ __global__ void __launch_bounds__(kDispThreads, 1) k_dispatch(DispatchLaunch L, 
   const int64_t H = L.H;
   const uint32_t in_bytes = (uint32_t)(2 * H);
   const int64_t nblk = H / 128;
-  const uint16_t* x = static_cast<const uint16_t*>(L.x);
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -104,86 +259,7 @@ __global__ void __launch_bounds__(kDispThreads, 1) k_dispatch(DispatchLaunch L, 
   bool overflow = false;
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    // pair metadata for tpb tokens per warp-wide load, prefetched one batch ahead
-    const int tpb = 32 / L.k, lanes_used = tpb * L.k;
-    const int64_t p_end = t_end * L.k;
-    const float* wsrc = L.scale_w ? L.scale_w : L.pair_w;
-    const bool views = L.recv_topk_idx || L.recv_topk_w;  // by-rank per-row top-k views
-    const int64_t* ids = views ? L.topk_idx : nullptr;
-    PairBatch cur = load_pair_batch(L.pair_rank, L.slot, wsrc, t_begin * L.k, p_end, lane, lanes_used, ids);
-    int64_t i = 0;
-    int s = 0;
-    uint32_t par = 0;  // (i / S) & 1
-    bool stop = false;
-    for (int64_t tb = t_begin; tb < t_end && !stop; tb += tpb) {
-      const PairBatch nxt =
-          load_pair_batch(L.pair_rank, L.slot, wsrc, (tb + tpb) * L.k, p_end, lane, lanes_used, ids);
-      const int nt = (int)min((int64_t)tpb, t_end - tb);
-      for (int q = 0; q < nt; ++q) {
-        const int64_t t = tb + q;
-        if (i >= S) {
-          bool ok = true;
-          if (lane == 0) ok = mbar_wait(empty0 + 8 * s, par ^ 1u, L.status);
-          if (!__shfl_sync(0xffffffffu, ok, 0)) {
-            stop = true;
-            break;
-          }
-        }
-        int64_t row = -1;
-        if (lane >= q * L.k && lane < (q + 1) * L.k && cur.rank >= 0 && cur.slot >= 0) {  // by-rank rows: -1 on repeats
-          if (cur.slot < L.cap) row = (int64_t)cur.rank * L.cap + cur.slot;
-          else overflow = true;
-        }
-        const uint32_t m = __ballot_sync(0xffffffffu, row >= 0);
-        if (row >= 0) {
-          const int pos = __popc(m & lanemask_lt());
-          meta[s].row[pos] = row;
-          meta[s].w[pos] = cur.w;
-          meta[s].rank[pos] = cur.rank;
-        }
-        if (lane == 0) meta[s].n = __popc(m);
-        __syncwarp();
-        if (views) {  // by-rank: each destination row gets the token's k ids / weights for its rank
-          const bool mine = lane >= q * L.k && lane < (q + 1) * L.k;
-          const int jj = lane - q * L.k;
-          const int n = __popc(m);
-          for (int d = 0; d < n; ++d) {
-            const int64_t row_d = meta[s].row[d];
-            const int r_d = meta[s].rank[d];
-            if (mine) {
-              const bool on = cur.rank == r_d;  // this choice of the token lives on rank r_d
-              if (L.recv_topk_idx) L.recv_topk_idx[row_d * L.k + jj] = on ? cur.e - r_d * L.E_loc : -1;
-              if (L.recv_topk_w) L.recv_topk_w[row_d * L.k + jj] = on ? cur.w : 0.0f;
-            }
-          }
-        }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(full0 + 8 * s, in_bytes);
-          if (dbg_ok(t < L.T && lay.in + (uint32_t)(s + 1) * in_bytes <= lay.total, L.status, 201, t))
-            bulk_load(base + lay.in + (uint32_t)s * in_bytes, x + t * H, in_bytes, full0 + 8 * s);
-        }
-        __syncwarp();
-        ++i;
-        if (++s == S) {
-          s = 0;
-          par ^= 1u;
-        }
-      }
-      cur = nxt;
-    }
-    // no load of this CTA may still be in flight when it exits: wait for the last S tokens
-    if (lane == 0) {
-      int ss = s;
-      uint32_t pp = par;
-      for (int64_t j = 0; j < min(i, (int64_t)S); ++j) {
-        if (--ss < 0) {
-          ss = S - 1;
-          pp ^= 1u;
-        }
-        mbar_wait(full0 + 8 * ss, pp, L.status);
-      }
-    }
+    dispatch_producer(L, S, full0, empty0, meta, base + lay.in, t_begin, t_end, lane, overflow);
   } else {
     // ---------------------------------------------------------------- consumers
     const int ctid = tid - 32;
@@ -201,36 +277,9 @@ __global__ void __launch_bounds__(kDispThreads, 1) k_dispatch(DispatchLaunch L, 
         const int64_t nunits = H / 16;  // 16 elements per lane and pass; 8 lanes per 1x128 block
         for (int64_t u = gtid; u - gtid < nunits; u += kDispGroupThreads) {
           const bool act = u < nunits;
-          uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+          float scale;
+          const uint4 qv = quantize_unit(in_s, u, act, scale);
           if (act) {
-            a = lds_v4(in_s + (uint32_t)u * 32);
-            b = lds_v4(in_s + (uint32_t)u * 32 + 16);
-          }
-          const uint32_t wd[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-          float v[16];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            v[2 * q] = bf16lo(wd[q]);
-            v[2 * q + 1] = bf16hi(wd[q]);
-          }
-          float amax = 0.0f;
-#pragma unroll
-          for (int q = 0; q < 16; ++q) amax = fmaxf(amax, fabsf(v[q]));
-          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-          const float am = fmaxf(amax, 1e-4f);
-          const float inv = __fdiv_rn(448.0f, am);
-          const float scale = __fdiv_rn(am, 448.0f);
-          uint32_t qw[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t lo = pack_e4m3x2(__fmul_rn(v[4 * q], inv), __fmul_rn(v[4 * q + 1], inv));
-            const uint32_t hi = pack_e4m3x2(__fmul_rn(v[4 * q + 2], inv), __fmul_rn(v[4 * q + 3], inv));
-            qw[q] = lo | (hi << 16);
-          }
-          if (act) {
-            const uint4 qv = make_uint4(qw[0], qw[1], qw[2], qw[3]);
             for (int j = 0; j < n; ++j) {
               const int64_t row = M.row[j];
               if (!dbg_ok(row >= 0 && row < L.R * L.cap && u * 16 + 16 <= H, L.status, 202, row)) continue;
@@ -267,30 +316,189 @@ __global__ void __launch_bounds__(kDispThreads, 1) k_dispatch(DispatchLaunch L, 
       }
     }
 
-    // ---------------------------------------------------------------- padding rows, a warp per row
-    if (L.zero_padding || L.recv_w) {
-      const int32_t total_pad = __ldg(L.pad_excl + L.E);
-      const int64_t row_bytes = kFp8 ? H : 2 * H;
-      const int64_t gw = (int64_t)blockIdx.x * kDispConsumerWarps + (ctid >> 5);
-      for (int64_t i = gw; i < total_pad; i += (int64_t)gridDim.x * kDispConsumerWarps) {
-        const int e = find_padding_expert(L.pad_excl, L.E, (int32_t)i);
-        const int32_t pad_e = __ldg(L.pad_excl + e + 1) - __ldg(L.pad_excl + e);
-        const int32_t row = __ldg(L.psum + e) - pad_e + ((int32_t)i - __ldg(L.pad_excl + e));
-        if (row >= L.cap) {
-          overflow = true;
-          continue;
+    zero_padding_rows<kFp8>(L, blockIdx.x * kDispConsumerWarps + (ctid >> 5), gridDim.x * kDispConsumerWarps, lane,
+                            overflow);
+  }
+  if (overflow) atomicOr(L.status, kStatusCapacity);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Bulk-store dispatch: every dispatch except the weight-scaled rows of the combine backward.  The
+// rows leave shared memory through cp.async.bulk stores (the TMA unit writes them; no register
+// traffic), which keeps more bytes in flight per SM than 16-byte register stores.
+//   warp 0      producer (dispatch_producer): metadata + one bulk load per token, input ring of S;
+//   warp 1      storer: tokens in order; lanes 0..n-1 each issue one bulk store of the row to
+//               their destination (BF16: straight from the input stage; FP8: from the output
+//               stage the consumers filled), and write recv_w; every lane commits a bulk group
+//               per token, so after cp.async.bulk.wait_group.read kBulkLag the stage of the token
+//               kBulkLag places back has been read and is handed back;
+//   warps 2..17 FP8: two consumer groups quantise alternate tokens from the input stage into an
+//               output stage (ring of O) and write the 1x128 scales with plain stores (a scale
+//               row of H / 128 floats need not be 16-byte aligned).  Then every warp zeroes
+//               padding rows; BF16 has nothing to compute, so its consumer warps start there.
+// Barriers: full[S] (producer expect_tx, count 1); empty[S] (BF16: the storer; FP8: the group's
+// warps + the storer, which reads the stage's metadata); ofull[O] (the group's warps, after
+// fence.proxy.async so the bulk engine sees their shared-memory writes); oempty[O] (the storer).
+constexpr int kBulkThreads = 64 + kDispConsumers;
+constexpr int kBulkMaxIn = 12;  // input stages, a multiple of the consumer-group count
+constexpr int kBulkOut = 8;     // FP8 output stages, a multiple of the consumer-group count
+constexpr int kBulkLag = 2;     // bulk groups a storer lane leaves reading shared memory
+
+struct BulkSmem {
+  uint32_t full, empty, ofull, oempty, meta, in, out, total;
+};
+
+__host__ __device__ inline BulkSmem bulk_smem(int64_t H, bool fp8, int S) {
+  const int O = fp8 ? kBulkOut : 0;
+  BulkSmem b;
+  uint32_t off = 0;
+  b.full = off;
+  off += 8 * S;
+  b.empty = off;
+  off += 8 * S;
+  b.ofull = off;
+  off += 8 * O;
+  b.oempty = off;
+  off += 8 * O;
+  off = round_to(off, 16);
+  b.meta = off;
+  off += (uint32_t)sizeof(DispMeta) * S;
+  off = round_to(off, 128);
+  b.in = off;
+  off += (uint32_t)(2 * H) * S;
+  b.out = off;
+  off += (uint32_t)H * O;
+  b.total = off;
+  return b;
+}
+
+template <bool kFp8>
+__global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunch L, int S) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const BulkSmem lay = bulk_smem(L.H, kFp8, S);
+  constexpr int O = kFp8 ? kBulkOut : 0;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t base = smem_u32(smem);
+  const uint32_t full0 = base + lay.full, empty0 = base + lay.empty;
+  const uint32_t ofull0 = base + lay.ofull, oempty0 = base + lay.oempty;
+  DispMeta* meta = reinterpret_cast<DispMeta*>(smem + lay.meta);
+  const int64_t H = L.H;
+  const uint32_t in_bytes = (uint32_t)(2 * H);
+  const uint32_t row_bytes = kFp8 ? (uint32_t)H : in_bytes;  // bytes of one destination row
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, kFp8 ? kDispGroupWarps + 1 : 1);
+    }
+    for (int o = 0; o < O; ++o) {
+      mbar_init(ofull0 + 8 * o, kDispGroupWarps);
+      mbar_init(oempty0 + 8 * o, 1);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  grid_dependents_launch();
+  grid_dependency_wait();  // the handle written by the layout kernels
+
+  int64_t t_begin, t_end;
+  cta_token_range(L.T, t_begin, t_end);
+  const int64_t n_items = t_end - t_begin;
+  bool overflow = false;
+
+  if (warp == 0) {
+    dispatch_producer(L, S, full0, empty0, meta, base + lay.in, t_begin, t_end, lane, overflow);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- storer
+    uint8_t* recv = static_cast<uint8_t*>(L.recv_x);
+    int s = 0, o = 0;
+    uint32_t par = 0, opar = 0;
+    for (int64_t i = 0; i < n_items; ++i) {
+      const uint32_t ready = kFp8 ? ofull0 + 8 * o : full0 + 8 * s;
+      if (!mbar_wait_warp(ready, kFp8 ? opar : par, L.status)) break;
+      const int n = meta[s].n;
+      if (!dbg_ok(n >= 0 && n <= L.k, L.status, 206, n)) break;
+      const int64_t row = lane < n ? meta[s].row[lane] : -1;
+      const float w = lane < n ? meta[s].w[lane] : 0.0f;
+      if constexpr (kFp8) {  // the metadata is read: the input stage is the consumers' to release now
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * s);
+      }
+      if (row >= 0 && dbg_ok(row < L.R * L.cap, L.status, 207, row)) {
+        const uint32_t src = kFp8 ? base + lay.out + (uint32_t)o * row_bytes : base + lay.in + (uint32_t)s * in_bytes;
+        bulk_store(recv + row * row_bytes, src, row_bytes);
+        if (L.recv_w) L.recv_w[row] = w;
+      }
+      bulk_commit();
+      bulk_wait_read<kBulkLag>();  // the group of token i - kBulkLag has read its stage
+      __syncwarp();
+      if (lane == 0 && i >= kBulkLag) {
+        if constexpr (kFp8) mbar_arrive(oempty0 + 8 * ((o - kBulkLag + O) % O));
+        else mbar_arrive(empty0 + 8 * ((s - kBulkLag + S) % S));
+      }
+      if (++s == S) {
+        s = 0;
+        par ^= 1u;
+      }
+      if constexpr (kFp8) {
+        if (++o == O) {
+          o = 0;
+          opar ^= 1u;
         }
-        const int64_t grow = (int64_t)(e / L.E_loc) * L.cap + row;
-        if (!dbg_ok(row >= 0 && grow < L.R * L.cap, L.status, 204, grow)) continue;
-        if (L.zero_padding) {
-          uint8_t* dst = static_cast<uint8_t*>(L.recv_x) + grow * row_bytes;
-          for (int64_t o = lane * 16; o < row_bytes; o += 32 * 16) st_stream_v4(dst + o, make_uint4(0, 0, 0, 0));
-          if (kFp8)
-            for (int64_t b = lane; b < nblk; b += 32) L.recv_scales[grow * nblk + b] = 0.0f;
-        }
-        if (L.recv_w && lane == 0) L.recv_w[grow] = 0.0f;
       }
     }
+    bulk_wait_all();  // no store may still read shared memory when the CTA exits
+  } else {
+    const int ctid = tid - 64;
+    if constexpr (kFp8) {
+      // ---------------------------------------------------------------- FP8 consumers
+      const int grp = (warp - 2) / kDispGroupWarps;
+      const int gtid = ctid - grp * kDispGroupThreads;
+      const int64_t nblk = H / 128, nunits = H / 16;
+      int s = grp % S, o = grp % O;
+      uint32_t par = (uint32_t)((grp / S) & 1), opar = (uint32_t)((grp / O) & 1);
+      for (int64_t i = grp; i < n_items; i += kDispGroups) {
+        if (!mbar_wait_warp(full0 + 8 * s, par, L.status)) break;
+        if (i >= O && !mbar_wait_warp(oempty0 + 8 * o, opar ^ 1u, L.status)) break;
+        const DispMeta& M = meta[s];
+        const int n = M.n;
+        if (!dbg_ok(n >= 0 && n <= L.k, L.status, 205, n)) break;
+        const uint32_t in_s = base + lay.in + (uint32_t)s * in_bytes;
+        const uint32_t out_s = base + lay.out + (uint32_t)o * row_bytes;
+        for (int64_t u = gtid; u - gtid < nunits; u += kDispGroupThreads) {
+          const bool act = u < nunits;
+          float scale;
+          const uint4 qv = quantize_unit(in_s, u, act, scale);
+          if (act) {
+            sts_v4(out_s + (uint32_t)u * 16, qv);
+            if ((gtid & 7) == 0)
+              for (int j = 0; j < n; ++j) {
+                const int64_t row = M.row[j];
+                if (!dbg_ok(row >= 0 && row < L.R * L.cap, L.status, 202, row)) continue;
+                L.recv_scales[row * nblk + u / 8] = scale;
+              }
+          }
+        }
+        fence_proxy_async_smem();  // the codes are read next by the bulk engine (async proxy)
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(empty0 + 8 * s);
+          mbar_arrive(ofull0 + 8 * o);
+        }
+        s += kDispGroups;
+        while (s >= S) {
+          s -= S;
+          par ^= 1u;
+        }
+        o += kDispGroups;
+        while (o >= O) {
+          o -= O;
+          opar ^= 1u;
+        }
+      }
+    }
+    zero_padding_rows<kFp8>(L, blockIdx.x * kDispConsumerWarps + (ctid >> 5), gridDim.x * kDispConsumerWarps, lane,
+                            overflow);
   }
   if (overflow) atomicOr(L.status, kStatusCapacity);
 }
@@ -305,7 +513,30 @@ int dispatch_stages(int64_t H) {
   return 0;
 }
 
+// Input stages of the bulk-store kernel (a multiple of the group count, more than kBulkLag);
+// 0 when not even the smallest ring fits.
+int dispatch_bulk_stages(int64_t H, bool fp8) {
+  static_assert(kBulkMaxIn % kDispGroups == 0 && kBulkOut % kDispGroups == 0, "stages per group");
+  static_assert(kBulkOut > kBulkLag, "the storer hands output stages back kBulkLag tokens late");
+  for (int s = kBulkMaxIn; s > kBulkLag; s -= kDispGroups)
+    if (bulk_smem(H, fp8, s).total <= kSmemBudget) return s;
+  return 0;
+}
+
 cudaError_t launch_dispatch(const DispatchLaunch& L, bool fp8, cudaStream_t st) {
+  if (!L.scale_w) {
+    const int S = dispatch_bulk_stages(L.H, fp8);
+    if (S > kBulkLag) {
+      const uint32_t smem = bulk_smem(L.H, fp8, S).total;
+      static unsigned long long done[2] = {0, 0};
+      auto kern = fp8 ? k_dispatch_bulk<true> : k_dispatch_bulk<false>;
+      cudaError_t err = set_smem_limit_once(kern, (int)kSmemBudget, &done[fp8 ? 1 : 0]);
+      if (err != cudaSuccess) return err;
+      err = launch_pdl(kern, dim3(L.grid), dim3(kBulkThreads), smem, st, L, S);
+      note_launch();
+      return err;
+    }
+  }
   const int S = dispatch_stages(L.H);
   if (S < kDispGroups) return cudaErrorInvalidValue;
   const uint32_t smem = disp_smem(L.H, S).total;
