@@ -37,27 +37,22 @@ __device__ __forceinline__ int32_t expert_of(int64_t e, int E) {
 __device__ __forceinline__ bool token_membership(const LayoutLaunch& L, int64_t t, bool valid, int32_t* hist,
                                                  int32_t* tok) {
   bool bad = false;
-  int32_t ev[kMaxTopk];
   const int64_t* ids = L.idx + t * L.k;
-#pragma unroll
-  for (int j = 0; j < kMaxTopk; ++j) {
-    ev[j] = (valid && j < L.k) ? expert_of(__ldg(ids + j), L.E) : -1;
-    if (ev[j] == -2) {
-      bad = true;
-      ev[j] = -1;
-    }
-  }
   uint8_t* member = L.d.token_in_rank + t * L.R;
   if (L.R <= 64) {
     uint64_t mask = 0;
-#pragma unroll
-    for (int j = 0; j < kMaxTopk; ++j)
-      if (ev[j] >= 0) {
-        if (hist) atomicAdd_block(&hist[ev[j]], 1);
-        mask |= 1ull << ((uint32_t)ev[j] / (uint32_t)L.E_loc);
+    if (valid) {
+#pragma unroll 4
+      for (int j = 0; j < L.k; ++j) {
+        const int32_t e = expert_of(__ldg(ids + j), L.E);
+        bad |= e == -2;
+        if (e >= 0) {
+          if (hist) atomicAdd_block(&hist[e], 1);
+          mask |= 1ull << ((uint32_t)e / (uint32_t)L.E_loc);
+        }
       }
-    if (valid)
       for (int r = 0; r < L.R; ++r) member[r] = (uint8_t)((mask >> r) & 1);
+    }
     const int lane = threadIdx.x & 31;
     for (int r = 0; r < L.R; ++r) {
       const int c = __popc(__ballot_sync(0xffffffffu, (mask >> r) & 1));
@@ -65,20 +60,22 @@ __device__ __forceinline__ bool token_membership(const LayoutLaunch& L, int64_t 
     }
   } else if (valid) {
     for (int r = 0; r < L.R; ++r) member[r] = 0;
-#pragma unroll
-    for (int j = 0; j < kMaxTopk; ++j)
-      if (ev[j] >= 0) {
-        if (hist) atomicAdd_block(&hist[ev[j]], 1);
-        const int r = (int)((uint32_t)ev[j] / (uint32_t)L.E_loc);
-        bool first = true;
-#pragma unroll
-        for (int j2 = 0; j2 < j; ++j2)
-          if (ev[j2] >= 0 && (int)((uint32_t)ev[j2] / (uint32_t)L.E_loc) == r) first = false;
-        if (first) {
-          member[r] = 1;
-          atomicAdd_block(&tok[r], 1);
-        }
+    for (int j = 0; j < L.k; ++j) {
+      const int32_t e = expert_of(__ldg(ids + j), L.E);
+      bad |= e == -2;
+      if (e < 0) continue;
+      if (hist) atomicAdd_block(&hist[e], 1);
+      const int r = (int)((uint32_t)e / (uint32_t)L.E_loc);
+      bool first = true;  // the token's first id on rank r counts it there
+      for (int j2 = 0; j2 < j; ++j2) {
+        const int32_t e2 = expert_of(__ldg(ids + j2), L.E);
+        if (e2 >= 0 && (int)((uint32_t)e2 / (uint32_t)L.E_loc) == r) first = false;
       }
+      if (first) {
+        member[r] = 1;
+        atomicAdd_block(&tok[r], 1);
+      }
+    }
   }
   return !bad;
 }
@@ -97,6 +94,7 @@ __device__ __forceinline__ void warp_histogram(const LayoutLaunch& L, int64_t wp
     }
 #pragma unroll
     for (int r = 0; r < kAssignBatch; ++r) {
+      if (base + r * 32 >= wp1) break;  // warp-uniform: the rest of the batch is empty
       const uint32_t peers = __match_any_sync(0xffffffffu, ev[r]);
       if (ev[r] >= 0 && lane == __ffs(peers) - 1) h[ev[r]] += __popc(peers);
       __syncwarp();
@@ -121,6 +119,7 @@ __device__ __forceinline__ bool warp_assign(const LayoutLaunch& L, int64_t wp0, 
     }
 #pragma unroll
     for (int r = 0; r < kAssignBatch; ++r) {
+      if (base + r * 32 >= wp1) break;  // warp-uniform: the rest of the batch is empty
       const int64_t p = base + r * 32 + lane;
       const int32_t e = ev[r];
       const uint32_t peers = __match_any_sync(0xffffffffu, e);
@@ -320,8 +319,8 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_count(LayoutLaunch L)
   for (int c = blockIdx.x; c < L.num_chunks; c += gridDim.x) {
     for (int i = tid; i < L.E + L.R; i += blockDim.x) sm[i] = 0;
     __syncthreads();
-    const int64_t t0 = (int64_t)c * kChunkTokens;
-    const int64_t t1 = min(L.T, t0 + kChunkTokens);
+    const int64_t t0 = (int64_t)c * L.chunk;
+    const int64_t t1 = min(L.T, t0 + L.chunk);
     for (int64_t tb = t0; tb < t1; tb += blockDim.x) {  // same trip count for every thread
       const int64_t t = tb + tid;
       ok &= token_membership(L, t, t < t1, hist, tok);
@@ -422,8 +421,8 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L
   grid_dependency_wait();  // offsets, counts and psum of the scan kernel
 
   for (int c = blockIdx.x; c < L.num_chunks; c += gridDim.x) {
-    const int64_t t0 = (int64_t)c * kChunkTokens;
-    const int64_t t1 = min(L.T, t0 + kChunkTokens);
+    const int64_t t0 = (int64_t)c * L.chunk;
+    const int64_t t1 = min(L.T, t0 + L.chunk);
     const int64_t p0 = t0 * L.k, np = (t1 - t0) * L.k;
     const int64_t per = (np + kLayoutWarps - 1) / kLayoutWarps;
     const int64_t wp0 = p0 + min(np, warp * per), wp1 = p0 + min(np, (warp + 1) * per);
@@ -443,7 +442,7 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L
     __syncthreads();
     overflow |= warp_assign(L, wp0, wp1, h);
     __syncthreads();
-    if (L.by_rank) {  // chunk = kChunkTokens = blockDim tokens: one group, based at the chunk offsets
+    if (L.by_rank) {  // chunk <= blockDim tokens: one group, based at the chunk offsets
       for (int r = tid; r < L.R; r += blockDim.x) base_r[r] = L.d.chunk_tok[(int64_t)c * L.R + r];
       __syncthreads();
       token_rows_group(L, t0, t1, base_r, wcnt);
@@ -456,9 +455,11 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L
 
 // ------------------------------------------------------------------------------------ small
 // The whole layout in one CTA of 32 warps, for small batches (T * k <= kSmallPairs and
-// E <= kSmallMaxExperts, e.g. decode): membership and id checks, per-warp histograms of
-// token-aligned pair ranges, cross-warp scan, psum, slots and row maps, all through shared
-// memory, in one launch.  The results equal those of count -> scan -> assign.
+// E <= kSmallMaxExperts): membership and id checks, per-warp histograms of token-aligned pair
+// ranges, cross-warp scan, psum, slots and row maps, all through shared memory, in one launch
+// and with no scratch beyond the handle's arrays.  The allocation-free entry point uses it; the
+// handle path runs count -> scan -> assign, which spreads a small batch over more SMs and is
+// faster.  The results are the same.
 __global__ void __launch_bounds__(kSmallThreads) k_layout_small(LayoutLaunch L, int64_t cap_check) {
   extern __shared__ int32_t sm[];
   const int E = L.E, tid = threadIdx.x, warp = tid >> 5;

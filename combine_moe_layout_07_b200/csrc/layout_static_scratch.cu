@@ -113,6 +113,7 @@ extern "C" int moe_layout_static_scratch(const moe_params_t* p, const int64_t* t
   L.R = (int)R;
   L.E_loc = (int)(E / R);
   L.A = p->expert_alignment;
+  L.chunk = kChunkTokens;
   L.num_chunks = (int)C;
   L.grid_chunks = (int)C;
   if (p->num_sms > 0 && L.grid_chunks > p->num_sms) L.grid_chunks = p->num_sms;

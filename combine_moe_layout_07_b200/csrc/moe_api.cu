@@ -145,7 +145,13 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
     return MOE_ERR_CUDA;
   }
   const int64_t T = p->num_tokens, k = p->topk, E = p->num_experts, R = p->num_logical_ranks;
-  h->num_chunks = (int)((T + kChunkTokens - 1) / kChunkTokens);
+  // Chunks of the count / assign kernels: halve from kChunkTokens down to 32 tokens while the
+  // batch gives fewer than two chunks per SM, so small batches still spread over many CTAs
+  // (a warp's run of pairs, chunk * k / 8, sets the assign kernel's serial work).
+  const int64_t want_chunks = 2 * (int64_t)sm_count(h->device);
+  int chunk = kChunkTokens;
+  while (chunk > 32 && (T + chunk - 1) / chunk < want_chunks) chunk /= 2;
+  h->num_chunks = (int)((T + chunk - 1) / chunk);
   const int64_t C = h->num_chunks;
 
   // One allocation for every array (256-byte aligned sub-arrays).  Without a capacity the row
@@ -205,6 +211,7 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   L.R = (int)R;
   L.E_loc = (int)E_loc;
   L.A = p->expert_alignment;
+  L.chunk = chunk;
   L.num_chunks = h->num_chunks;
   L.grid_chunks = h->num_chunks;
   if (p->num_sms > 0 && L.grid_chunks > p->num_sms) L.grid_chunks = p->num_sms;
@@ -213,14 +220,12 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   L.d = d;
 
   // count -> scan -> assign back to back; with do_cpu_sync one host wait at the end
+  // (Small batches too: 32-token chunks over many CTAs beat the one-CTA kernel, whose warps
+  // each walk hundreds of pairs.)
   cudaError_t err = cudaMemsetAsync(d.status, 0, (size_t)(32 + 4 * R), s);
-  if (layout_fits_one_cta(T, (int)k, (int)E)) {
-    if (err == cudaSuccess) err = launch_layout_small(L, p->recv_capacity_rows, s);
-  } else {
-    if (err == cudaSuccess) err = launch_layout_count(L, s);
-    if (err == cudaSuccess) err = launch_layout_scan(L, p->recv_capacity_rows, s);
-    if (err == cudaSuccess) err = launch_layout_assign(L, s);
-  }
+  if (err == cudaSuccess) err = launch_layout_count(L, s);
+  if (err == cudaSuccess) err = launch_layout_scan(L, p->recv_capacity_rows, s);
+  if (err == cudaSuccess) err = launch_layout_assign(L, s);
   if (err != cudaSuccess) {
     release(h);
     return MOE_ERR_CUDA;

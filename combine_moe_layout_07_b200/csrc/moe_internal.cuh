@@ -24,7 +24,7 @@ constexpr bool kDebugChecks = false;
 
 // Layout tiling: a chunk of tokens per CTA (a thread per token in the count kernel); 8 warps per
 // layout CTA.
-constexpr int kChunkTokens = 256;
+constexpr int kChunkTokens = 256;      // largest chunk: one token per thread of the count kernel
 constexpr int kLayoutThreads = 256;
 constexpr int kLayoutWarps = kLayoutThreads / 32;
 constexpr int kScanThreads = 1024;
@@ -81,7 +81,8 @@ struct LayoutLaunch {
   const float* w;
   int64_t T;
   int k, E, R, E_loc, A;
-  int num_chunks;
+  int chunk;        // tokens per chunk of the count / assign kernels (<= kChunkTokens)
+  int num_chunks;   // ceil(T / chunk)
   int grid_chunks;  // CTAs for the per-chunk kernels (<= num_chunks)
   int64_t row_cap;  // 0 -> row maps not written (filled by a later assign launch)
   int by_rank;      // also build the non-expanded layout (R <= kMaxByRankRanks)
