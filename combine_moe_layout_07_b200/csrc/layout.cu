@@ -82,6 +82,46 @@ __device__ __forceinline__ bool token_membership(const LayoutLaunch& L, int64_t 
 
 constexpr int kAssignBatch = 8;  // rounds of 32 pairs a warp loads before it works on them
 
+// One round of 32 pairs of a warp's run (lane = pair, e = expert id or -1): the group of lanes
+// with equal ids adds its size to h[e] through its first lane.
+__device__ __forceinline__ void histogram_round(int32_t e, int32_t* h) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t peers = __match_any_sync(0xffffffffu, e);
+  if (e >= 0 && lane == __ffs(peers) - 1) h[e] += __popc(peers);
+  __syncwarp();
+}
+
+// One round of the assignment: pair p (when in_range) with expert e (or -1) and weight w gets
+// row h[e] + (lanes below it with the same id); h[e] advances by the group's size.  Writes slot,
+// pair rank, pair weight and the row maps.  Returns true on a row >= row_cap.
+__device__ __forceinline__ bool assign_round(const LayoutLaunch& L, int64_t p, bool in_range, int32_t e, float w,
+                                             int32_t* h) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t peers = __match_any_sync(0xffffffffu, e);
+  int32_t row = -1;
+  if (e >= 0) row = h[e] + __popc(peers & lanemask_lt());
+  __syncwarp();
+  if (e >= 0 && lane == __ffs(peers) - 1) h[e] += __popc(peers);
+  __syncwarp();
+  bool overflow = false;
+  if (in_range) {
+    // 32-bit divisions: e < E and p < T * k < 2^31
+    const int rk = e >= 0 ? (int)((uint32_t)e / (uint32_t)L.E_loc) : -1;
+    L.d.slot[p] = row;
+    L.d.pair_rank[p] = rk;
+    L.d.pair_w[p] = w;
+    if (e >= 0) {
+      if (row < L.row_cap) {
+        L.d.row_src[(int64_t)rk * L.row_cap + row] = (int32_t)((uint32_t)p / (uint32_t)L.k);
+        L.d.row_w[(int64_t)rk * L.row_cap + row] = w;
+      } else {
+        overflow = true;
+      }
+    }
+  }
+  return overflow;
+}
+
 // Phase 1 of the slot assignment: histogram h[E] of the warp's pairs [wp0, wp1) (h zeroed).
 __device__ __forceinline__ void warp_histogram(const LayoutLaunch& L, int64_t wp0, int64_t wp1, int32_t* h) {
   const int lane = threadIdx.x & 31;
@@ -95,9 +135,7 @@ __device__ __forceinline__ void warp_histogram(const LayoutLaunch& L, int64_t wp
 #pragma unroll
     for (int r = 0; r < kAssignBatch; ++r) {
       if (base + r * 32 >= wp1) break;  // warp-uniform: the rest of the batch is empty
-      const uint32_t peers = __match_any_sync(0xffffffffu, ev[r]);
-      if (ev[r] >= 0 && lane == __ffs(peers) - 1) h[ev[r]] += __popc(peers);
-      __syncwarp();
+      histogram_round(ev[r], h);
     }
   }
 }
@@ -106,7 +144,6 @@ __device__ __forceinline__ void warp_histogram(const LayoutLaunch& L, int64_t wp
 // Writes slot, pair rank, pair weight and the row maps.  Returns true on a row >= row_cap.
 __device__ __forceinline__ bool warp_assign(const LayoutLaunch& L, int64_t wp0, int64_t wp1, int32_t* h) {
   const int lane = threadIdx.x & 31;
-  const uint32_t lt = lanemask_lt();
   bool overflow = false;
   for (int64_t base = wp0; base < wp1; base += 32 * kAssignBatch) {
     int32_t ev[kAssignBatch];
@@ -121,28 +158,7 @@ __device__ __forceinline__ bool warp_assign(const LayoutLaunch& L, int64_t wp0, 
     for (int r = 0; r < kAssignBatch; ++r) {
       if (base + r * 32 >= wp1) break;  // warp-uniform: the rest of the batch is empty
       const int64_t p = base + r * 32 + lane;
-      const int32_t e = ev[r];
-      const uint32_t peers = __match_any_sync(0xffffffffu, e);
-      int32_t row = -1;
-      if (e >= 0) row = h[e] + __popc(peers & lt);
-      __syncwarp();
-      if (e >= 0 && lane == __ffs(peers) - 1) h[e] += __popc(peers);
-      __syncwarp();
-      if (p < wp1) {
-        // 32-bit divisions: e < E and p < T * k < 2^31
-        const int rk = e >= 0 ? (int)((uint32_t)e / (uint32_t)L.E_loc) : -1;
-        L.d.slot[p] = row;
-        L.d.pair_rank[p] = rk;
-        L.d.pair_w[p] = wv[r];
-        if (e >= 0) {
-          if (row < L.row_cap) {
-            L.d.row_src[(int64_t)rk * L.row_cap + row] = (int32_t)((uint32_t)p / (uint32_t)L.k);
-            L.d.row_w[(int64_t)rk * L.row_cap + row] = wv[r];
-          } else {
-            overflow = true;
-          }
-        }
-      }
+      overflow |= assign_round(L, p, p < wp1, ev[r], wv[r], h);
     }
   }
   return overflow;
@@ -257,10 +273,12 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
 // Given cnt[] (global memory written by other CTAs when kCntGlobal, else this CTA's shared
 // memory), one CTA computes, with al / pad / gincl / pad_s as [E] or [E + 1] shared arrays:
 // align_up(cnt, A), the padding prefix over all experts (to pad_excl and pad_s), psum restarted
-// at every rank (to psum and psum_s), rows_per_rank and the capacity flag.
+// at every rank (to psum and psum_s), rows_per_rank and the capacity flag.  With publish = false
+// only the shared arrays are written (CTAs that compute the same values for their own use).
 template <bool kCntGlobal>
 __device__ __forceinline__ void block_psum(const LayoutLaunch& L, const int32_t* cnt, int64_t cap_check, int32_t* al,
-                                           int32_t* pad, int32_t* gincl, int32_t* pad_s, int32_t* psum_s) {
+                                           int32_t* pad, int32_t* gincl, int32_t* pad_s, int32_t* psum_s,
+                                           bool publish = true) {
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t totals[2];
   const int E = L.E, tid = threadIdx.x;
@@ -280,24 +298,24 @@ __device__ __forceinline__ void block_psum(const LayoutLaunch& L, const int32_t*
   int32_t ra = block_exclusive_scan(sa, warp_tot, &totals[0]);
   int32_t rp = block_exclusive_scan(sp, warp_tot, &totals[1]);
   for (int x = e0; x < e1; ++x) {
-    L.d.pad_excl[x] = rp;
+    if (publish) L.d.pad_excl[x] = rp;
     if (pad_s) pad_s[x] = rp;
     rp += pad[x];
     ra += al[x];
     gincl[x] = ra;
   }
   if (tid == 0) {
-    L.d.pad_excl[E] = totals[1];
+    if (publish) L.d.pad_excl[E] = totals[1];
     if (pad_s) pad_s[E] = totals[1];
   }
   __syncthreads();
   for (int x = tid; x < E; x += blockDim.x) {
     const int first = (x / L.E_loc) * L.E_loc;
     const int32_t v = gincl[x] - (gincl[first] - al[first]);
-    L.d.psum[x] = v;
+    if (publish) L.d.psum[x] = v;
     if (psum_s) psum_s[x] = v;
   }
-  for (int r = tid; r < L.R; r += blockDim.x) {
+  for (int r = tid; publish && r < L.R; r += blockDim.x) {
     const int first = r * L.E_loc, last = first + L.E_loc - 1;
     const int32_t nrows = gincl[last] - (gincl[first] - al[first]);
     L.d.rows_per_rank[r] = nrows;
@@ -453,6 +471,159 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L
   if (overflow) atomicOr(L.d.status, kStatusCapacity);
 }
 
+// ------------------------------------------------------------------------------------ fused
+// Batches of at most one chunk per SM in one cooperative launch (every CTA resident at once), a
+// CTA per chunk of 256 threads:
+//   1. count: each warp loads its contiguous run of the chunk's pairs into registers (at most
+//      kFusedRounds rounds of 32) and histograms it; token membership as k_layout_count; chunk
+//      counts to global memory; then the CTA arrives at a grid barrier (the ticket word, cleared
+//      before the launch) and waits, bounded, until every CTA has arrived;
+//   2. every CTA sums the chunk counts of all chunks itself: its chunk's offsets inside each
+//      expert (chunks before it) and the expert totals; then align / padding prefix / psum as
+//      the scan kernel's last CTA (CTA 0 alone publishes cnt, psum, pad_excl, rows_per_rank);
+//   3. assign: as k_layout_assign for its chunk (pairs from registers), based at those offsets;
+//      padding rows of the row maps over all CTAs' warps; by rank, the token rows based at the
+//      chunk's rank offsets.
+// One launch and one global handoff instead of three kernels; the results are the same.
+__device__ __forceinline__ bool wait_count_reached(const int32_t* p, int32_t target, int32_t* status) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 0;; ++n) {
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    if (v >= target) return true;
+    if ((n & 63) == 63 && globaltimer_ns() - t0 > kWaitLimitNs) break;
+  }
+  atomicOr(status, kStatusTimeout);
+  return false;
+}
+
+__global__ void __launch_bounds__(kLayoutThreads, 1) k_layout_fused(LayoutLaunch L, int64_t cap_check) {
+  extern __shared__ int32_t sm[];
+  const int E = L.E, R = L.R, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = blockIdx.x, C = gridDim.x;
+  int32_t* whist = sm;                        // [kLayoutWarps][E]
+  int32_t* hist = whist + kLayoutWarps * E;   // [E]  expert totals
+  int32_t* off = hist + E;                    // [E]  rows of each expert in the chunks before c
+  int32_t* al = off + E;                      // [E]
+  int32_t* pad = al + E;                      // [E]
+  int32_t* gincl = pad + E;                   // [E]
+  int32_t* psum_s = gincl + E;                // [E]
+  int32_t* pad_s = psum_s + E;                // [E + 1]
+  int32_t* tok = pad_s + E + 1;               // [R]
+  __shared__ int32_t base_r[kMaxByRankRanks];
+  __shared__ int32_t wcnt[kLayoutWarps * kMaxByRankRanks];
+  __shared__ int32_t go;
+  grid_dependents_launch();
+
+  // the warp's contiguous run of the chunk's pairs, held in registers for counting and assigning
+  const int64_t t0 = (int64_t)c * L.chunk, t1 = min(L.T, t0 + L.chunk);
+  const int64_t p0 = t0 * L.k, np = (t1 - t0) * L.k;
+  const int64_t per = (np + kLayoutWarps - 1) / kLayoutWarps;
+  const int64_t wp0 = p0 + min(np, warp * per), wp1 = p0 + min(np, (warp + 1) * per);
+  int32_t ev[kFusedRounds];
+  float wv[kFusedRounds];
+  bool ok = true;
+#pragma unroll
+  for (int r = 0; r < kFusedRounds; ++r) {
+    const int64_t p = wp0 + r * 32 + lane;
+    const int32_t e = p < wp1 ? expert_of(__ldg(L.idx + p), L.E) : -1;
+    ok &= e != -2;
+    ev[r] = max(e, -1);
+    wv[r] = (p < wp1 && L.w) ? __ldg(L.w + p) : 0.0f;
+  }
+  int32_t* h = whist + warp * E;
+  for (int e = lane; e < E; e += 32) h[e] = 0;
+  for (int r = tid; r < R; r += blockDim.x) tok[r] = 0;
+  __syncthreads();
+  // 1. count: per-warp histograms, token membership (ids now in L1), chunk counts
+#pragma unroll
+  for (int r = 0; r < kFusedRounds; ++r)
+    if (wp0 + r * 32 < wp1) histogram_round(ev[r], h);
+  for (int64_t tb = t0; tb < t1; tb += blockDim.x) {  // same trip count for every thread
+    const int64_t t = tb + tid;
+    ok &= token_membership(L, t, t < t1, nullptr, tok);
+  }
+  if (!ok) atomicOr(L.d.status, kStatusBadExpert);
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    int32_t n = 0;
+    for (int w = 0; w < kLayoutWarps; ++w) n += whist[w * E + e];
+    L.d.chunk_cnt[(int64_t)c * E + e] = n;
+  }
+  for (int r = tid; r < R; r += blockDim.x) {
+    if (tok[r]) atomicAdd(L.d.tokens_per_rank + r, tok[r]);  // integer sum: order-free
+    if (L.by_rank) L.d.chunk_tok[(int64_t)c * R + r] = tok[r];
+  }
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    atomicAdd(L.d.ticket, 1);
+    go = wait_count_reached(L.d.ticket, C, L.d.status);
+  }
+  __syncthreads();
+  if (!go) return;
+
+  // 2. offsets and totals from every chunk's counts (kFusedLoads loads in flight), then psum
+  for (int e = tid; e < E; e += blockDim.x) {
+    int32_t before = 0, total = 0;
+    for (int cb = 0; cb < C; cb += kFusedLoads) {
+      int32_t v[kFusedLoads];
+#pragma unroll
+      for (int q = 0; q < kFusedLoads; ++q)
+        v[q] = cb + q < C ? __ldcg(L.d.chunk_cnt + (int64_t)(cb + q) * E + e) : 0;
+#pragma unroll
+      for (int q = 0; q < kFusedLoads; ++q) {
+        before += cb + q < c ? v[q] : 0;
+        total += v[q];
+      }
+    }
+    off[e] = before;
+    hist[e] = total;
+    if (c == 0) L.d.cnt[e] = total;
+  }
+  if (L.by_rank)
+    for (int r = tid; r < R; r += blockDim.x) {
+      int32_t before = 0;
+      for (int cc = 0; cc < c; ++cc) before += __ldcg(L.d.chunk_tok + (int64_t)cc * R + r);
+      base_r[r] = before;
+    }
+  __syncthreads();
+  block_psum<false>(L, hist, cap_check, al, pad, gincl, pad_s, psum_s, c == 0);
+
+  // 3. assign: warp bases (exclusive over warps, from the expert's segment start and the chunk's
+  // offset), then the warp's pairs from registers
+  for (int e = tid; e < E; e += blockDim.x) {
+    int32_t base = psum_s[e] - al[e] + off[e];
+    for (int w = 0; w < kLayoutWarps; ++w) {
+      const int32_t v = whist[w * E + e];
+      whist[w * E + e] = base;
+      base += v;
+    }
+  }
+  __syncthreads();
+  bool overflow = false;
+#pragma unroll
+  for (int r = 0; r < kFusedRounds; ++r) {
+    const int64_t p = wp0 + r * 32 + lane;
+    if (wp0 + r * 32 < wp1) overflow |= assign_round(L, p, p < wp1, ev[r], wv[r], h);
+  }
+  overflow |= row_map_padding(L, pad_s, psum_s, (int64_t)c * kLayoutWarps + warp, (int64_t)C * kLayoutWarps);
+  if (overflow) atomicOr(L.d.status, kStatusCapacity);
+  if (L.by_rank) {
+    __syncthreads();
+    token_rows_group(L, t0, t1, base_r, wcnt);
+  }
+}
+
+size_t fused_layout_smem(int E, int R) { return sizeof(int32_t) * ((size_t)(kLayoutWarps + 7) * E + 1 + R); }
+
+// At most one chunk per SM (so every CTA can be resident), the chunk's pairs in the warps'
+// registers, and bounded redundant summing.
+bool layout_fits_fused(int num_chunks, int chunk, int k, int E, int device) {
+  return num_chunks >= 1 && num_chunks <= sm_count(device) && E <= kFusedMaxExperts &&
+         (int64_t)chunk * k <= (int64_t)kLayoutThreads * kFusedRounds && (int64_t)num_chunks * E <= kFusedMaxChunkCounts;
+}
+
 // ------------------------------------------------------------------------------------ small
 // The whole layout in one CTA of 32 warps, for small batches (T * k <= kSmallPairs and
 // E <= kSmallMaxExperts): membership and id checks, per-warp histograms of token-aligned pair
@@ -547,6 +718,9 @@ static cudaError_t ensure_smem_attrs() {
   if (err == cudaSuccess)
     err = cudaFuncSetAttribute(k_layout_assign, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(sizeof(int32_t) * kLayoutWarps * kMaxExperts));
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(k_layout_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)fused_layout_smem(kFusedMaxExperts, kFusedMaxExperts));  // R <= E
   if (err == cudaSuccess && dev < 64) done |= 1ull << dev;
   return err;
 }
@@ -565,6 +739,26 @@ cudaError_t launch_layout_small(const LayoutLaunch& L, int64_t cap_check, cudaSt
   k_layout_small<<<1, kSmallThreads, small_layout_smem(L.E, L.R), s>>>(L, cap_check);
   note_launch();
   return cudaGetLastError();
+}
+
+// One CTA per chunk, launched cooperatively so that all of them are resident (the grid barrier
+// inside waits for every CTA).
+cudaError_t launch_layout_fused(const LayoutLaunch& L, int64_t cap_check, cudaStream_t s) {
+  cudaError_t err = ensure_smem_attrs();
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(L.num_chunks);
+  cfg.blockDim = dim3(kLayoutThreads);
+  cfg.dynamicSmemBytes = fused_layout_smem(L.E, L.R);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, k_layout_fused, L, cap_check);
+  note_launch();
+  return err;
 }
 
 cudaError_t launch_layout_scan(const LayoutLaunch& L, int64_t cap_check, cudaStream_t s) {

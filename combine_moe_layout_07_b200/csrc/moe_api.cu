@@ -219,13 +219,17 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   L.by_rank = by_rank ? 1 : 0;
   L.d = d;
 
-  // count -> scan -> assign back to back; with do_cpu_sync one host wait at the end
-  // (Small batches too: 32-token chunks over many CTAs beat the one-CTA kernel, whose warps
-  // each walk hundreds of pairs.)
+  // count -> scan -> assign back to back, or all three in one cooperative launch when there is
+  // at most a chunk per SM; with do_cpu_sync one host wait at the end.  (Small batches take
+  // 32-token chunks over many CTAs: faster than one CTA whose warps each walk hundreds of pairs.)
   cudaError_t err = cudaMemsetAsync(d.status, 0, (size_t)(32 + 4 * R), s);
-  if (err == cudaSuccess) err = launch_layout_count(L, s);
-  if (err == cudaSuccess) err = launch_layout_scan(L, p->recv_capacity_rows, s);
-  if (err == cudaSuccess) err = launch_layout_assign(L, s);
+  if (layout_fits_fused(L.num_chunks, L.chunk, L.k, L.E, h->device)) {
+    if (err == cudaSuccess) err = launch_layout_fused(L, p->recv_capacity_rows, s);
+  } else {
+    if (err == cudaSuccess) err = launch_layout_count(L, s);
+    if (err == cudaSuccess) err = launch_layout_scan(L, p->recv_capacity_rows, s);
+    if (err == cudaSuccess) err = launch_layout_assign(L, s);
+  }
   if (err != cudaSuccess) {
     release(h);
     return MOE_ERR_CUDA;
