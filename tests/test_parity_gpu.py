@@ -109,16 +109,28 @@ def test_small_fp8_roundtrip(hidden, zero_padding):
     dict(hidden=136),                                    # ragged vector tail in the warp loop
     dict(experts=512, ranks=8, topk=8, tokens_per_rank=700, alignment=128),
     dict(hidden=7168, tokens_per_rank=300, experts=32, ranks=4, topk=8),   # several column chunks
-    dict(tokens_per_rank=1024, ranks=1, experts=8, topk=8),   # 8192 pairs: one-CTA layout
-    dict(tokens_per_rank=1025, ranks=1, experts=8, topk=8),   # 8200 pairs: three-kernel layout
+    dict(tokens_per_rank=1024, ranks=1, experts=8, topk=8),   # 8192 pairs, 32 chunks (fused layout)
+    dict(tokens_per_rank=1025, ranks=1, experts=8, topk=8),   # a one-token last chunk
     dict(experts=128, ranks=128, topk=4, tokens_per_rank=2),  # more than 64 ranks (membership)
-    dict(experts=128, ranks=128, topk=4, tokens_per_rank=70), # ... on the three-kernel layout
+    dict(experts=128, ranks=128, topk=4, tokens_per_rank=70), # ... with 280 chunks (three-kernel layout)
     dict(hidden=4104, tokens_per_rank=200, experts=16, ranks=2, topk=3),   # ragged last chunk
 ])
 def test_shapes_and_edges(kw):
     wl = W.WORKLOADS["tiny"].with_(**kw)
     idx, w, x = inputs(wl, 0.1)
     _roundtrip_small(wl, idx, w, x, weighted=True, with_bias=True)
+
+
+@pytest.mark.parametrize("extra", [0, 1])
+def test_fused_and_three_kernel_layouts_at_the_boundary(extra):
+    """The handle's layout runs as one cooperative kernel while the batch has at most one 32-token
+    chunk per SM, else as count -> scan -> assign: both sides of that boundary, every byte."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    wl = W.WORKLOADS["tiny"].with_(tokens_per_rank=16 * sms + extra, ranks=2, experts=16, topk=4)
+    assert -(-wl.tokens // 32) == sms + extra
+    idx, w, x = inputs(wl, 0.1)
+    _roundtrip_small(wl, idx, w, x, weighted=True, with_bias=True)
+    _roundtrip_small(wl, idx, w, x, cpu_sync=False)
 
 
 def test_duplicate_experts_in_one_token():
