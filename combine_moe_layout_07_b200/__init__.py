@@ -16,6 +16,7 @@ import torch
 
 from . import build as _build
 
+MOE_NOT_READY = 1
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = -1
 MOE_ERR_BAD_EXPERT = -2
@@ -28,6 +29,7 @@ MOE_ERR_TIMEOUT = -8
 MOE_DTYPE_BF16 = 0
 MOE_DTYPE_FP8_E4M3 = 1
 MOE_LAYOUT_BY_RANK = 1
+MOE_DEFER_EPILOGUE = 2
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -55,9 +57,10 @@ class MoeParams(ctypes.Structure):
 
 def params(num_tokens: int, num_logical_ranks: int, num_experts: int, topk: int, hidden: int,
            expert_alignment: int, recv_capacity_rows: int = 0, num_sms: int = 0,
-           do_cpu_sync: bool = True, by_rank: bool = False) -> MoeParams:
+           do_cpu_sync: bool = True, by_rank: bool = False, defer_epilogue: bool = False) -> MoeParams:
+    flags = (MOE_LAYOUT_BY_RANK if by_rank else 0) | (MOE_DEFER_EPILOGUE if defer_epilogue else 0)
     return MoeParams(num_tokens, num_logical_ranks, num_experts, topk, hidden, expert_alignment,
-                     num_sms, int(do_cpu_sync), MOE_LAYOUT_BY_RANK if by_rank else 0, recv_capacity_rows)
+                     num_sms, int(do_cpu_sync), flags, recv_capacity_rows)
 
 
 _P, _I64, _I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
@@ -87,6 +90,12 @@ def lib() -> ctypes.CDLL:
         L.moe_handle_row_capacity.argtypes = [_P]
         L.moe_handle_row_capacity.restype = _I64
         L.moe_handle_free.argtypes = [_P]
+        L.moe_handle_wait.argtypes = [_P, _P]
+        L.moe_event_record.argtypes = [_P, ctypes.POINTER(_P)]
+        for name in ("wait",):
+            getattr(L, f"moe_event_{name}").argtypes = [_P, _P]
+        for name in ("synchronize", "query", "free"):
+            getattr(L, f"moe_event_{name}").argtypes = [_P]
         L.moe_status_string.argtypes = [_I32]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_kernel_launch_count.argtypes = []
@@ -188,9 +197,11 @@ def moe_recv_capacity_hint(p: MoeParams, max_tokens_per_rank: int) -> int:
 
 def moe_layout(p: MoeParams, topk_idx: torch.Tensor, topk_weights: Optional[torch.Tensor] = None,
                stream=None) -> Handle:
-    """Layout of one dispatch; with ``do_cpu_sync`` the host row counts are on the handle."""
+    """Layout of one dispatch; with ``do_cpu_sync`` the host row counts are on the handle (with
+    ``defer_epilogue`` only after ``moe_handle_wait``)."""
     h = ctypes.c_void_p()
-    rows = np.zeros(p.num_logical_ranks, np.int32) if p.do_cpu_sync else None
+    deferred = bool(p.flags & MOE_DEFER_EPILOGUE)
+    rows = np.zeros(p.num_logical_ranks, np.int32) if p.do_cpu_sync and not deferred else None
     rc = lib().moe_layout(ctypes.byref(p), _ptr(topk_idx), _ptr(topk_weights), _stream(stream),
                           ctypes.byref(h), None if rows is None else rows.ctypes.data_as(_P))
     _check(rc, "moe_layout")
@@ -278,3 +289,45 @@ def moe_layout_static_scratch(p: MoeParams, topk_idx: torch.Tensor, topk_weights
            _ptr(device_status), None if rows is None else rows.ctypes.data_as(_P), _stream(stream))
     _check(rc, "moe_layout_static_scratch")
     return rows
+
+
+def moe_handle_wait(handle: Handle) -> np.ndarray:
+    """The deferred epilogue of a ``defer_epilogue`` layout: blocks until the counts are on the
+    host, raises ``MoeError`` on a bad expert id or a capacity overflow, and returns (and keeps on
+    the handle) the rows each logical rank receives."""
+    rows = np.zeros(handle.params.num_logical_ranks, np.int32)
+    _check(lib().moe_handle_wait(handle.ptr, rows.ctypes.data_as(_P)), "moe_handle_wait")
+    handle.host_rows_per_rank = rows
+    return rows
+
+
+class Event:
+    """A point recorded on a stream (``moe_event_record``); freed when collected."""
+
+    def __init__(self, stream=None):
+        e = ctypes.c_void_p()
+        _check(lib().moe_event_record(_stream(stream), ctypes.byref(e)), "moe_event_record")
+        self.ptr = e.value
+
+    def wait(self, stream=None) -> None:
+        """Work enqueued on ``stream`` after this call waits for the event (returns at once)."""
+        _check(lib().moe_event_wait(self.ptr, _stream(stream)), "moe_event_wait")
+
+    def synchronize(self) -> None:
+        _check(lib().moe_event_synchronize(self.ptr), "moe_event_synchronize")
+
+    def query(self) -> bool:
+        rc = lib().moe_event_query(self.ptr)
+        if rc == MOE_NOT_READY:
+            return False
+        _check(rc, "moe_event_query")
+        return True
+
+    def __del__(self):
+        if getattr(self, "ptr", None) and _lib is not None:
+            _lib.moe_event_free(self.ptr)
+            self.ptr = None
+
+
+def moe_event_record(stream=None) -> Event:
+    return Event(stream)

@@ -89,11 +89,66 @@ struct PinnedStage {
 };
 static thread_local PinnedStage g_stage;
 
+// Pinned blocks for deferred count copies: a handle holds one until it is freed, then it goes
+// back to this list for the next deferred layout (no cudaMallocHost on the steady path).
+static std::mutex g_pin_mu;
+static std::vector<std::pair<size_t, void*>> g_pin_free;
+
+static void* pinned_take(size_t need, size_t* got) {
+  need = (need + 4095) / 4096 * 4096;
+  {
+    std::lock_guard<std::mutex> lock(g_pin_mu);
+    for (size_t i = 0; i < g_pin_free.size(); ++i)
+      if (g_pin_free[i].first >= need) {
+        void* p = g_pin_free[i].second;
+        *got = g_pin_free[i].first;
+        g_pin_free.erase(g_pin_free.begin() + (long)i);
+        return p;
+      }
+  }
+  void* p = nullptr;
+  if (cudaMallocHost(&p, need) != cudaSuccess) return nullptr;
+  *got = need;
+  return p;
+}
+
+static void pinned_give(void* p, size_t n) {
+  if (!p) return;
+  std::lock_guard<std::mutex> lock(g_pin_mu);
+  g_pin_free.emplace_back(n, p);
+}
+
+// Staging of the do_cpu_sync copy: [unused][rows_per_rank R][status 4, ticket, pad 3][tokens R].
+static size_t count_stage_bytes(int64_t R) { return sizeof(int32_t) * (size_t)(9 + 2 * R); }
+
+static cudaError_t enqueue_count_copy(const moe_handle_t* h, int32_t* stage, cudaStream_t s) {
+  const int64_t R = h->p.num_logical_ranks;
+  cudaError_t err = cudaMemcpyAsync(stage + 1 + R, h->d.status, (size_t)(32 + 4 * R), cudaMemcpyDeviceToHost, s);
+  if (err == cudaSuccess) err = cudaMemcpyAsync(stage + 1, h->d.rows_per_rank, 4 * R, cudaMemcpyDeviceToHost, s);
+  return err;
+}
+
+// The do_cpu_sync epilogue once the copy into `stage` is complete: the status flags decide the
+// result; on success the host counts are kept on the handle (and copied to host_rows_per_rank).
+static int count_epilogue(moe_handle_t* h, const int32_t* stage, int32_t* host_rows_per_rank) {
+  const int64_t R = h->p.num_logical_ranks;
+  const int32_t flags = stage[1 + R];
+  if (flags & kStatusBadExpert) return MOE_ERR_BAD_EXPERT;
+  if (flags & kStatusCapacity) return MOE_ERR_CAPACITY;
+  const int32_t* tokens = stage + 1 + R + 8;
+  h->host_rows.assign(stage + 1, stage + 1 + R);
+  h->host_tokens.assign(tokens, tokens + R);
+  h->counts_on_host = true;
+  if (host_rows_per_rank) std::memcpy(host_rows_per_rank, stage + 1, sizeof(int32_t) * (size_t)R);
+  return MOE_OK;
+}
+
 static int check_params(const moe_params_t* p) {
   if (!p) return MOE_ERR_INVALID_ARG;
   if (p->num_tokens < 0 || p->num_logical_ranks < 1 || p->num_experts < 1 || p->topk < 1 ||
       p->expert_alignment < 1 || p->hidden < 8 || p->hidden % 8 != 0 || p->num_sms < 0 ||
-      (p->flags & ~MOE_LAYOUT_BY_RANK) != 0 || (p->do_cpu_sync != 0 && p->do_cpu_sync != 1) ||
+      (p->flags & ~(MOE_LAYOUT_BY_RANK | MOE_DEFER_EPILOGUE)) != 0 ||
+      (p->do_cpu_sync != 0 && p->do_cpu_sync != 1) || ((p->flags & MOE_DEFER_EPILOGUE) && !p->do_cpu_sync) ||
       p->recv_capacity_rows < 0)
     return MOE_ERR_INVALID_ARG;
   if (p->num_experts % p->num_logical_ranks != 0) return MOE_ERR_INVALID_ARG;
@@ -109,6 +164,8 @@ static int check_params(const moe_params_t* p) {
 static void release(moe_handle_t* h) {
   if (!h) return;
   if (h->block) cudaFreeAsync(h->block, h->stream);
+  if (h->epi_event) cudaEventDestroy(h->epi_event);
+  pinned_give(h->epi_stage, h->epi_bytes);
   delete h;
 }
 
@@ -235,37 +292,54 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
     return MOE_ERR_CUDA;
   }
 
-  if (p->do_cpu_sync) {
-    // [status flags, ticket, tokens_per_rank[R]] (one adjacent block) and rows_per_rank[R]
-    // layout: [flags][rows_per_rank R][status 4, ticket, pad 3][tokens_per_rank R]
-    int32_t* stage = static_cast<int32_t*>(g_stage.get(sizeof(int32_t) * (size_t)(9 + 2 * R)));
-    if (!stage) {
+  if (p->do_cpu_sync && (p->flags & MOE_DEFER_EPILOGUE)) {
+    // the copy is enqueued into the handle's own pinned block; moe_handle_wait waits for it
+    h->epi_stage = static_cast<int32_t*>(pinned_take(count_stage_bytes(R), &h->epi_bytes));
+    if (!h->epi_stage) {
       release(h);
-      return MOE_ERR_CUDA;
+      return MOE_ERR_OOM;
     }
-    int32_t* tokens_stage = stage + 1 + R + 8;
-    err = cudaMemcpyAsync(tokens_stage - 8, d.status, (size_t)(32 + 4 * R), cudaMemcpyDeviceToHost, s);
-    if (err == cudaSuccess) err = cudaMemcpyAsync(stage + 1, d.rows_per_rank, 4 * R, cudaMemcpyDeviceToHost, s);
-    if (err == cudaSuccess) err = cudaStreamSynchronize(s);
-    if (err == cudaSuccess) stage[0] = tokens_stage[-8];  // status flags
+    err = cudaEventCreateWithFlags(&h->epi_event, cudaEventDisableTiming);
+    if (err == cudaSuccess) err = enqueue_count_copy(h, h->epi_stage, s);
+    if (err == cudaSuccess) err = cudaEventRecord(h->epi_event, s);
     if (err != cudaSuccess) {
       release(h);
       return MOE_ERR_CUDA;
     }
-    if (stage[0] & kStatusBadExpert) {
+    h->epi_pending = true;
+  } else if (p->do_cpu_sync) {
+    int32_t* stage = static_cast<int32_t*>(g_stage.get(count_stage_bytes(R)));
+    if (!stage) {
       release(h);
-      return MOE_ERR_BAD_EXPERT;
+      return MOE_ERR_CUDA;
     }
-    if (stage[0] & kStatusCapacity) {
+    err = enqueue_count_copy(h, stage, s);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+    if (err != cudaSuccess) {
       release(h);
-      return MOE_ERR_CAPACITY;
+      return MOE_ERR_CUDA;
     }
-    h->host_rows.assign(stage + 1, stage + 1 + R);
-    h->host_tokens.assign(tokens_stage, tokens_stage + R);
-    h->counts_on_host = true;
-    if (host_rows_per_rank) std::memcpy(host_rows_per_rank, stage + 1, sizeof(int32_t) * (size_t)R);
+    rc = count_epilogue(h, stage, host_rows_per_rank);
+    if (rc != MOE_OK) {
+      release(h);
+      return rc;
+    }
   }
   *out_handle = h;
+  return MOE_OK;
+}
+
+int moe_handle_wait(moe_handle_t* h, int32_t* host_rows_per_rank) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (h->epi_pending) {
+    if (cudaEventSynchronize(h->epi_event) != cudaSuccess) return MOE_ERR_CUDA;
+    h->epi_pending = false;
+    h->epi_rc = count_epilogue(h, h->epi_stage, nullptr);
+  }
+  if (h->epi_rc != MOE_OK) return h->epi_rc;
+  if (!h->counts_on_host) return MOE_ERR_INVALID_ARG;  // do_cpu_sync = 0: nothing comes to the host
+  if (host_rows_per_rank)
+    std::memcpy(host_rows_per_rank, h->host_rows.data(), sizeof(int32_t) * h->host_rows.size());
   return MOE_OK;
 }
 
@@ -505,14 +579,62 @@ int64_t moe_handle_row_capacity(const moe_handle_t* h) { return h ? h->row_cap :
 int moe_handle_free(moe_handle_t* h) {
   if (!h) return MOE_OK;
   int rc = MOE_OK;
+  // a deferred count copy still in flight writes into the handle's pinned block: let it land
+  if (h->epi_pending && cudaEventSynchronize(h->epi_event) != cudaSuccess) rc = MOE_ERR_CUDA;
   if (h->block && cudaFreeAsync(h->block, h->stream) != cudaSuccess) rc = MOE_ERR_CUDA;
+  if (h->epi_event && cudaEventDestroy(h->epi_event) != cudaSuccess) rc = MOE_ERR_CUDA;
+  pinned_give(h->epi_stage, h->epi_bytes);
   delete h;
+  return rc;
+}
+
+int moe_event_record(void* stream, moe_event_t** out_event) {
+  if (!out_event) return MOE_ERR_INVALID_ARG;
+  *out_event = nullptr;
+  moe_event_t* e = new (std::nothrow) moe_event_t();
+  if (!e) return MOE_ERR_OOM;
+  if (cudaEventCreateWithFlags(&e->ev, cudaEventDisableTiming) != cudaSuccess) {
+    delete e;
+    return MOE_ERR_CUDA;
+  }
+  if (cudaEventRecord(e->ev, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaEventDestroy(e->ev);
+    delete e;
+    return MOE_ERR_CUDA;
+  }
+  *out_event = e;
+  return MOE_OK;
+}
+
+int moe_event_wait(const moe_event_t* e, void* stream) {
+  if (!e) return MOE_ERR_INVALID_ARG;
+  return cudaStreamWaitEvent(static_cast<cudaStream_t>(stream), e->ev, 0) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_event_synchronize(const moe_event_t* e) {
+  if (!e) return MOE_ERR_INVALID_ARG;
+  return cudaEventSynchronize(e->ev) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_event_query(const moe_event_t* e) {
+  if (!e) return MOE_ERR_INVALID_ARG;
+  const cudaError_t err = cudaEventQuery(e->ev);
+  if (err == cudaSuccess) return MOE_OK;
+  if (err == cudaErrorNotReady) return MOE_NOT_READY;
+  return MOE_ERR_CUDA;
+}
+
+int moe_event_free(moe_event_t* e) {
+  if (!e) return MOE_OK;
+  const int rc = cudaEventDestroy(e->ev) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  delete e;
   return rc;
 }
 
 const char* moe_status_string(int status) {
   switch (status) {
     case MOE_OK: return "ok";
+    case MOE_NOT_READY: return "not complete yet";
     case MOE_ERR_INVALID_ARG: return "invalid argument";
     case MOE_ERR_BAD_EXPERT: return "expert id outside [-1, num_experts)";
     case MOE_ERR_CAPACITY: return "a logical rank needs more rows than the receive capacity";

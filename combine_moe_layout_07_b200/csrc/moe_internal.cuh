@@ -75,7 +75,19 @@ struct moe_handle {
   bool counts_on_host = false;
   std::vector<int32_t> host_rows;    // rows_per_rank, when do_cpu_sync
   std::vector<int32_t> host_tokens;  // tokens_per_rank, when do_cpu_sync
+  // MOE_DEFER_EPILOGUE: the count copy lands in epi_stage (pinned, owned until free) and
+  // epi_event marks its completion; moe_handle_wait finishes the epilogue.
+  int32_t* epi_stage = nullptr;
+  size_t epi_bytes = 0;
+  cudaEvent_t epi_event = nullptr;
+  bool epi_pending = false;
+  int epi_rc = 0;                    // the epilogue's result once run (sticky)
   moe::DeviceArrays d;
+};
+
+// A recorded point on a stream (moe_event_record).
+struct moe_event {
+  cudaEvent_t ev = nullptr;
 };
 
 namespace moe {

@@ -48,6 +48,7 @@ extern "C" {
 #define MOE_ABI_VERSION 1
 
 enum moe_status_code {
+  MOE_NOT_READY = 1,        /* moe_event_query only: the recorded work has not completed yet */
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = -1, /* bad size, flag, null or misaligned pointer */
   MOE_ERR_BAD_EXPERT = -2,  /* a topk_idx entry outside [-1, E) */
@@ -67,6 +68,14 @@ enum moe_dtype { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_E4M3 = 1 };
  * moe_dispatch_by_rank / moe_combine_by_rank / moe_dispatch(do_expand = 0) need (R <= 64). */
 #define MOE_LAYOUT_BY_RANK 1
 
+/* moe_params_t.flags, with do_cpu_sync = 1 only: defer the epilogue of the count sync
+ * ("Why MoE gets stuck on communication", section 2, issue / drain / epilogue: defer_epilogue
+ * moves the host's wait for the receive counts to the wait on the pending work).  moe_layout
+ * then enqueues the copy of the counts into pinned memory owned by the handle and returns at
+ * once, without blocking the host; moe_handle_wait blocks for them and reports the device
+ * conditions.  The handle's device arrays are usable by later stream-ordered calls at once. */
+#define MOE_DEFER_EPILOGUE 2
+
 /* Problem description for moe_layout.  All fields are read once; the handle keeps a copy. */
 typedef struct moe_params {
   int64_t num_tokens;         /* T >= 0 */
@@ -77,7 +86,7 @@ typedef struct moe_params {
   int32_t expert_alignment;   /* A >= 1; T*k + E*A < 2^31 */
   int32_t num_sms;            /* SMs the layout kernels may occupy; 0 = all */
   int32_t do_cpu_sync;        /* 1: moe_layout waits for the counts and copies them to host */
-  int32_t flags;              /* 0 or MOE_LAYOUT_BY_RANK */
+  int32_t flags;              /* 0 or MOE_LAYOUT_BY_RANK | MOE_DEFER_EPILOGUE */
   int64_t recv_capacity_rows; /* cap per rank for the handle's row maps; 0 only with
                                  do_cpu_sync=1 (the rows are then sized from the counts) */
 } moe_params_t;
@@ -102,7 +111,9 @@ int64_t moe_recv_capacity_hint(const moe_params_t* params, int64_t max_tokens_pe
  * tokens_per_rank[R], token_in_rank[T, R] (uint8), slot[T, k] (row inside its rank, -1 if
  * masked), row_src[R, row_cap] (source token, -1 for padding rows), row_w[R, row_cap].
  * With do_cpu_sync = 1 the call blocks until the counts reach the host and returns
- * MOE_ERR_BAD_EXPERT / MOE_ERR_CAPACITY directly (no handle is returned then).
+ * MOE_ERR_BAD_EXPERT / MOE_ERR_CAPACITY directly (no handle is returned then).  With
+ * MOE_DEFER_EPILOGUE as well it does not block: host_rows_per_rank is not written, the handle is
+ * returned, and moe_handle_wait later delivers the counts and those two conditions.
  */
 int moe_layout(const moe_params_t* params, const int64_t* topk_idx, const float* topk_weights,
                void* stream, moe_handle_t** out_handle, int32_t* host_rows_per_rank);
@@ -186,6 +197,41 @@ int moe_combine_backward(const moe_handle_t* handle, const void* grad_out, const
                          void* grad_y, int64_t cap, int do_zero_padding, const void* y,
                          float* grad_weights, int num_sms, void* stream);
 
+/*
+ * The deferred epilogue of a MOE_DEFER_EPILOGUE layout ("Why MoE gets stuck on communication",
+ * section 2: the host waits for the receive counts at wait time, not at issue).  Blocks the host
+ * until the layout's count copy has landed, then returns MOE_ERR_BAD_EXPERT / MOE_ERR_CAPACITY
+ * as moe_layout would have, or MOE_OK with host_rows_per_rank (int32 [R], host, nullable) filled
+ * with the rows each logical rank receives.  The result is kept: later calls return it again
+ * without waiting.  A handle laid out with do_cpu_sync = 1 and no deferral returns MOE_OK (its
+ * counts are already on the host); one laid out with do_cpu_sync = 0 returns
+ * MOE_ERR_INVALID_ARG (its counts never come to the host: use the device arrays).
+ */
+int moe_handle_wait(moe_handle_t* handle, int32_t* host_rows_per_rank);
+
+/*
+ * Events: the pending-object half of "Why MoE gets stuck on communication", section 1 (dispatch
+ * and combine return at once; independent work such as the shared expert runs; wait() orders the
+ * consumer after them) and section 2 (wait() makes the current stream wait on the recorded event;
+ * that orders only that stream, not the host).  To run the round trip on a communication stream
+ * asynchronously to a compute stream: record an event on the compute stream, make the
+ * communication stream wait for it, issue moe_layout / moe_dispatch / moe_combine there, record
+ * an event after them, and make the compute stream wait for that event before it reads the
+ * results.  The handle is freed stream-ordered on its layout stream (moe_handle_free).
+ */
+typedef struct moe_event moe_event_t; /* opaque */
+
+/* Records a new event at the current end of `stream`; *out_event receives it. */
+int moe_event_record(void* stream, moe_event_t** out_event);
+/* Makes work enqueued on `stream` after this call wait for the event (device side; returns at once). */
+int moe_event_wait(const moe_event_t* event, void* stream);
+/* Blocks the host until the event's work has completed. */
+int moe_event_synchronize(const moe_event_t* event);
+/* MOE_OK when the event's work has completed, MOE_NOT_READY while it has not. */
+int moe_event_query(const moe_event_t* event);
+/* Destroys the event (pending waits on it stay valid).  NULL is accepted. */
+int moe_event_free(moe_event_t* event);
+
 /* Waits for `stream`, then returns the handle's device status (MOE_OK, MOE_ERR_BAD_EXPERT,
  * MOE_ERR_CAPACITY or MOE_ERR_TIMEOUT) as left by every layout / dispatch / combine ordered
  * before it. */
@@ -206,7 +252,8 @@ int64_t moe_handle_row_capacity(const moe_handle_t* handle);           /* row_ca
 
 /* Releases the handle.  Its device memory is freed stream-ordered on the layout stream, so
  * every dispatch / combine that uses the handle must be ordered before this call on that
- * stream (or already complete).  NULL is accepted. */
+ * stream (or already complete).  A deferred count copy still in flight is waited for first
+ * (host).  NULL is accepted. */
 int moe_handle_free(moe_handle_t* handle);
 
 /* Static description of a status code. */

@@ -48,7 +48,7 @@ def test_capacity_hint_formula():
     ("hidden", 100, moe.MOE_ERR_INVALID_ARG),           # not a multiple of 8
     ("expert_alignment", 0, moe.MOE_ERR_INVALID_ARG),
     ("num_tokens", -1, moe.MOE_ERR_INVALID_ARG),
-    ("flags", 2, moe.MOE_ERR_INVALID_ARG),               # only MOE_LAYOUT_BY_RANK is defined
+    ("flags", 4, moe.MOE_ERR_INVALID_ARG),               # only MOE_LAYOUT_BY_RANK | MOE_DEFER_EPILOGUE
     ("do_cpu_sync", 2, moe.MOE_ERR_INVALID_ARG),
     ("num_tokens", 1 << 40, moe.MOE_ERR_UNSUPPORTED),   # row indices would overflow int32
 ])
@@ -85,3 +85,21 @@ def test_null_and_misaligned_arguments():
 def test_status_strings():
     for code in range(-8, 1):
         assert moe.status_string(code) and moe.status_string(code) != "unknown status"
+
+
+def test_deferred_epilogue_needs_a_host_sync():
+    p = moe.params(64, 2, 8, 2, 256, 16, recv_capacity_rows=64, do_cpu_sync=False, defer_epilogue=True)
+    h = ctypes.c_void_p(123)
+    rc = moe.lib().moe_layout(ctypes.byref(p), ctypes.c_void_p(0x1000), None, None, ctypes.byref(h), None)
+    assert rc == moe.MOE_ERR_INVALID_ARG and h.value is None
+
+
+def test_wait_and_event_calls_reject_null_on_the_host():
+    L = moe.lib()
+    assert L.moe_handle_wait(None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_event_wait(None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_event_synchronize(None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_event_query(None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_event_record(None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_event_free(None) == moe.MOE_OK
+    assert moe.status_string(moe.MOE_NOT_READY) == "not complete yet"
