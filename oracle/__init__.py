@@ -56,6 +56,7 @@ def lib() -> ctypes.CDLL:
         L.oracle_layout_by_rank.argtypes = [_I64, _I32, _I32, _I32, _P, _P, _P]
         L.oracle_dispatch_by_rank.argtypes = [_I64, _I32, _I32, _I32, _I64, _I64, _P, _P, _P, _P, _I32, _P, _P, _P, _P]
         L.oracle_combine_by_rank.argtypes = [_I64, _I32, _I32, _I32, _I64, _I64, _P, _P, _P, _P, _P]
+        L.oracle_grouped_gemm_f64.argtypes = [_I32, _I32, _I32, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P]
         _lib = L
     return _lib
 
@@ -272,3 +273,20 @@ def combine_by_rank(idx, token_row, y_bits, E: int, R: int, bias_bits=None):
     out = np.zeros((T, H), np.uint16)
     st = lib().oracle_combine_by_rank(T, k, E, R, H, cap, _p(idx), _p(tr), _p(y_bits), _p(bias_bits), _p(out))
     return st, out
+
+
+def grouped_gemm_f64(lay: Layout, codes, scales, w_codes, w_scales, E: int, R: int, A: int):
+    """Expert GEMM over the dispatch layout, binary64 ("From DeepEP to Mega MoE" s3.2 Linear1 and
+    s4.5 GEMM L1 on the expert buffer): (status, out float64 [R, cap, N]); rows outside every
+    expert range stay NaN."""
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.float32)
+    w_codes = _c(w_codes, np.uint8)
+    w_scales = _c(w_scales, np.float32)
+    _, cap, H = codes.shape
+    N = w_codes.shape[1]
+    out = np.full((R, cap, N), np.nan, np.float64)
+    st = lib().oracle_grouped_gemm_f64(E, R, A, cap, H, N, _p(lay.cnt), _p(lay.psum), _p(codes), _p(scales),
+                                       _p(w_codes), _p(w_scales), _p(out))
+    return st, out
+

@@ -19,6 +19,9 @@
  *        intensity" (do_cpu_sync=False exposes psum_num_recv_tokens_per_expert).
  *   [P5] "Chapter 2: repository map and module responsibilities" (bowenzhou.top),
  *        section 2.1, the layout.cu row (rank count, expert count, membership).
+ *   [P1] again for the expert GEMM: section 3.2 (Linear1, the first expert GEMM, fed by the
+ *        dispatched tokens and their scale factors) and section 4.5 (the separated dataflow:
+ *        dispatch -> expert buffer in HBM -> GEMM L1).
  *
  * Conventions shared with the library's C ABI (argument meaning only, no code):
  *   T tokens, k top-k, E experts, R logical ranks, E_loc = E/R, A = expert_alignment.
@@ -554,3 +557,45 @@ int oracle_combine_by_rank(int64_t T, int k, int E, int R, int64_t H, int64_t ca
     free(seen);
     return status;
 }
+
+/*
+ * Expert GEMM over the dispatch layout ([P1] 3.2 Linear1 and 4.5 GEMM L1 on the expert buffer;
+ * [P3] 1: expert_alignment is the grouped GEMM's row alignment).  Inputs are the FP8 dispatch
+ * output (codes qx [R, cap, H] and 1x128 scales sx [R, cap, H/128]) and per-expert FP8 weights
+ * (codes qw [E, N, H], row n = output column n, and 128x128 block scales sw [E, N/128, H/128]).
+ * For every logical rank r, every expert e of r and every row of e's range
+ * [psum[e] - align_up(cnt[e], A), psum[e]) (routed rows and padding rows alike), and n < N:
+ *   out[r, row, n] = sum over K-blocks b of ( sx[r, row, b] * sw[e, n / 128, b]
+ *                    * sum over h in block b of E4M3(qx[r, row, h]) * E4M3(qw[e, n, h]) )
+ * in binary64, blocks and columns in ascending order.  Rows outside every range are not
+ * written.  Needs H % 128 == 0 and N % 128 == 0; returns -1 otherwise.
+ */
+int oracle_grouped_gemm_f64(int E, int R, int A, int64_t cap, int64_t H, int64_t N, const int32_t* cnt,
+                            const int32_t* psum, const uint8_t* qx, const float* sx, const uint8_t* qw,
+                            const float* sw, double* out) {
+    if (H % 128 != 0 || N % 128 != 0 || E % R != 0) return -1;
+    const int E_loc = E / R;
+    const int64_t KB = H / 128, NB = N / 128;
+    for (int e = 0; e < E; ++e) {
+        const int r = e / E_loc;
+        const int64_t end = psum[e], begin = end - align_up(cnt[e], A);
+        for (int64_t row = begin; row < end; ++row) {
+            const uint8_t* x = qx + ((int64_t)r * cap + row) * H;
+            const float* xs = sx + ((int64_t)r * cap + row) * KB;
+            for (int64_t n = 0; n < N; ++n) {
+                const uint8_t* wr = qw + ((int64_t)e * N + n) * H;
+                const float* ws = sw + ((int64_t)e * NB + n / 128) * KB;
+                double acc = 0.0;
+                for (int64_t b = 0; b < KB; ++b) {
+                    double dot = 0.0;
+                    for (int64_t h = b * 128; h < b * 128 + 128; ++h)
+                        dot += oracle_e4m3_to_double(x[h]) * oracle_e4m3_to_double(wr[h]);
+                    acc += (double)xs[b] * (double)ws[b] * dot;
+                }
+                out[((int64_t)r * cap + row) * N + n] = acc;
+            }
+        }
+    }
+    return 0;
+}
+

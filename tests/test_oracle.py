@@ -508,3 +508,107 @@ def test_by_rank_dispatch_copies_and_topk_views():
     members = np.array([[tr[t, r] >= 0 for r in range(R)] for t in range(wl.tokens)]).sum(1)
     expect = bits((x.float() * torch.from_numpy(members).float()[:, None]).to(torch.bfloat16))
     assert (out == expect).all()
+
+
+# ----------------------------------------------------------------------------- expert GEMM
+def _gemm_case(H=256, N=256, mask=0.1):
+    wl = W.WORKLOADS["tiny"].with_(hidden=H, fp8=True, tokens_per_rank=40, experts=4, topk=2, alignment=128)
+    idx, w = W.gen_routing(wl)
+    idx = W.mask_entries(wl, idx, mask)
+    x = W.gen_x(wl)
+    E, R, A = wl.experts, wl.ranks, wl.alignment
+    lay = oracle.layout(idx.numpy(), w.numpy(), E, R, A)
+    cap = int(lay.rows_per_rank.max()) + 5
+    lay = oracle.layout(idx.numpy(), w.numpy(), E, R, A, cap=cap)
+    st, codes, scales, _ = oracle.dispatch_fp8(lay, idx.numpy(), w.numpy(), bits(x), E, R, A, cap, True, fill=0)
+    assert st == oracle.OK
+    return wl, idx.numpy(), lay, codes, scales
+
+
+def _e4m3_table():
+    return np.array([oracle.e4m3_to_double(c) for c in range(256)], np.float64)
+
+
+def test_grouped_gemm_identity_weights_return_the_dequantised_rows():
+    """W_e = I (code 0x38 = 1.0 on the diagonal, scale 1): every row of every expert comes back
+    as its dequantised dispatch row, exactly (one nonzero product per output)."""
+    wl, _, lay, codes, scales = _gemm_case()
+    E, R, A, H = wl.experts, wl.ranks, wl.alignment, wl.hidden
+    qw = np.zeros((E, H, H), np.uint8)
+    qw[:, np.arange(H), np.arange(H)] = 0x38
+    sw = np.ones((E, H // 128, H // 128), np.float32)
+    st, out = oracle.grouped_gemm_f64(lay, codes, scales, qw, sw, E, R, A)
+    assert st == 0
+    deq = _e4m3_table()[codes] * np.repeat(scales.astype(np.float64), 128, axis=2)
+    for r in range(R):
+        n = int(lay.rows_per_rank[r])
+        assert (out[r, :n] == deq[r, :n]).all()
+        assert np.isnan(out[r, n:]).all()          # rows beyond the rank's rows untouched
+
+
+def test_grouped_gemm_selects_each_rows_expert_and_block_scales():
+    """All-ones weights with scale (e + 1) * (c + 1) * 2^b for column block c and K-block b:
+    out[row, n] = (e + 1) * (n // 128 + 1) * sum_b 2^b * sx[row, b] * sum_{h in b} deq(x[row, h])
+    for the row's expert e, read from the routing (row slot[t, j] of expert idx[t, j]); padding
+    rows, zero-filled, give 0."""
+    wl, idx, lay, codes, scales = _gemm_case(H=384, N=256)
+    E, R, A, H, N = wl.experts, wl.ranks, wl.alignment, wl.hidden, 256
+    KB = H // 128
+    qw = np.full((E, N, H), 0x38, np.uint8)
+    sw = np.empty((E, N // 128, KB), np.float32)
+    for e in range(E):
+        for c in range(N // 128):
+            for b in range(KB):
+                sw[e, c, b] = (e + 1) * (c + 1) * 2.0 ** b
+    st, out = oracle.grouped_gemm_f64(lay, codes, scales, qw, sw, E, R, A)
+    assert st == 0
+    table = _e4m3_table()
+    e_loc = E // R
+    seen = np.zeros((R, codes.shape[1]), bool)
+    T, k = idx.shape
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            if e < 0:
+                continue
+            r, row = e // e_loc, int(lay.slot[t, j])
+            blocks = table[codes[r, row]].reshape(KB, 128).sum(axis=1)
+            base = (e + 1) * sum(2.0 ** b * float(scales[r, row, b]) * blocks[b] for b in range(KB))
+            ref = base * (np.arange(N) // 128 + 1)
+            assert np.allclose(out[r, row], ref, rtol=1e-12, atol=0), (t, j)
+            seen[r, row] = True
+    for r in range(R):
+        n = int(lay.rows_per_rank[r])
+        assert (out[r, :n][~seen[r, :n]] == 0).all()   # padding rows
+
+
+def test_grouped_gemm_is_linear_in_the_weight_scales():
+    wl, _, lay, codes, scales = _gemm_case(H=256, N=128)
+    E, R, A, H = wl.experts, wl.ranks, wl.alignment, wl.hidden
+    rng = np.random.default_rng(3)
+    qw = rng.integers(0, 256, (E, 128, H), dtype=np.uint8)
+    qw[(qw & 0x7F) == 0x7F] = 0                        # no NaN codes
+    sw = rng.uniform(0.5, 2.0, (E, 1, H // 128)).astype(np.float32)
+    st, a = oracle.grouped_gemm_f64(lay, codes, scales, qw, sw, E, R, A)
+    st2, b = oracle.grouped_gemm_f64(lay, codes, scales, qw, (sw * 2).astype(np.float32), E, R, A)
+    assert st == st2 == 0
+    ok = ~np.isnan(a)
+    assert (b[ok] == 2 * a[ok]).all()                  # a power-of-two scale is exact
+    # swapping two experts' weights swaps nothing else: experts keep their own rows
+    qw2, sw2 = qw.copy(), sw.copy()
+    qw2[[0, 1]], sw2[[0, 1]] = qw[[1, 0]], sw[[1, 0]]
+    st3, c = oracle.grouped_gemm_f64(lay, codes, scales, qw2, sw2, E, R, A)
+    assert st3 == 0
+    e_loc = E // R
+    for e in range(2, E):                              # rows of experts 2.. are unchanged
+        r = e // e_loc
+        end = int(lay.psum[e]); beg = end - align_up(int(lay.cnt[e]), A)
+        assert (c[r, beg:end] == a[r, beg:end]).all()
+
+
+def test_grouped_gemm_rejects_unaligned_shapes():
+    wl, _, lay, codes, scales = _gemm_case()
+    E, R, A = wl.experts, wl.ranks, wl.alignment
+    st, _ = oracle.grouped_gemm_f64(lay, codes, scales, np.zeros((E, 100, 256), np.uint8),
+                                    np.ones((E, 1, 2), np.float32), E, R, A)
+    assert st == -1

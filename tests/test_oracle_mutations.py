@@ -30,6 +30,12 @@ MUTATIONS = [
     ("combine drops the bias", "            if (bias) acc = acc + oracle_bf16_to_float(bias[t * H + h]);\n            out[t * H + h] = oracle_float_to_bf16(acc);\n        }\n    return status;\n}\n\n/* The same sum",
      "            out[t * H + h] = oracle_float_to_bf16(acc);\n        }\n    return status;\n}\n\n/* The same sum"),
     ("bf16 rounding truncates", "    if (lo > 0x8000u || (lo == 0x8000u && (hi & 1u))) hi += 1;", "    (void)lo;"),
+    ("expert GEMM uses the next expert's weights", "const uint8_t* wr = qw + ((int64_t)e * N + n) * H;",
+     "const uint8_t* wr = qw + ((int64_t)((e + 1) % E) * N + n) * H;"),
+    ("expert GEMM reads the first weight-scale block", "const float* ws = sw + ((int64_t)e * NB + n / 128) * KB;",
+     "const float* ws = sw + ((int64_t)e * NB) * KB;"),
+    ("expert GEMM drops the row scale", "acc += (double)xs[b] * (double)ws[b] * dot;",
+     "acc += (double)ws[b] * dot;"),
 ]
 
 
