@@ -390,6 +390,44 @@ def skewed_overlap(step, stream, dev, n_steps: int = 50) -> dict:
 
 
 # --------------------------------------------------------------------------- our arm
+def expert_gemm_measurement(moe, wl, h, x, cap: int, N: int, stream, dev, iters: int = 5) -> dict:
+    """The first expert GEMM on this step's FP8 dispatch output, timed alone with CUDA events:
+    out [R, cap, N] = per-expert E4M3 x E4M3 GEMM over K = H with 1x128 row scales and 128x128
+    weight scales (synthetic weights).  FLOPs count every row the GEMM computes (routed rows and
+    alignment padding); the peak is the measured bf16 burst x 2 (the FP8 / BF16 nominal ratio)."""
+    E, R, H = wl.experts, wl.ranks, wl.hidden
+    g = torch.Generator(device=dev).manual_seed(21)
+    qw = torch.randint(0, 256, (E, N, H), generator=g, dtype=torch.uint8, device=dev)
+    qw[(qw & 0x7F) == 0x7F] = 0x38
+    sw = torch.rand((E, N // 128, H // 128), generator=g, device=dev) / 64 + 1 / 256
+    recv = torch.empty(R, cap, H, dtype=torch.uint8, device=dev)
+    sc = torch.empty(R, cap, H // 128, dtype=torch.float32, device=dev)
+    out = torch.empty(R, cap, N, dtype=torch.bfloat16, device=dev)
+    moe.moe_dispatch(h, x, moe.MOE_DTYPE_FP8_E4M3, recv, sc, None, cap=cap, stream=stream)
+    rows = int(torch.clamp(h.rows_per_rank(), max=cap).sum())
+    for _ in range(2):
+        moe.moe_expert_gemm_fp8(h, recv, sc, qw, sw, out, cap=cap, stream=stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(iters):
+        moe.moe_expert_gemm_fp8(h, recv, sc, qw, sw, out, cap=cap, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / iters
+    flops = 2.0 * rows * N * H
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    bf16 = float(peaks.get("bf16_tflops", 1590.0))
+    peak = 2.0 * bf16
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"kernel": "k_expert_gemm", "bound": "tensor", "N": N, "K": H, "rows": rows, "ms": ms,
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_source": ("measured bf16 burst x 2 (MEASURED_PEAKS.json bf16_tflops; fp8/bf16 nominal ratio 2)"
+                            if "bf16_tflops" in peaks else "fallback 1.59 PFLOP/s bf16 x 2"),
+            "iters": iters}
+
+
 def run_ours(args) -> int:
     world, rank, local = dist_setup("nccl")
     torch.cuda.set_device(local)
@@ -501,6 +539,12 @@ def run_ours(args) -> int:
     e2e = None if args.no_e2e else run_e2e(args, world, dev, stream, step, step_bytes, x, idx, w, y, bias, out,
                                            x_c, idx_c, w_c, bias_c)
     extras = {}
+    if args.expert_gemm:
+        if not wl.fp8 or wl.alignment % 128 or wl.hidden % 128 or args.expert_gemm % 128:
+            raise SystemExit("--expert-gemm needs an FP8 workload, expert_alignment and N multiples of 128")
+        hg = moe.moe_layout(make_params(cap), idx, w, stream=stream)
+        extras["expert_gemm"] = expert_gemm_measurement(moe, wl, hg, x, cap, args.expert_gemm, stream, dev)
+        moe.moe_handle_free(hg)
     if wl.name == "decode":
         extras["latency"] = decode_latency(step_parts, stream, dev)
     if wl.name == "skewed":
@@ -556,6 +600,8 @@ def main() -> int:
     ap.add_argument("--cpu-tokens", type=int, default=16384, help="tokens in the CPU-oracle baseline sample")
     ap.add_argument("--ref-tokens", type=int, default=4096, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--expert-gemm", type=int, default=0, metavar="N",
+                    help="also time the first expert GEMM (E4M3, K = hidden, N output columns) on the dispatch output")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--tokens-per-rank", type=int, default=0, help="override the workload's tokens per rank "
                     "(smaller cases for profiling)")

@@ -91,6 +91,7 @@ def lib() -> ctypes.CDLL:
         L.moe_handle_row_capacity.restype = _I64
         L.moe_handle_free.argtypes = [_P]
         L.moe_handle_wait.argtypes = [_P, _P]
+        L.moe_expert_gemm_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, _P]
         L.moe_event_record.argtypes = [_P, ctypes.POINTER(_P)]
         for name in ("wait",):
             getattr(L, f"moe_event_{name}").argtypes = [_P, _P]
@@ -331,3 +332,16 @@ class Event:
 
 def moe_event_record(stream=None) -> Event:
     return Event(stream)
+
+
+def moe_expert_gemm_fp8(handle: Handle, recv_x: torch.Tensor, recv_scales: torch.Tensor, w: torch.Tensor,
+                        w_scales: torch.Tensor, out: torch.Tensor, cap: Optional[int] = None, num_sms: int = 0,
+                        stream=None) -> None:
+    """The first expert GEMM on an FP8 dispatch's output: out [R, cap, N] (bf16) from recv_x
+    [R, cap, H] (E4M3 codes as uint8), recv_scales, w [E, N, H] (E4M3 codes) and w_scales
+    [E, N/128, H/128]."""
+    cap = recv_x.shape[1] if cap is None else cap
+    rc = lib().moe_expert_gemm_fp8(handle.ptr, _ptr(recv_x), _ptr(recv_scales), _ptr(w), _ptr(w_scales), _ptr(out),
+                                   w.shape[1], cap, num_sms, _stream(stream))
+    _check(rc, "moe_expert_gemm_fp8")
+

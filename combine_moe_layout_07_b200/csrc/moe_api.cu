@@ -588,6 +588,38 @@ int moe_handle_free(moe_handle_t* h) {
   return rc;
 }
 
+int moe_expert_gemm_fp8(const moe_handle_t* h, const void* recv_x, const float* recv_scales, const void* w,
+                        const float* w_scales, void* out, int64_t N, int64_t cap, int num_sms, void* stream) {
+  if (!h || !recv_x || !recv_scales || !w || !w_scales || !out) return MOE_ERR_INVALID_ARG;
+  if (N <= 0 || cap < 1 || num_sms < 0) return MOE_ERR_INVALID_ARG;
+  const moe_params_t& p = h->p;
+  const int64_t H = p.hidden, R = p.num_logical_ranks, E = p.num_experts;
+  if (H % 128 != 0 || N % 128 != 0 || p.expert_alignment % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (R * cap >= (int64_t)1 << 31 || E * N >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+  if (expert_gemm_smem_bytes((int)R, (int)E) > 227u * 1024u) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(recv_x) || !aligned16(w) || !aligned16(out) || !aligned4(recv_scales) || !aligned4(w_scales))
+    return MOE_ERR_INVALID_ARG;
+  if (h->counts_on_host)
+    for (int32_t v : h->host_rows)
+      if (v > cap) return MOE_ERR_CAPACITY;
+  GemmLaunch L{};
+  L.psum = h->d.psum;
+  L.rows_per_rank = h->d.rows_per_rank;
+  L.sx = recv_scales;
+  L.sw = w_scales;
+  L.out = out;
+  L.cap = cap;
+  L.N = N;
+  L.R = (int)R;
+  L.E = (int)E;
+  L.E_loc = (int)(E / R);
+  L.NB = (int)(N / 128);
+  L.KB = (int)(H / 128);
+  L.grid = grid_for(num_sms, h->device);
+  L.status = h->d.status;
+  return launch_expert_gemm(L, recv_x, w, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 int moe_event_record(void* stream, moe_event_t** out_event) {
   if (!out_event) return MOE_ERR_INVALID_ARG;
   *out_event = nullptr;

@@ -167,6 +167,21 @@ struct GradWeightsLaunch {
 
 cudaError_t launch_grad_weights(const GradWeightsLaunch& L, cudaStream_t s);
 
+struct GemmLaunch {
+  const int32_t* psum;           // handle: inclusive aligned prefix per rank [E]
+  const int32_t* rows_per_rank;  // handle [R]
+  const float* sx;               // [R, cap, KB] row scales of the dispatched rows
+  const float* sw;               // [E, NB, KB] weight block scales
+  void* out;                     // bf16 [R, cap, N]
+  int64_t cap, N;
+  int R, E, E_loc, NB, KB;
+  int grid;
+  int32_t* status;
+};
+
+cudaError_t launch_expert_gemm(const GemmLaunch& L, const void* x, const void* w, cudaStream_t s);
+uint32_t expert_gemm_smem_bytes(int R, int E);
+
 void note_launch(int n = 1);
 int sm_count(int device);
 

@@ -232,6 +232,29 @@ int moe_event_query(const moe_event_t* event);
 /* Destroys the event (pending waits on it stay valid).  NULL is accepted. */
 int moe_event_free(moe_event_t* event);
 
+/*
+ * The first expert GEMM on the FP8 dispatch layout, on the tensor cores ("From DeepEP to Mega MoE"
+ * 3.2 Linear1 and 4.5: dispatch -> expert buffer -> GEMM L1; "Why MoE gets stuck on
+ * communication" 1: expert_alignment is the grouped GEMM's row alignment).  For every logical
+ * rank r, every expert e of r and every row of e's range [psum[e] - align_up(cnt[e], A), psum[e]):
+ *   out[r, row, n] = bf16( sum over K-blocks b of recv_scales[r, row, b] * w_scales[e, n/128, b]
+ *                          * sum over h in block b of E4M3(recv_x[r, row, h]) * E4M3(w[e, n, h]) )
+ * Each 128-wide K-block is summed on the tensor cores (fp32), then scaled and added in fp32 in
+ * ascending b; one rounding to bf16 (nearest even) at the end.
+ *   recv_x       E4M3 [R, cap, H] and recv_scales fp32 [R, cap, H/128]: an FP8 moe_dispatch's output
+ *                for this handle (do_expand = 1).
+ *   w            E4M3 [E, N, H]: row n of expert e is output column n (K contiguous).
+ *   w_scales     fp32 [E, N/128, H/128]: one scale per 128 x 128 block of w.
+ *   out          bf16 [R, cap, N]: the rows of every expert range are written (padding rows too:
+ *                zero when the dispatch zeroed them); other rows are not touched.
+ * Needs H % 128 == 0, N % 128 == 0 and expert_alignment % 128 == 0, and R * cap and E * N below
+ * 2^31 (MOE_ERR_UNSUPPORTED otherwise); recv_x, w and out 16-byte aligned.  Returns
+ * MOE_ERR_CAPACITY when the host counts exceed cap; without host counts, rows beyond cap are not
+ * computed (the layout's status reports the overflow).  Stream-ordered after the dispatch.
+ */
+int moe_expert_gemm_fp8(const moe_handle_t* handle, const void* recv_x, const float* recv_scales, const void* w,
+                        const float* w_scales, void* out, int64_t N, int64_t cap, int num_sms, void* stream);
+
 /* Waits for `stream`, then returns the handle's device status (MOE_OK, MOE_ERR_BAD_EXPERT,
  * MOE_ERR_CAPACITY or MOE_ERR_TIMEOUT) as left by every layout / dispatch / combine ordered
  * before it. */
