@@ -6,8 +6,8 @@ tensor cores, the blocks are scaled and summed in fp32, and the result is rounde
 With M = sum_b |sx * sw| * sum_h |qx * qw| (the magnitude the sums run over):
     |got - ref| <= 2^-8 |ref| + 2^-10 M
 bf16 rounding is at most 2^-9 |result|.  The tensor cores sum E4M3 products with fewer
-accumulator bits than fp32: on these inputs the error reaches about 2^-12.2 M, which 2^-10 M
-covers four times over while a lost K-block or a wrong scale (errors near M / 50) still fails.
+accumulator bits than fp32, which the M term covers: the worst error on these cases is 0.65 of
+the bound, while a lost K-block or a wrong scale (errors near M / 50) fails by far.
 The identity case below has one nonzero product per output, so no accumulation error at all:
 it must match bit for bit.  Rows outside the expert ranges must keep their fill pattern.
 """
