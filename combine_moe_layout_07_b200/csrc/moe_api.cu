@@ -118,28 +118,27 @@ static void pinned_give(void* p, size_t n) {
   g_pin_free.emplace_back(n, p);
 }
 
-// Staging of the do_cpu_sync copy: [unused][rows_per_rank R][status 4, ticket, pad 3][tokens R].
-static size_t count_stage_bytes(int64_t R) { return sizeof(int32_t) * (size_t)(9 + 2 * R); }
+// The do_cpu_sync copy: the handle keeps [status 4, ticket, pad 3][tokens_per_rank R]
+// [rows_per_rank R] adjacent, so one copy brings flags and counts to the host.
+static size_t count_stage_bytes(int64_t R) { return sizeof(int32_t) * (size_t)(8 + 2 * R); }
 
 static cudaError_t enqueue_count_copy(const moe_handle_t* h, int32_t* stage, cudaStream_t s) {
-  const int64_t R = h->p.num_logical_ranks;
-  cudaError_t err = cudaMemcpyAsync(stage + 1 + R, h->d.status, (size_t)(32 + 4 * R), cudaMemcpyDeviceToHost, s);
-  if (err == cudaSuccess) err = cudaMemcpyAsync(stage + 1, h->d.rows_per_rank, 4 * R, cudaMemcpyDeviceToHost, s);
-  return err;
+  return cudaMemcpyAsync(stage, h->d.status, count_stage_bytes(h->p.num_logical_ranks), cudaMemcpyDeviceToHost, s);
 }
 
 // The do_cpu_sync epilogue once the copy into `stage` is complete: the status flags decide the
 // result; on success the host counts are kept on the handle (and copied to host_rows_per_rank).
 static int count_epilogue(moe_handle_t* h, const int32_t* stage, int32_t* host_rows_per_rank) {
   const int64_t R = h->p.num_logical_ranks;
-  const int32_t flags = stage[1 + R];
+  const int32_t flags = stage[0];
   if (flags & kStatusBadExpert) return MOE_ERR_BAD_EXPERT;
   if (flags & kStatusCapacity) return MOE_ERR_CAPACITY;
-  const int32_t* tokens = stage + 1 + R + 8;
-  h->host_rows.assign(stage + 1, stage + 1 + R);
+  const int32_t* tokens = stage + 8;
+  const int32_t* rows = tokens + R;
+  h->host_rows.assign(rows, rows + R);
   h->host_tokens.assign(tokens, tokens + R);
   h->counts_on_host = true;
-  if (host_rows_per_rank) std::memcpy(host_rows_per_rank, stage + 1, sizeof(int32_t) * (size_t)R);
+  if (host_rows_per_rank) std::memcpy(host_rows_per_rank, rows, sizeof(int32_t) * (size_t)R);
   return MOE_OK;
 }
 
@@ -223,8 +222,9 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
     off = align_up64(off + bytes, 256);
     return at;
   };
-  // status[4], the scan ticket and tokens_per_rank[R] are adjacent: one memset clears them
-  const int64_t o_status = take(32 + 4 * R), o_rows = take(4 * R), o_cnt = take(4 * E), o_psum = take(4 * E),
+  // status[4], the scan ticket, tokens_per_rank[R] and rows_per_rank[R] are adjacent: one memset
+  // clears the first three (the kernels write every row count), one copy reads them all back
+  const int64_t o_status = take(32 + 8 * R), o_cnt = take(4 * E), o_psum = take(4 * E),
                 o_pad = take(4 * (E + 1)), o_tir = take(T * R), o_slot = take(4 * T * k),
                 o_prank = take(4 * T * k), o_pw = take(4 * T * k), o_ccnt = take(4 * C * E),
                 o_rsrc = take(4 * R * h->row_cap), o_rw = take(4 * R * h->row_cap);
@@ -242,7 +242,7 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   d.status = reinterpret_cast<int32_t*>(b + o_status);
   d.ticket = d.status + 4;
   d.tokens_per_rank = d.status + 8;
-  d.rows_per_rank = reinterpret_cast<int32_t*>(b + o_rows);
+  d.rows_per_rank = d.tokens_per_rank + R;
   d.cnt = reinterpret_cast<int32_t*>(b + o_cnt);
   d.psum = reinterpret_cast<int32_t*>(b + o_psum);
   d.pad_excl = reinterpret_cast<int32_t*>(b + o_pad);
