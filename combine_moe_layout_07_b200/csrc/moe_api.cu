@@ -13,6 +13,7 @@
 #include <new>
 
 #include "moe_internal.cuh"
+#include "trace.cuh"
 
 namespace moe {
 
@@ -183,6 +184,7 @@ int64_t moe_recv_capacity_hint(const moe_params_t* p, int64_t max_tokens_per_ran
 
 int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk_weights, void* stream,
                moe_handle_t** out_handle, int32_t* host_rows_per_rank) {
+  TraceRange trace("moe_layout");
   if (!out_handle) return MOE_ERR_INVALID_ARG;
   *out_handle = nullptr;
   int rc = check_params(p);
@@ -330,6 +332,7 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
 }
 
 int moe_handle_wait(moe_handle_t* h, int32_t* host_rows_per_rank) {
+  TraceRange trace("moe_handle_wait");
   if (!h) return MOE_ERR_INVALID_ARG;
   if (h->epi_pending) {
     if (cudaEventSynchronize(h->epi_event) != cudaSuccess) return MOE_ERR_CUDA;
@@ -346,6 +349,7 @@ int moe_handle_wait(moe_handle_t* h, int32_t* host_rows_per_rank) {
 int moe_dispatch(const moe_handle_t* h, const void* x, int out_dtype, void* recv_x, float* recv_scales,
                  float* recv_weights, int64_t cap, int do_expand, int do_zero_padding, int num_sms,
                  void* stream) {
+  TraceRange trace("moe_dispatch");
   if (!h) return MOE_ERR_INVALID_ARG;
   if (do_expand != 0 && do_expand != 1) return MOE_ERR_INVALID_ARG;
   if (do_zero_padding != 0 && do_zero_padding != 1) return MOE_ERR_INVALID_ARG;
@@ -389,6 +393,7 @@ int moe_dispatch(const moe_handle_t* h, const void* x, int out_dtype, void* recv
 
 int moe_combine(const moe_handle_t* h, const void* y, const float* topk_weights, const void* bias, void* out,
                 int64_t cap, int num_sms, void* stream) {
+  TraceRange trace("moe_combine");
   if (!h) return MOE_ERR_INVALID_ARG;
   if (cap < 0 || cap >= (int64_t)1 << 31 || num_sms < 0) return MOE_ERR_INVALID_ARG;
   const moe_params_t& p = h->p;
@@ -419,6 +424,7 @@ int moe_combine(const moe_handle_t* h, const void* y, const float* topk_weights,
 int moe_dispatch_by_rank(const moe_handle_t* h, const void* x, const int64_t* topk_idx, int out_dtype, void* recv_x,
                          float* recv_scales, int32_t* recv_topk_idx, float* recv_topk_weights, int64_t cap,
                          int num_sms, void* stream) {
+  TraceRange trace("moe_dispatch_by_rank");
   if (!h) return MOE_ERR_INVALID_ARG;
   if (out_dtype != MOE_DTYPE_BF16 && out_dtype != MOE_DTYPE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
   if (cap < 0 || cap >= (int64_t)1 << 31 || num_sms < 0) return MOE_ERR_INVALID_ARG;
@@ -463,6 +469,7 @@ int moe_dispatch_by_rank(const moe_handle_t* h, const void* x, const int64_t* to
 
 int moe_combine_by_rank(const moe_handle_t* h, const void* y, const void* bias, void* out, int64_t cap, int num_sms,
                         void* stream) {
+  TraceRange trace("moe_combine_by_rank");
   if (!h) return MOE_ERR_INVALID_ARG;
   if (cap < 0 || cap >= (int64_t)1 << 31 || num_sms < 0) return MOE_ERR_INVALID_ARG;
   const moe_params_t& p = h->p;
@@ -494,6 +501,7 @@ int moe_combine_by_rank(const moe_handle_t* h, const void* y, const void* bias, 
 int moe_combine_backward(const moe_handle_t* h, const void* grad_out, const float* topk_weights, void* grad_y,
                          int64_t cap, int do_zero_padding, const void* y, float* grad_weights, int num_sms,
                          void* stream) {
+  TraceRange trace("moe_combine_backward");
   if (!h) return MOE_ERR_INVALID_ARG;
   if (cap < 0 || cap >= (int64_t)1 << 31 || num_sms < 0) return MOE_ERR_INVALID_ARG;
   if (do_zero_padding != 0 && do_zero_padding != 1) return MOE_ERR_INVALID_ARG;
@@ -548,6 +556,7 @@ int moe_combine_backward(const moe_handle_t* h, const void* grad_out, const floa
 }
 
 int moe_handle_status(const moe_handle_t* h, void* stream) {
+  TraceRange trace("moe_handle_status");
   if (!h) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* stage = static_cast<int32_t*>(g_stage.get(16));
@@ -577,6 +586,7 @@ const int32_t* moe_handle_token_rows(const moe_handle_t* h) { return h ? h->d.to
 int64_t moe_handle_row_capacity(const moe_handle_t* h) { return h ? h->row_cap : -1; }
 
 int moe_handle_free(moe_handle_t* h) {
+  TraceRange trace("moe_handle_free");
   if (!h) return MOE_OK;
   int rc = MOE_OK;
   // a deferred count copy still in flight writes into the handle's pinned block: let it land
@@ -590,6 +600,7 @@ int moe_handle_free(moe_handle_t* h) {
 
 int moe_expert_gemm_fp8(const moe_handle_t* h, const void* recv_x, const float* recv_scales, const void* w,
                         const float* w_scales, void* out, int64_t N, int64_t cap, int num_sms, void* stream) {
+  TraceRange trace("moe_expert_gemm_fp8");
   if (!h || !recv_x || !recv_scales || !w || !w_scales || !out) return MOE_ERR_INVALID_ARG;
   if (N <= 0 || cap < 1 || num_sms < 0) return MOE_ERR_INVALID_ARG;
   const moe_params_t& p = h->p;
@@ -644,6 +655,7 @@ int moe_event_wait(const moe_event_t* e, void* stream) {
 }
 
 int moe_event_synchronize(const moe_event_t* e) {
+  TraceRange trace("moe_event_synchronize");
   if (!e) return MOE_ERR_INVALID_ARG;
   return cudaEventSynchronize(e->ev) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
