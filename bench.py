@@ -51,9 +51,15 @@ def algorithmic_bytes(wl: W.Workload, valid_pairs: int, pad_rows: int, weighted:
 
 
 def kernel_source_digest(*files: str) -> str:
+    """sha256 (first 12 hex digits) of the kernel's sources with comments and blank lines removed,
+    so that a traffic record stays tied to the code it measured but survives comment edits."""
     h = hashlib.sha256()
     for f in files:
-        h.update(open(os.path.join(ROOT, "combine_moe_layout_07_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "combine_moe_layout_07_b200", "csrc", f)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        code = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+        h.update(code.encode())
     return h.hexdigest()[:12]
 
 

@@ -7,16 +7,21 @@
 // do_expand / do_zero_padding of "Why MoE gets stuck on communication" (locsic.com) section 1 and
 // FP8 dispatch of "DeepEP expert-parallel communication" (blog.hotdry.top), key techniques.
 //
-// B200 mapping (HBM-bound data movement, one CTA per SM so num_sms caps SMs):
-//   warp 0      producer: per token, computes the destination rows from the handle and issues
-//               one cp.async.bulk load of the bf16 row into a ring of shared-memory stages
-//               (mbarrier full/empty pairs), so several rows per SM are always in flight;
-//   warps 1..16 two consumer groups of 8 warps take alternate tokens; they read the staged row
-//               from shared memory and write it, from registers,
-//               to each of its k destination rows with 16-byte evict-first stores.  FP8: eight
-//               lanes own a 1x128 block, amax by three xor-shuffles, inv = 448/a and a/448 as IEEE
-//               divisions, codes by cvt.rn.satfinite.e4m3x2.  Each warp releases the stage on its
-//               mbarrier when done.
+// B200 mapping (HBM-bound data movement, one CTA per SM so num_sms caps SMs).  Two kernels share
+// the producer (dispatch_producer) and the padding pass (zero_padding_rows):
+//   k_dispatch_bulk   every dispatch except the weight-scaled rows of the combine backward.  A
+//                     storer warp writes each row to its destinations with cp.async.bulk stores
+//                     from shared memory (BF16: straight from the loaded stage; FP8: from an
+//                     output stage the quantising consumer warps fill); see its own comment.
+//   k_dispatch        the register-store form, for rows that differ per destination
+//                     (bf16(w * g) of the backward).  Warp 0 is the producer: per token it
+//                     computes the destination rows from the handle and issues one
+//                     cp.async.bulk load of the bf16 row into a ring of shared-memory stages
+//                     (mbarrier full/empty pairs); warps 1..16 form two consumer groups of 8 warps
+//                     that take alternate tokens, read the staged row and write it, from
+//                     registers, to each destination with 16-byte evict-first stores.
+//   FP8 (both): eight lanes own a 1x128 block, amax by three xor-shuffles, inv = 448/a and a/448
+//   as IEEE divisions, codes by cvt.rn.satfinite.e4m3x2.
 //   Padding rows are zeroed by the consumer warps after the tokens, a warp per row.
 // Every wait is an mbarrier try_wait bounded by wall-clock time (status kStatusTimeout on
 // expiry); there are no named barriers.
