@@ -133,6 +133,20 @@ def test_fused_and_three_kernel_layouts_at_the_boundary(extra):
     _roundtrip_small(wl, idx, w, x, cpu_sync=False)
 
 
+@pytest.mark.parametrize("kw", [
+    dict(tokens_per_rank=64, ranks=8, experts=2048, topk=8, alignment=1, hidden=64),   # E at the fused limit
+    dict(tokens_per_rank=64, ranks=8, experts=4096, topk=8, alignment=1, hidden=64),   # beyond it: three kernels
+    dict(tokens_per_rank=256, ranks=8, experts=1024, topk=4, alignment=2, hidden=64),  # C * E = 65536: fused
+    dict(tokens_per_rank=260, ranks=8, experts=1024, topk=4, alignment=2, hidden=64),  # C * E = 66560: three kernels
+])
+def test_fused_layout_expert_limits(kw):
+    """The one-launch layout also stops at E = 2048 and at C * E = 65536 chunk counts (what every
+    CTA sums); both sides of each limit, every byte."""
+    wl = W.WORKLOADS["tiny"].with_(**kw)
+    idx, w, x = inputs(wl, 0.1)
+    _roundtrip_small(wl, idx, w, x, weighted=True)
+
+
 def test_duplicate_experts_in_one_token():
     wl = W.WORKLOADS["tiny"].with_(topk=4)
     idx, w, x = inputs(wl)
