@@ -617,10 +617,10 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) k_layout_fused(LayoutLaunch
 
 size_t fused_layout_smem(int E, int R) { return sizeof(int32_t) * ((size_t)(kLayoutWarps + 7) * E + 1 + R); }
 
-// At most one chunk per SM (so every CTA can be resident), the chunk's pairs in the warps'
-// registers, and bounded redundant summing.
-bool layout_fits_fused(int num_chunks, int chunk, int k, int E, int device) {
-  return num_chunks >= 1 && num_chunks <= sm_count(device) && E <= kFusedMaxExperts &&
+// At most one chunk per SM of the budget (so every CTA can be resident), the chunk's pairs in
+// the warps' registers, and bounded redundant summing.
+bool layout_fits_fused(int num_chunks, int chunk, int k, int E, int sm_budget) {
+  return num_chunks >= 1 && num_chunks <= sm_budget && E <= kFusedMaxExperts &&
          (int64_t)chunk * k <= (int64_t)kLayoutThreads * kFusedRounds && (int64_t)num_chunks * E <= kFusedMaxChunkCounts;
 }
 

@@ -203,12 +203,20 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
     return MOE_ERR_CUDA;
   }
   const int64_t T = p->num_tokens, k = p->topk, E = p->num_experts, R = p->num_logical_ranks;
-  // Chunks of the count / assign kernels: halve from kChunkTokens down to 32 tokens while the
-  // batch gives fewer than two chunks per SM, so small batches still spread over many CTAs
+  // Chunks.  The one-launch layout takes the smallest chunk of 32..256 tokens that leaves at most
+  // one chunk per SM the layout may use, if its other limits hold (layout_fits_fused).
+  // Otherwise the count / assign kernels halve the chunk from kChunkTokens down to 32 tokens
+  // while the batch gives fewer than two chunks per SM, so it still spreads over many CTAs
   // (a warp's run of pairs, chunk * k / 8, sets the assign kernel's serial work).
-  const int64_t want_chunks = 2 * (int64_t)sm_count(h->device);
-  int chunk = kChunkTokens;
-  while (chunk > 32 && (T + chunk - 1) / chunk < want_chunks) chunk /= 2;
+  const int sm_budget = grid_for(p->num_sms, h->device);
+  int chunk = 32;
+  while ((T + chunk - 1) / chunk > sm_budget && chunk < kChunkTokens) chunk *= 2;
+  const bool fused = layout_fits_fused((int)((T + chunk - 1) / chunk), chunk, (int)k, (int)E, sm_budget);
+  if (!fused) {
+    const int64_t want_chunks = 2 * (int64_t)sm_count(h->device);
+    chunk = kChunkTokens;
+    while (chunk > 32 && (T + chunk - 1) / chunk < want_chunks) chunk /= 2;
+  }
   h->num_chunks = (int)((T + chunk - 1) / chunk);
   const int64_t C = h->num_chunks;
 
@@ -282,7 +290,7 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   // at most a chunk per SM; with do_cpu_sync one host wait at the end.  (Small batches take
   // 32-token chunks over many CTAs: faster than one CTA whose warps each walk hundreds of pairs.)
   cudaError_t err = cudaMemsetAsync(d.status, 0, (size_t)(32 + 4 * R), s);
-  if (layout_fits_fused(L.num_chunks, L.chunk, L.k, L.E, h->device)) {
+  if (fused) {
     if (err == cudaSuccess) err = launch_layout_fused(L, p->recv_capacity_rows, s);
   } else {
     if (err == cudaSuccess) err = launch_layout_count(L, s);

@@ -26,7 +26,7 @@ constexpr bool kDebugChecks = false;
 // layout CTA.
 constexpr int kFusedMaxExperts = 2048;      // fused layout: 15 shared arrays of E counts
 constexpr int kFusedMaxChunkCounts = 65536; // fused layout: C * E counts every CTA sums
-constexpr int kFusedRounds = 4;             // fused layout: rounds of 32 pairs a warp holds in registers
+constexpr int kFusedRounds = 8;             // fused layout: rounds of 32 pairs a warp holds in registers
 constexpr int kFusedLoads = 32;             // fused layout: chunk counts a thread loads at once
 constexpr int kChunkTokens = 256;      // largest chunk: one token per thread of the count kernel
 constexpr int kLayoutThreads = 256;
@@ -111,7 +111,7 @@ cudaError_t launch_layout_assign(const LayoutLaunch& L, cudaStream_t s);
 cudaError_t launch_layout_small(const LayoutLaunch& L, int64_t cap_check, cudaStream_t s);
 cudaError_t launch_layout_fused(const LayoutLaunch& L, int64_t cap_check, cudaStream_t s);
 bool layout_fits_one_cta(int64_t T, int k, int E);
-bool layout_fits_fused(int num_chunks, int chunk, int k, int E, int device);
+bool layout_fits_fused(int num_chunks, int chunk, int k, int E, int sm_budget);
 
 struct DispatchLaunch {
   const void* x;

@@ -62,8 +62,9 @@ def _round_trip(wl, mask=0.1, with_bias=True, via_moe_dispatch=False):
 
 @pytest.mark.parametrize("fp8", [False, True])
 @pytest.mark.parametrize("kw", [
-    dict(tokens_per_rank=100, ranks=4, experts=16, topk=4),          # fused layout (13 chunks)
-    dict(tokens_per_rank=600, ranks=8, experts=64, topk=6),          # three-kernel layout (150 chunks)
+    dict(tokens_per_rank=100, ranks=4, experts=16, topk=4),          # fused layout (13 chunks of 32)
+    dict(tokens_per_rank=5000, ranks=8, experts=64, topk=4),         # three-kernel layout (157 chunks of 256)
+    dict(tokens_per_rank=600, ranks=8, experts=64, topk=6),          # fused layout (75 chunks of 64)
     dict(tokens_per_rank=40, ranks=64, experts=128, topk=8),         # 64 ranks
     dict(tokens_per_rank=200, ranks=2, experts=8, topk=2, alignment=1),
 ])

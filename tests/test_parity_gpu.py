@@ -112,7 +112,7 @@ def test_small_fp8_roundtrip(hidden, zero_padding):
     dict(tokens_per_rank=1024, ranks=1, experts=8, topk=8),   # 8192 pairs, 32 chunks (fused layout)
     dict(tokens_per_rank=1025, ranks=1, experts=8, topk=8),   # a one-token last chunk
     dict(experts=128, ranks=128, topk=4, tokens_per_rank=2),  # more than 64 ranks (membership)
-    dict(experts=128, ranks=128, topk=4, tokens_per_rank=70), # ... with 280 chunks (three-kernel layout)
+    dict(experts=128, ranks=128, topk=4, tokens_per_rank=70), # ... 8960 tokens: 70 chunks of 128 (fused)
     dict(hidden=4104, tokens_per_rank=200, experts=16, ranks=2, topk=3),   # ragged last chunk
 ])
 def test_shapes_and_edges(kw):
@@ -123,14 +123,24 @@ def test_shapes_and_edges(kw):
 
 @pytest.mark.parametrize("extra", [0, 1])
 def test_fused_and_three_kernel_layouts_at_the_boundary(extra):
-    """The handle's layout runs as one cooperative kernel while the batch has at most one 32-token
-    chunk per SM, else as count -> scan -> assign: both sides of that boundary, every byte."""
+    """The handle's layout runs as one cooperative kernel while some chunk of 32..256 tokens gives
+    at most one chunk per SM, else as count -> scan -> assign: both sides of that boundary (256
+    tokens per SM), every byte."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    wl = W.WORKLOADS["tiny"].with_(tokens_per_rank=16 * sms + extra, ranks=2, experts=16, topk=4)
-    assert -(-wl.tokens // 32) == sms + extra
+    wl = W.WORKLOADS["tiny"].with_(tokens_per_rank=128 * sms + extra, ranks=2, experts=16, topk=4, hidden=64)
+    assert -(-wl.tokens // 256) == sms + extra
     idx, w, x = inputs(wl, 0.1)
     _roundtrip_small(wl, idx, w, x, weighted=True, with_bias=True)
     _roundtrip_small(wl, idx, w, x, cpu_sync=False)
+
+
+def test_fused_layout_respects_the_sm_budget():
+    """With num_sms = 24 a 32-chunk batch may not take the one-launch layout (it needs a CTA per
+    chunk resident at once); the results are the same either way."""
+    wl = W.WORKLOADS["tiny"].with_(tokens_per_rank=512, ranks=2, experts=16, topk=4, hidden=64)
+    idx, w, x = inputs(wl, 0.1)
+    _roundtrip_small(wl, idx, w, x, weighted=True, num_sms=24)
+    _roundtrip_small(wl, idx, w, x, weighted=True, num_sms=32)
 
 
 @pytest.mark.parametrize("kw", [
