@@ -324,6 +324,27 @@ __device__ __forceinline__ void block_psum(const LayoutLaunch& L, const int32_t*
   __syncthreads();
 }
 
+// With do_cpu_sync: hand the status flags and the per-rank counts to the host as soon as they
+// are final (after psum), through mapped pinned memory, so the host's wait overlaps the rest of
+// the layout.  Words: [0] status flags, [7] ready = 1 (written last, after system-scope fences),
+// [8, 8 + R) tokens_per_rank, [8 + R, 8 + 2R) rows_per_rank.  Called by every thread of the CTA
+// that published psum / rows_per_rank, after block_psum.
+__device__ __forceinline__ void publish_host_counts(const LayoutLaunch& L) {
+  int32_t* hc = L.d.host_counts;
+  if (hc == nullptr) return;
+  for (int r = threadIdx.x; r < L.R; r += blockDim.x) {
+    hc[8 + r] = __ldcg(L.d.tokens_per_rank + r);
+    hc[8 + L.R + r] = __ldcg(L.d.rows_per_rank + r);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    hc[0] = atomicOr(L.d.status, 0);
+    __threadfence_system();
+    *reinterpret_cast<volatile int32_t*>(hc + 7) = 1;
+    __threadfence_system();
+  }
+}
+
 // ------------------------------------------------------------------------------------ count
 // A thread per token: its k ids are loaded together, counted into the chunk's shared-memory
 // histogram (atomicAdd_block), and its rank membership is written and counted.
@@ -419,6 +440,7 @@ __global__ void __launch_bounds__(kScanThreads) k_layout_scan(LayoutLaunch L, in
   __threadfence();
   if (tid == 0) *L.d.ticket = 0;  // ready for the next layout on this scratch
   block_psum<true>(L, L.d.cnt, cap_check, sm, sm + E, sm + 2 * E, nullptr, nullptr);
+  publish_host_counts(L);
 }
 
 // ------------------------------------------------------------------------------------ assign
@@ -589,6 +611,7 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) k_layout_fused(LayoutLaunch
     }
   __syncthreads();
   block_psum<false>(L, hist, cap_check, al, pad, gincl, pad_s, psum_s, c == 0);
+  if (c == 0) publish_host_counts(L);
 
   // 3. assign: warp bases (exclusive over warps, from the expert's segment start and the chunk's
   // offset), then the warp's pairs from registers

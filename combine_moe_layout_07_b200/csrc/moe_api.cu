@@ -7,6 +7,7 @@
 // dispatch-combine" (phantomic12.github.io): with it, the counts are copied to the host and
 // the call waits; without it, nothing waits and consumers read the device-side psum.
 #include <atomic>
+#include <chrono>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -119,6 +120,35 @@ static void pinned_give(void* p, size_t n) {
   g_pin_free.emplace_back(n, p);
 }
 
+// Mapped pinned blocks through which the layout kernels hand the counts to a waiting host
+// (do_cpu_sync); a handle holds one until it is freed.
+static std::mutex g_map_mu;
+static std::vector<std::pair<size_t, int32_t*>> g_map_free;
+
+static int32_t* mapped_take(size_t need, size_t* got) {
+  need = (need + 4095) / 4096 * 4096;
+  {
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    for (size_t i = 0; i < g_map_free.size(); ++i)
+      if (g_map_free[i].first >= need) {
+        int32_t* p = g_map_free[i].second;
+        *got = g_map_free[i].first;
+        g_map_free.erase(g_map_free.begin() + (long)i);
+        return p;
+      }
+  }
+  void* p = nullptr;
+  if (cudaHostAlloc(&p, need, cudaHostAllocMapped | cudaHostAllocPortable) != cudaSuccess) return nullptr;
+  *got = need;
+  return static_cast<int32_t*>(p);
+}
+
+static void mapped_give(int32_t* p, size_t n) {
+  if (!p) return;
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  g_map_free.emplace_back(n, p);
+}
+
 // The do_cpu_sync copy: the handle keeps [status 4, ticket, pad 3][tokens_per_rank R]
 // [rows_per_rank R] adjacent, so one copy brings flags and counts to the host.
 static size_t count_stage_bytes(int64_t R) { return sizeof(int32_t) * (size_t)(8 + 2 * R); }
@@ -166,7 +196,24 @@ static void release(moe_handle_t* h) {
   if (h->block) cudaFreeAsync(h->block, h->stream);
   if (h->epi_event) cudaEventDestroy(h->epi_event);
   pinned_give(h->epi_stage, h->epi_bytes);
+  mapped_give(h->host_block, h->host_block_bytes);
   delete h;
+}
+
+// Host side of publish_host_counts: spin until the layout marks the counts ready.  Bounded: a
+// stream error, a stream that finished without publishing, or 10 s return false.
+static bool wait_host_counts(const moe_handle_t* h, cudaStream_t s) {
+  volatile int32_t* ready = h->host_block + 7;
+  const auto t0 = std::chrono::steady_clock::now();
+  for (uint32_t n = 1; *ready == 0; ++n) {
+    if ((n & 1023) != 0) continue;
+    const cudaError_t q = cudaStreamQuery(s);
+    if (q == cudaSuccess) return *ready != 0;
+    if (q != cudaErrorNotReady) return false;
+    if (std::chrono::steady_clock::now() - t0 > std::chrono::seconds(10)) return false;
+  }
+  std::atomic_thread_fence(std::memory_order_acquire);
+  return true;
 }
 
 }  // namespace moe
@@ -269,6 +316,20 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
     d.tslot = reinterpret_cast<int32_t*>(b + o_tslot);
   }
 
+  // do_cpu_sync without deferral: the kernels publish the counts into a mapped pinned block
+  const bool publish = p->do_cpu_sync && !(p->flags & MOE_DEFER_EPILOGUE);
+  if (publish) {
+    h->host_block = mapped_take(count_stage_bytes(R), &h->host_block_bytes);
+    void* dev_view = nullptr;
+    if (!h->host_block || cudaHostGetDevicePointer(&dev_view, h->host_block, 0) != cudaSuccess) {
+      cudaGetLastError();
+      release(h);
+      return MOE_ERR_OOM;
+    }
+    reinterpret_cast<volatile int32_t*>(h->host_block)[7] = 0;
+    d.host_counts = static_cast<int32_t*>(dev_view);
+  }
+
   LayoutLaunch L{};
   L.idx = topk_idx;
   L.w = topk_weights;
@@ -317,20 +378,18 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
       return MOE_ERR_CUDA;
     }
     h->epi_pending = true;
-  } else if (p->do_cpu_sync) {
-    int32_t* stage = static_cast<int32_t*>(g_stage.get(count_stage_bytes(R)));
-    if (!stage) {
+  } else if (publish) {
+    // the host waits only for the counts; the rest of the layout runs on, stream-ordered
+    // before every later use of the handle
+    if (!wait_host_counts(h, s)) {
+      cudaStreamSynchronize(s);
+      cudaGetLastError();
       release(h);
       return MOE_ERR_CUDA;
     }
-    err = enqueue_count_copy(h, stage, s);
-    if (err == cudaSuccess) err = cudaStreamSynchronize(s);
-    if (err != cudaSuccess) {
-      release(h);
-      return MOE_ERR_CUDA;
-    }
-    rc = count_epilogue(h, stage, host_rows_per_rank);
+    rc = count_epilogue(h, h->host_block, host_rows_per_rank);
     if (rc != MOE_OK) {
+      cudaStreamSynchronize(s);  // the handle goes away: no kernel may still use its memory
       release(h);
       return rc;
     }
@@ -602,6 +661,7 @@ int moe_handle_free(moe_handle_t* h) {
   if (h->block && cudaFreeAsync(h->block, h->stream) != cudaSuccess) rc = MOE_ERR_CUDA;
   if (h->epi_event && cudaEventDestroy(h->epi_event) != cudaSuccess) rc = MOE_ERR_CUDA;
   pinned_give(h->epi_stage, h->epi_bytes);
+  mapped_give(h->host_block, h->host_block_bytes);  // written only before its ready flag, which the host saw
   delete h;
   return rc;
 }

@@ -61,6 +61,9 @@ struct DeviceArrays {
                                       //          first pair of the token on that rank, else -1
   int32_t* row_src = nullptr;         // [R * row_cap]
   float* row_w = nullptr;             // [R * row_cap]
+  int32_t* host_counts = nullptr;     // do_cpu_sync: mapped host memory [status, .., ready at 7]
+                                      // [tokens_per_rank R][rows_per_rank R], written once the
+                                      // counts are final (layout.cu, publish_host_counts)
 };
 
 }  // namespace moe
@@ -77,6 +80,8 @@ struct moe_handle {
   std::vector<int32_t> host_tokens;  // tokens_per_rank, when do_cpu_sync
   // MOE_DEFER_EPILOGUE: the count copy lands in epi_stage (pinned, owned until free) and
   // epi_event marks its completion; moe_handle_wait finishes the epilogue.
+  int32_t* host_block = nullptr;     // mapped pinned block behind d.host_counts (do_cpu_sync)
+  size_t host_block_bytes = 0;
   int32_t* epi_stage = nullptr;
   size_t epi_bytes = 0;
   cudaEvent_t epi_event = nullptr;
