@@ -111,7 +111,10 @@ int64_t moe_recv_capacity_hint(const moe_params_t* params, int64_t max_tokens_pe
  * tokens_per_rank[R], token_in_rank[T, R] (uint8), slot[T, k] (row inside its rank, -1 if
  * masked), row_src[R, row_cap] (source token, -1 for padding rows), row_w[R, row_cap].
  * With do_cpu_sync = 1 the call blocks until the counts reach the host and returns
- * MOE_ERR_BAD_EXPERT / MOE_ERR_CAPACITY directly (no handle is returned then).  With
+ * MOE_ERR_BAD_EXPERT / MOE_ERR_CAPACITY directly (no handle is returned then).  The counts are
+ * handed over as soon as they are final, through mapped pinned memory, so the call can return
+ * while the slot assignment still runs; it is stream-ordered before every later use of the
+ * handle.  With
  * MOE_DEFER_EPILOGUE as well it does not block: host_rows_per_rank is not written, the handle is
  * returned, and moe_handle_wait later delivers the counts and those two conditions.
  */
