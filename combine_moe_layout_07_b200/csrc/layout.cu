@@ -326,7 +326,7 @@ __device__ __forceinline__ void block_psum(const LayoutLaunch& L, const int32_t*
 
 // With do_cpu_sync: hand the status flags and the per-rank counts to the host as soon as they
 // are final (after psum), through mapped pinned memory, so the host's wait overlaps the rest of
-// the layout.  Words: [0] status flags, [7] ready = 1 (written last, after system-scope fences),
+// the layout.  Words: [0] status flags, [7] ready = 1 (written last, after a system-scope fence),
 // [8, 8 + R) tokens_per_rank, [8 + R, 8 + 2R) rows_per_rank.  Called by every thread of the CTA
 // that published psum / rows_per_rank, after block_psum.
 __device__ __forceinline__ void publish_host_counts(const LayoutLaunch& L) {
@@ -339,9 +339,8 @@ __device__ __forceinline__ void publish_host_counts(const LayoutLaunch& L) {
   __syncthreads();
   if (threadIdx.x == 0) {
     hc[0] = atomicOr(L.d.status, 0);
-    __threadfence_system();
+    __threadfence_system();  // the counts reach host memory before the flag
     *reinterpret_cast<volatile int32_t*>(hc + 7) = 1;
-    __threadfence_system();
   }
 }
 
