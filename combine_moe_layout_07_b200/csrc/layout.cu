@@ -497,11 +497,12 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L
 // CTA per chunk of 256 threads:
 //   1. count: each warp loads its contiguous run of the chunk's pairs into registers (at most
 //      kFusedRounds rounds of 32) and histograms it; token membership as k_layout_count; chunk
-//      counts to global memory; then the CTA arrives at a grid barrier (the ticket word, cleared
-//      before the launch) and waits, bounded, until every CTA has arrived;
-//   2. every CTA sums the chunk counts of all chunks itself: its chunk's offsets inside each
-//      expert (chunks before it) and the expert totals; then align / padding prefix / psum as
-//      the scan kernel's last CTA (CTA 0 alone publishes cnt, psum, pad_excl, rows_per_rank);
+//      counts to global memory and added atomically into the expert totals cnt; then the CTA
+//      arrives at a grid barrier (the ticket word; ticket and cnt cleared before the launch) and
+//      waits, bounded, until every CTA has arrived;
+//   2. every CTA reads the totals and sums the counts of the chunks before its own (its offsets
+//      inside each expert); then align / padding prefix / psum as the scan kernel's last CTA
+//      (CTA 0 alone publishes psum, pad_excl, rows_per_rank);
 //   3. assign: as k_layout_assign for its chunk (pairs from registers), based at those offsets;
 //      padding rows of the row maps over all CTAs' warps; by rank, the token rows based at the
 //      chunk's rank offsets.
@@ -570,6 +571,7 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) k_layout_fused(LayoutLaunch
     int32_t n = 0;
     for (int w = 0; w < kLayoutWarps; ++w) n += whist[w * E + e];
     L.d.chunk_cnt[(int64_t)c * E + e] = n;
+    if (n) atomicAdd(L.d.cnt + e, n);  // expert totals (cleared before the launch): order-free
   }
   for (int r = tid; r < R; r += blockDim.x) {
     if (tok[r]) atomicAdd(L.d.tokens_per_rank + r, tok[r]);  // integer sum: order-free
@@ -584,23 +586,21 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) k_layout_fused(LayoutLaunch
   __syncthreads();
   if (!go) return;
 
-  // 2. offsets and totals from every chunk's counts (kFusedLoads loads in flight), then psum
+  // 2. the expert totals, and the chunk's offsets from the counts of the chunks before it
+  // (kFusedLoads loads in flight); then psum.  CTA 0 needs no offsets, so the counts reach the
+  // host right after the barrier.
   for (int e = tid; e < E; e += blockDim.x) {
-    int32_t before = 0, total = 0;
-    for (int cb = 0; cb < C; cb += kFusedLoads) {
+    int32_t before = 0;
+    for (int cb = 0; cb < c; cb += kFusedLoads) {
       int32_t v[kFusedLoads];
 #pragma unroll
       for (int q = 0; q < kFusedLoads; ++q)
-        v[q] = cb + q < C ? __ldcg(L.d.chunk_cnt + (int64_t)(cb + q) * E + e) : 0;
+        v[q] = cb + q < c ? __ldcg(L.d.chunk_cnt + (int64_t)(cb + q) * E + e) : 0;
 #pragma unroll
-      for (int q = 0; q < kFusedLoads; ++q) {
-        before += cb + q < c ? v[q] : 0;
-        total += v[q];
-      }
+      for (int q = 0; q < kFusedLoads; ++q) before += v[q];
     }
     off[e] = before;
-    hist[e] = total;
-    if (c == 0) L.d.cnt[e] = total;
+    hist[e] = __ldcg(L.d.cnt + e);
   }
   if (L.by_rank)
     for (int r = tid; r < R; r += blockDim.x) {

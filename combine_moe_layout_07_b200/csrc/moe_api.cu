@@ -279,9 +279,10 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
     off = align_up64(off + bytes, 256);
     return at;
   };
-  // status[4], the scan ticket, tokens_per_rank[R] and rows_per_rank[R] are adjacent: one memset
-  // clears the first three (the kernels write every row count), one copy reads them all back
-  const int64_t o_status = take(32 + 8 * R), o_cnt = take(4 * E), o_psum = take(4 * E),
+  // status[4], the scan ticket, tokens_per_rank[R], rows_per_rank[R] and cnt[E] are adjacent: one
+  // memset clears them all (the one-launch layout sums cnt atomically), one copy reads the first
+  // four back
+  const int64_t o_status = take(32 + 8 * R + 4 * E), o_psum = take(4 * E),
                 o_pad = take(4 * (E + 1)), o_tir = take(T * R), o_slot = take(4 * T * k),
                 o_prank = take(4 * T * k), o_pw = take(4 * T * k), o_ccnt = take(4 * C * E),
                 o_rsrc = take(4 * R * h->row_cap), o_rw = take(4 * R * h->row_cap);
@@ -300,7 +301,7 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   d.ticket = d.status + 4;
   d.tokens_per_rank = d.status + 8;
   d.rows_per_rank = d.tokens_per_rank + R;
-  d.cnt = reinterpret_cast<int32_t*>(b + o_cnt);
+  d.cnt = d.rows_per_rank + R;
   d.psum = reinterpret_cast<int32_t*>(b + o_psum);
   d.pad_excl = reinterpret_cast<int32_t*>(b + o_pad);
   d.token_in_rank = reinterpret_cast<uint8_t*>(b + o_tir);
@@ -350,7 +351,7 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   // count -> scan -> assign back to back, or all three in one cooperative launch when there is
   // at most a chunk per SM; with do_cpu_sync one host wait at the end.  (Small batches take
   // 32-token chunks over many CTAs: faster than one CTA whose warps each walk hundreds of pairs.)
-  cudaError_t err = cudaMemsetAsync(d.status, 0, (size_t)(32 + 4 * R), s);
+  cudaError_t err = cudaMemsetAsync(d.status, 0, (size_t)(32 + 8 * R + 4 * E), s);
   if (fused) {
     if (err == cudaSuccess) err = launch_layout_fused(L, p->recv_capacity_rows, s);
   } else {
