@@ -590,6 +590,7 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) k_layout_fused(LayoutLaunch
   // (kFusedLoads loads in flight); then psum.  CTA 0 needs no offsets, so the counts reach the
   // host right after the barrier.
   for (int e = tid; e < E; e += blockDim.x) {
+    const int32_t total = __ldcg(L.d.cnt + e);  // issued first: in flight with the chunk loads
     int32_t before = 0;
     for (int cb = 0; cb < c; cb += kFusedLoads) {
       int32_t v[kFusedLoads];
@@ -600,7 +601,7 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) k_layout_fused(LayoutLaunch
       for (int q = 0; q < kFusedLoads; ++q) before += v[q];
     }
     off[e] = before;
-    hist[e] = __ldcg(L.d.cnt + e);
+    hist[e] = total;
   }
   if (L.by_rank)
     for (int r = tid; r < R; r += blockDim.x) {

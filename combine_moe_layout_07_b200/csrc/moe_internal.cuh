@@ -25,7 +25,7 @@ constexpr bool kDebugChecks = false;
 // Layout tiling: a chunk of tokens per CTA (a thread per token in the count kernel); 8 warps per
 // layout CTA.
 constexpr int kFusedMaxExperts = 2048;      // fused layout: 15 shared arrays of E counts
-constexpr int kFusedMaxChunkCounts = 65536; // fused layout: C * E counts every CTA sums
+constexpr int kFusedMaxChunkCounts = 65536; // fused layout: C * E chunk counts (the last CTA sums C - 1 of each E)
 constexpr int kFusedRounds = 8;             // fused layout: rounds of 32 pairs a warp holds in registers
 constexpr int kFusedLoads = 32;             // fused layout: chunk counts a thread loads at once
 constexpr int kChunkTokens = 256;      // largest chunk: one token per thread of the count kernel
