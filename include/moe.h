@@ -114,9 +114,9 @@ int64_t moe_recv_capacity_hint(const moe_params_t* params, int64_t max_tokens_pe
  * MOE_ERR_BAD_EXPERT / MOE_ERR_CAPACITY directly (no handle is returned then).  The counts are
  * handed over as soon as they are final, through mapped pinned memory, so the call can return
  * while the slot assignment still runs; it is stream-ordered before every later use of the
- * handle.  With
- * MOE_DEFER_EPILOGUE as well it does not block: host_rows_per_rank is not written, the handle is
- * returned, and moe_handle_wait later delivers the counts and those two conditions.
+ * handle.  With MOE_DEFER_EPILOGUE as well it does not block: host_rows_per_rank is not
+ * written, the handle is returned, and moe_handle_wait later delivers the counts and those two
+ * conditions.
  */
 int moe_layout(const moe_params_t* params, const int64_t* topk_idx, const float* topk_weights,
                void* stream, moe_handle_t** out_handle, int32_t* host_rows_per_rank);
