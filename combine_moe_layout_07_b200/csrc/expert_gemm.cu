@@ -15,18 +15,20 @@
 // The dispatch's 1x128 scales are fp32 (a / 448), not the power-of-two factors the block-scaled
 // MMA kinds take, so each 128-wide K-block is one plain E4M3 x E4M3 MMA group (4 x K=32) into a
 // fresh tensor-memory accumulator, and the epilogue warps promote it: acc += partial * (sx * sw)
-// in fp32 registers.  Four accumulator buffers in tensor memory let the MMAs run three K-blocks
-// ahead of the epilogue (one buffer's handoff round trip is longer than a K-block of MMAs).
+// in fp32 registers.  The 512 tensor-memory columns hold 512 / kN accumulator buffers (4 for
+// kN = 128, 2 for kN = 256), so the MMAs run up to that many K-blocks ahead of the epilogue.
 //
-// One CTA per SM, persistent over 128 x 128 output tiles in m-major order (consecutive tiles
-// share their 128 rows; an expert's weight columns are reused across its row tiles from L2).
-//   warp 0      TMA producer: per K-block, one 128x128-byte tile of rows and one of weights
-//               (128-byte swizzle) into a ring of stages (full/empty mbarriers);
+// One CTA per SM, persistent over 128 x kN output tiles (kN = 256 when N % 256 == 0, else 128)
+// in m-major order (consecutive tiles share their 128 rows; an expert's weight columns are
+// reused across its row tiles from L2).
+//   warp 0      TMA producer: per K-block, one 128 x 128-byte tile of rows and one kN x 128-byte
+//               tile of weights (128-byte swizzle) into a ring of stages (full/empty mbarriers);
 //   warp 1      allocates all 512 tensor-memory columns; one lane issues the MMAs and commits
 //               them to the stage's empty barrier and to the accumulator's full barrier;
 //   warps 2..9  epilogue: warp w reads tensor-memory lanes 32 * (w % 4) .. (one output row per
-//               thread) and half (w - 2) / 4 of the tile's 128 columns: per K-block two 32-column
-//               loads, one wait, 64 promotions; a bf16 store of its 64 columns per tile.
+//               thread) and half (w - 2) / 4 of the tile's kN columns (kN / 2 accumulators per
+//               thread): per K-block, 32-column loads in rounds of kRoundCols with one wait per
+//               round, then the promotions; a bf16 store of its kN / 2 columns per tile.
 // Every wait is an mbarrier wait bounded by wall-clock time (status kStatusTimeout).  No TMA
 // load here uses cluster multicast.
 #include <cuda.h>
