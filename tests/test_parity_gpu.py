@@ -150,8 +150,8 @@ def test_fused_layout_respects_the_sm_budget():
     dict(tokens_per_rank=260, ranks=8, experts=1024, topk=4, alignment=2, hidden=64),  # C * E = 66560: three kernels
 ])
 def test_fused_layout_expert_limits(kw):
-    """The one-launch layout also stops at E = 2048 and at C * E = 65536 chunk counts (what every
-    CTA sums); both sides of each limit, every byte."""
+    """The one-launch layout also stops at E = 2048 and at C * E = 65536 chunk counts (the last
+    CTA sums C - 1 of each expert's); both sides of each limit, every byte."""
     wl = W.WORKLOADS["tiny"].with_(**kw)
     idx, w, x = inputs(wl, 0.1)
     _roundtrip_small(wl, idx, w, x, weighted=True)
