@@ -184,8 +184,9 @@ def barrier():
 
 # --------------------------------------------------------------------------- CPU oracle sample
 def oracle_sample(wl: W.Workload, tokens: int):
-    """Run the CPU oracle (layout, dispatch, combine) on the first `tokens` tokens of the
-    workload's batch; returns (seconds, algorithmic bytes, description)."""
+    """Inputs for the CPU oracle (layout, dispatch, combine) on the first `tokens` tokens of the
+    workload's batch, generated once; returns run() -> (seconds, algorithmic bytes, description),
+    which times one oracle pass over them."""
     import oracle
     tpr = max(1, tokens // wl.ranks)
     sw = wl.with_(tokens_per_rank=tpr)
@@ -198,20 +199,32 @@ def oracle_sample(wl: W.Workload, tokens: int):
     cap = int(lay.rows_per_rank.max())
     y = W.gen_y(sw, cap).view(torch.int16).numpy().view(np.uint16)
     bias = W.gen_bias(sw).view(torch.int16).numpy().view(np.uint16) if sw.bias else None
-    t0 = time.perf_counter()
-    lay = oracle.layout(idx, w, E, R, A, cap=cap)
-    if sw.fp8:
-        oracle.dispatch_fp8(lay, idx, w, xb, E, R, A, cap, sw.zero_padding, want_w=False)
-    else:
-        oracle.dispatch_bf16(lay, idx, w, xb, E, R, A, cap, sw.zero_padding, want_w=False)
-    oracle.combine(idx, lay.slot, y, E, R, bias_bits=bias)
-    dt = time.perf_counter() - t0
-    valid = int(lay.cnt.sum())
-    pad = int(lay.rows_per_rank.sum()) - valid
-    b = algorithmic_bytes(sw, valid, pad)
     desc = (f"first {sw.tokens} tokens ({tpr}/rank) of the {wl.name} batch, same E/R/k/H/A; "
             f"layout+dispatch+combine by the single-threaded C oracle")
-    return dt, b["dispatch"] + b["combine"], desc
+
+    def run():
+        t0 = time.perf_counter()
+        lay = oracle.layout(idx, w, E, R, A, cap=cap)
+        if sw.fp8:
+            oracle.dispatch_fp8(lay, idx, w, xb, E, R, A, cap, sw.zero_padding, want_w=False)
+        else:
+            oracle.dispatch_bf16(lay, idx, w, xb, E, R, A, cap, sw.zero_padding, want_w=False)
+        oracle.combine(idx, lay.slot, y, E, R, bias_bits=bias)
+        dt = time.perf_counter() - t0
+        valid = int(lay.cnt.sum())
+        pad = int(lay.rows_per_rank.sum()) - valid
+        b = algorithmic_bytes(sw, valid, pad)
+        return dt, b["dispatch"] + b["combine"], desc
+
+    return run
+
+
+def reference_tokens(wl: W.Workload, steps: int, warmup: int) -> int:
+    """Tokens per step of the reference arm: 4096 for short runs, fewer for long ones, so that the
+    whole run stays near a minute of oracle time (about 0.5 s per 1000 DeepSeek-V3 tokens)."""
+    t = int(4096 * 30 / max(1, steps + warmup))
+    t = max(16 * wl.ranks, min(4096, t))
+    return t // wl.ranks * wl.ranks
 
 
 def workload_config(wl: W.Workload, cap: int, extra: dict | None = None) -> dict:
@@ -235,10 +248,11 @@ def run_reference(args) -> int:
     if rank != 0:
         return 0
     wl = W.WORKLOADS[args.workload]
-    tokens = args.ref_tokens
+    tokens = args.ref_tokens or reference_tokens(wl, args.steps, args.warmup)
+    run = oracle_sample(wl, tokens)
     times, nbytes, desc = [], 0, ""
     for i in range(args.warmup + args.steps):
-        dt, nbytes, desc = oracle_sample(wl, tokens)
+        dt, nbytes, desc = run()
         if i >= args.warmup:
             times.append(dt)
     mean = sum(times) / len(times)
@@ -568,7 +582,7 @@ def run_ours(args) -> int:
 
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        dt, cb, desc = oracle_sample(wl, args.cpu_tokens)
+        dt, cb, desc = oracle_sample(wl, args.cpu_tokens)()
         cpu = {"value": cb / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
 
     if rank == 0:
@@ -604,7 +618,8 @@ def main() -> int:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default="deepseek")
     ap.add_argument("--cpu-tokens", type=int, default=16384, help="tokens in the CPU-oracle baseline sample")
-    ap.add_argument("--ref-tokens", type=int, default=4096, help="tokens per step of the reference arm")
+    ap.add_argument("--ref-tokens", type=int, default=0,
+                    help="tokens per step of the reference arm (0: 4096, fewer for long runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--expert-gemm", type=int, default=0, metavar="N",
                     help="also time the first expert GEMM (E4M3, K = hidden, N output columns) on the dispatch output")
