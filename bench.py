@@ -69,7 +69,7 @@ KERNEL_SOURCES = {"combine": ("combine.cu", "moe_internal.cuh"), "dispatch": ("d
 def measured_traffic(kernel: str, workload: str):
     """dram read+write bytes per launch recorded from an ncu capture of the same kernel source;
     None if no record or if the kernel source changed since."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    path = os.path.join(ROOT, "profiles", "dram_traffic_dispatch_combine_deepseek_v3_prefill.md")
     if not os.path.exists(path):
         return None
     digest = kernel_source_digest(*KERNEL_SOURCES[kernel])
