@@ -582,6 +582,44 @@ def test_grouped_gemm_selects_each_rows_expert_and_block_scales():
         assert (out[r, :n][~seen[r, :n]] == 0).all()   # padding rows
 
 
+def test_grouped_gemm_random_weights_match_a_dense_blockwise_product():
+    """Random E4M3 weights and block scales against the same sum written as dense float64 matrix
+    products, one per 128-wide K-block: out[rows of e] = sum_b (sx[:, b] outer sw[e, n / 128, b])
+    * (deq(x[:, b]) @ deq(w[e, :, b])^T).  Square H = N, so a transposed weight operand stays in
+    bounds and fails here by value."""
+    wl, _, lay, codes, scales = _gemm_case(H=256, N=256)
+    E, R, A, H, N = wl.experts, wl.ranks, wl.alignment, wl.hidden, 256
+    KB = H // 128
+    rng = np.random.default_rng(17)
+    qw = rng.integers(0, 256, (E, N, H), dtype=np.uint8)
+    qw[(qw & 0x7F) == 0x7F] = 0x38                     # no NaN codes
+    sw = rng.uniform(0.25, 4.0, (E, N // 128, KB)).astype(np.float32)
+    st, out = oracle.grouped_gemm_f64(lay, codes, scales, qw, sw, E, R, A)
+    assert st == 0
+    table = _e4m3_table()
+    e_loc = E // R
+    checked = 0
+    for e in range(E):
+        r = e // e_loc
+        end = int(lay.psum[e]); beg = end - align_up(int(lay.cnt[e]), A)
+        if end == beg:
+            continue
+        X = table[codes[r, beg:end]]                   # [m, H]
+        Wd = table[qw[e]]                              # [N, H]
+        sx = scales[r, beg:end].astype(np.float64)     # [m, KB]
+        swn = np.repeat(sw[e].astype(np.float64), 128, axis=0)   # [N, KB]
+        ref = np.zeros((end - beg, N))
+        mag = np.zeros((end - beg, N))
+        for b in range(KB):
+            cols = slice(128 * b, 128 * b + 128)
+            f = np.outer(sx[:, b], swn[:, b])
+            ref += f * (X[:, cols] @ Wd[:, cols].T)
+            mag += np.abs(f) * (np.abs(X[:, cols]) @ np.abs(Wd[:, cols]).T)
+        assert (np.abs(out[r, beg:end] - ref) <= 1e-12 * mag + 1e-300).all(), e
+        checked += end - beg
+    assert checked > 0
+
+
 def test_grouped_gemm_is_linear_in_the_weight_scales():
     wl, _, lay, codes, scales = _gemm_case(H=256, N=128)
     E, R, A, H = wl.experts, wl.ranks, wl.alignment, wl.hidden

@@ -36,6 +36,11 @@ MUTATIONS = [
      "const float* ws = sw + ((int64_t)e * NB) * KB;"),
     ("expert GEMM drops the row scale", "acc += (double)xs[b] * (double)ws[b] * dot;",
      "acc += (double)ws[b] * dot;"),
+    ("expert GEMM reads the weights transposed",
+     "dot += oracle_e4m3_to_double(x[h]) * oracle_e4m3_to_double(wr[h]);",
+     "dot += oracle_e4m3_to_double(x[h]) * oracle_e4m3_to_double(qw[((int64_t)e * H + h) * N + n]);"),
+    ("expert GEMM drops the last K-block", "for (int64_t b = 0; b < KB; ++b) {\n                    double dot",
+     "for (int64_t b = 0; b + 1 < KB; ++b) {\n                    double dot"),
 ]
 
 
