@@ -371,6 +371,42 @@ def test_combine_fp32_within_tolerance_of_f64(weighted, with_bias):
         assert np.allclose(acc, ref[t], rtol=0, atol=1e-12)
 
 
+# bf16 bit patterns of the hand-worked order cases below
+_ONE, _2M8, _2M24 = 0x3F80, 0x3B80, 0x3380       # 1.0, 2^-8, 2^-24
+
+
+def _one_token(rows, bias=None, weighted=False, H=8):
+    """One token whose k = len(rows) pairs hit experts 0..k-1 of one rank, slot j holding rows[j]."""
+    k = len(rows)
+    idx = np.arange(k, dtype=np.int64)[None, :]
+    slot = np.arange(k, dtype=np.int32)[None, :]
+    y = np.repeat(np.array(rows, np.uint16)[None, :, None], H, axis=2)
+    w = np.ones((1, k), np.float32) if weighted else None
+    b = None if bias is None else np.full((1, H), bias, np.uint16)
+    st, out = oracle.combine(idx, slot, y, k, 1, w=w, bias_bits=b)
+    assert st == oracle.OK
+    return out[0]
+
+
+@pytest.mark.parametrize("weighted", [False, True])
+def test_combine_adds_the_rows_in_ascending_j(weighted):
+    """Rows 1, 2^-8, 2^-24, 2^-24 in that j order.  In fp32: 1 + 2^-8 is exact; each + 2^-24 is
+    half an ulp (2^-23) from an even value and rounds back to 1 + 2^-8; that is a bf16 tie,
+    which rounds to even: 1.0.  Summed in descending j the two 2^-24 first make 2^-23, the total
+    1 + 2^-8 + 2^-23 is exact and lies above the tie: bf16 1 + 2^-7 (0x3F81).  Unit weights
+    (fma(1, y, acc)) change nothing."""
+    assert (_one_token([_ONE, _2M8, _2M24, _2M24], weighted=weighted) == _ONE).all()
+    assert (_one_token([_2M24, _2M24, _2M8, _ONE], weighted=weighted) == 0x3F81).all()
+
+
+def test_combine_adds_the_bias_last():
+    """Rows 2^-24, 2^-24, 2^-8 and bias 1.0: the rows sum exactly to 2^-8 + 2^-23, then the bias
+    gives 1 + 2^-8 + 2^-23 exactly, above the bf16 tie: 0x3F81.  Had the bias come first, 1 +
+    2^-24 would round back to 1 twice and the result would be the tie 1 + 2^-8, rounded to 1.0."""
+    assert (_one_token([_2M24, _2M24, _2M8], bias=_ONE) == 0x3F81).all()
+    assert (_one_token([_ONE, _2M24, _2M24, _2M8]) == _ONE).all()   # the same values, bias-first order
+
+
 def test_bf16_rounding_definition():
     for v in [1.0, -2.5, 3.0e38, 1e-40, 0.1, 1.00390625, 1.01171875]:
         assert oracle.float_to_bf16(v) == bits(torch.tensor([v], dtype=torch.float32).to(torch.bfloat16))[0]

@@ -36,6 +36,14 @@ MUTATIONS = [
      "const float* ws = sw + ((int64_t)e * NB) * KB;"),
     ("expert GEMM drops the row scale", "acc += (double)xs[b] * (double)ws[b] * dot;",
      "acc += (double)ws[b] * dot;"),
+    ("combine sums in descending j",
+     "            float acc = 0.0f;\n            for (int j = 0; j < k; ++j) {\n                int32_t row = slot[t * k + j];\n"
+     "                if (row < 0) continue;\n                if (row >= cap) { status = ORC_ERR_CAPACITY; continue; }",
+     "            float acc = 0.0f;\n            for (int j = k - 1; j >= 0; --j) {\n                int32_t row = slot[t * k + j];\n"
+     "                if (row < 0) continue;\n                if (row >= cap) { status = ORC_ERR_CAPACITY; continue; }"),
+    ("combine adds the bias first",
+     '            float acc = 0.0f;\n            for (int j = 0; j < k; ++j) {\n                int32_t row = slot[t * k + j];\n                if (row < 0) continue;\n                if (row >= cap) { status = ORC_ERR_CAPACITY; continue; }\n                int r = (int)(idx[t * k + j] / E_loc);\n                float v = oracle_bf16_to_float(y[((int64_t)r * cap + row) * H + h]);\n                acc = w ? fmaf(w[t * k + j], v, acc) : acc + v;\n            }\n            if (bias) acc = acc + oracle_bf16_to_float(bias[t * H + h]);',
+     '            float acc = bias ? oracle_bf16_to_float(bias[t * H + h]) : 0.0f;\n            for (int j = 0; j < k; ++j) {\n                int32_t row = slot[t * k + j];\n                if (row < 0) continue;\n                if (row >= cap) { status = ORC_ERR_CAPACITY; continue; }\n                int r = (int)(idx[t * k + j] / E_loc);\n                float v = oracle_bf16_to_float(y[((int64_t)r * cap + row) * H + h]);\n                acc = w ? fmaf(w[t * k + j], v, acc) : acc + v;\n            }'),
     ("expert GEMM reads the weights transposed",
      "dot += oracle_e4m3_to_double(x[h]) * oracle_e4m3_to_double(wr[h]);",
      "dot += oracle_e4m3_to_double(x[h]) * oracle_e4m3_to_double(qw[((int64_t)e * H + h) * N + n]);"),
