@@ -9,6 +9,7 @@ import itertools
 import json
 import math
 import os
+import struct
 
 import numpy as np
 import pytest
@@ -232,6 +233,17 @@ def test_quantize_block_roundtrip_bound_and_max_code():
             assert codes[i] & 0x7F == 0x7E            # the block's largest element codes to 448
 
 
+def test_quantize_block_inv_is_one_ieee_division():
+    """Block [504, 9 * 2^-13, 0, ...]: a = 504, inv = fl(448 / 504) = fl(8 / 9), and
+    9 * 2^-13 * fl(8 / 9) rounds to exactly 2^-10, half the smallest E4M3 subnormal: a tie, to
+    even, code 0x00.  inv taken as 448 * fl(1 / 504) is one ulp larger and would give code 0x01.
+    The amax element codes to 448 (0x7E) and the scale is 504 / 448 = 1.125 exactly."""
+    xb = bits(torch.tensor([504.0, 9 * 2.0 ** -13] + [0.0] * 126).to(torch.bfloat16))
+    codes, scale = oracle.quantize_block(xb)
+    assert codes[0] == 0x7E and codes[1] == 0x00 and (codes[2:] == 0).all()
+    assert scale == 1.125
+
+
 def test_quantize_block_zero_and_floor():
     codes, s = oracle.quantize_block(np.zeros(128, np.uint16))
     assert (codes == 0).all() and s == np.float32(1e-4) / np.float32(448.0)
@@ -399,6 +411,34 @@ def test_combine_adds_the_rows_in_ascending_j(weighted):
     assert (_one_token([_2M24, _2M24, _2M8, _ONE], weighted=weighted) == 0x3F81).all()
 
 
+def test_combine_weighted_rows_use_one_fused_multiply_add():
+    """Rows 1.0 (w = 1) and y = 1.5 * 2^-8 with w = 11184982 * 2^-24: w * y is exactly
+    2^-8 + 2^-24 + 2^-32.  With fma(w, y, acc) the fp32 sum 1 + 2^-8 + 2^-24 + 2^-32 lies above
+    the tie at 2^-24 and rounds to 1 + 2^-8 + 2^-23, above the bf16 tie: 0x3F81.  Rounding the
+    product first gives 2^-8 + 2^-24 (a tie, to even), then the sum 1 + 2^-8 + 2^-24 rounds to
+    even, 1 + 2^-8, the bf16 tie, and the result would be 1.0."""
+    idx = np.arange(2, dtype=np.int64)[None, :]
+    slot = np.arange(2, dtype=np.int32)[None, :]
+    y = np.array([[[_ONE] * 8, [0x3BC0] * 8]], np.uint16)      # 1.0, 1.5 * 2^-8
+    w = np.array([[1.0, 11184982 * 2.0 ** -24]], np.float32)
+    assert float(w[0, 1]) == 11184982 * 2.0 ** -24               # exactly representable
+    st, out = oracle.combine(idx, slot, y, 2, 1, w=w)
+    assert st == oracle.OK and (out == 0x3F81).all()
+
+
+def test_combine_by_rank_adds_ranks_in_first_appearance_order():
+    """One token whose experts sit on ranks 3, 2, 1, 0 in j order, each rank's partial row being
+    1, 2^-8, 2^-24, 2^-24: in that order the sum rounds to bf16 1.0 (the ascending-j case above);
+    in ascending rank order it would be 1 + 2^-7."""
+    idx = np.array([[3, 2, 1, 0]], np.int64)
+    token_row = np.zeros((1, 4), np.int32)
+    y = np.zeros((4, 1, 8), np.uint16)
+    for r, v in zip((3, 2, 1, 0), (_ONE, _2M8, _2M24, _2M24)):
+        y[r, 0, :] = v
+    st, out = oracle.combine_by_rank(idx, token_row, y, 4, 4)
+    assert st == oracle.OK and (out == _ONE).all()
+
+
 def test_combine_adds_the_bias_last():
     """Rows 2^-24, 2^-24, 2^-8 and bias 1.0: the rows sum exactly to 2^-8 + 2^-23, then the bias
     gives 1 + 2^-8 + 2^-23 exactly, above the bf16 tie: 0x3F81.  Had the bias come first, 1 +
@@ -411,6 +451,10 @@ def test_bf16_rounding_definition():
     for v in [1.0, -2.5, 3.0e38, 1e-40, 0.1, 1.00390625, 1.01171875]:
         assert oracle.float_to_bf16(v) == bits(torch.tensor([v], dtype=torch.float32).to(torch.bfloat16))[0]
     assert oracle.float_to_bf16(float("nan")) == 0x7FC0
+    # any NaN, whatever its sign or payload, becomes the one canonical pattern
+    payload_nan = struct.unpack("<f", struct.pack("<I", 0x7FC12345))[0]
+    assert oracle.float_to_bf16(payload_nan) == 0x7FC0
+    assert oracle.float_to_bf16(-float("nan")) == 0x7FC0
     # ties: 1 + 2^-8 is halfway between 1 and 1 + 2^-7 -> even (1.0)
     assert oracle.float_to_bf16(1.00390625) == 0x3F80
 

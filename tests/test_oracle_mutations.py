@@ -29,6 +29,7 @@ MUTATIONS = [
      "                acc = acc + v;"),
     ("combine drops the bias", "            if (bias) acc = acc + oracle_bf16_to_float(bias[t * H + h]);\n            out[t * H + h] = oracle_float_to_bf16(acc);\n        }\n    return status;\n}\n\n/* The same sum",
      "            out[t * H + h] = oracle_float_to_bf16(acc);\n        }\n    return status;\n}\n\n/* The same sum"),
+    ("bf16 NaN keeps its sign and payload", "return 0x7FC0;", "return (uint16_t)(u >> 16);"),
     ("bf16 rounding truncates", "    if (lo > 0x8000u || (lo == 0x8000u && (hi & 1u))) hi += 1;", "    (void)lo;"),
     ("expert GEMM uses the next expert's weights", "const uint8_t* wr = qw + ((int64_t)e * N + n) * H;",
      "const uint8_t* wr = qw + ((int64_t)((e + 1) % E) * N + n) * H;"),
@@ -44,6 +45,15 @@ MUTATIONS = [
     ("combine adds the bias first",
      '            float acc = 0.0f;\n            for (int j = 0; j < k; ++j) {\n                int32_t row = slot[t * k + j];\n                if (row < 0) continue;\n                if (row >= cap) { status = ORC_ERR_CAPACITY; continue; }\n                int r = (int)(idx[t * k + j] / E_loc);\n                float v = oracle_bf16_to_float(y[((int64_t)r * cap + row) * H + h]);\n                acc = w ? fmaf(w[t * k + j], v, acc) : acc + v;\n            }\n            if (bias) acc = acc + oracle_bf16_to_float(bias[t * H + h]);',
      '            float acc = bias ? oracle_bf16_to_float(bias[t * H + h]) : 0.0f;\n            for (int j = 0; j < k; ++j) {\n                int32_t row = slot[t * k + j];\n                if (row < 0) continue;\n                if (row >= cap) { status = ORC_ERR_CAPACITY; continue; }\n                int r = (int)(idx[t * k + j] / E_loc);\n                float v = oracle_bf16_to_float(y[((int64_t)r * cap + row) * H + h]);\n                acc = w ? fmaf(w[t * k + j], v, acc) : acc + v;\n            }'),
+    ("FP8 inv by a reciprocal multiply", "float inv = 448.0f / a;", "float inv = 448.0f * (1.0f / a);"),
+    ("weighted combine rounds the product first", "acc = w ? fmaf(w[t * k + j], v, acc) : acc + v;",
+     "acc = w ? w[t * k + j] * v + acc : acc + v;"),
+    ("by-rank combine in ascending rank order",
+     "            for (int j = 0; j < k; ++j) {\n                int64_t e = idx[t * k + j];\n                if (e < 0 || e >= E) continue;\n"
+     "                int r = (int)(e / E_loc);\n                if (seen[r]) continue;\n                seen[r] = 1;",
+     "            for (int r = 0; r < R; ++r) {\n                int hit = 0;\n"
+     "                for (int j = 0; j < k; ++j) { int64_t e = idx[t * k + j]; if (e >= 0 && e < E && e / E_loc == r) hit = 1; }\n"
+     "                if (!hit) continue;\n                if (seen[r]) continue;\n                seen[r] = 1;"),
     ("expert GEMM reads the weights transposed",
      "dot += oracle_e4m3_to_double(x[h]) * oracle_e4m3_to_double(wr[h]);",
      "dot += oracle_e4m3_to_double(x[h]) * oracle_e4m3_to_double(qw[((int64_t)e * H + h) * N + n]);"),
