@@ -138,6 +138,15 @@ def test_layout_brute_force_tiny():
     assert n > 1000
 
 
+def test_layout_without_weights_gives_zero_row_weights():
+    """topk_weights may be NULL: every row weight then reads 0, routed rows and padding alike."""
+    wl = W.WORKLOADS["tiny"]
+    idx, _ = W.gen_routing(wl)
+    lay = oracle.layout(idx.numpy(), None, wl.experts, wl.ranks, wl.alignment)
+    for r in range(wl.ranks):
+        assert (lay.row_w[r, :int(lay.rows_per_rank[r])] == 0.0).all()
+
+
 def test_layout_errors():
     idx = np.array([[0, 1], [2, 7]], np.int64)
     assert oracle.layout(idx, None, 8, 2, 4).status == oracle.OK
@@ -439,6 +448,18 @@ def test_combine_by_rank_adds_ranks_in_first_appearance_order():
     assert st == oracle.OK and (out == _ONE).all()
 
 
+def test_combine_by_rank_adds_the_bias_last():
+    """By rank, partial rows 2^-24, 2^-24, 2^-8 (ranks 0, 1, 2 in j order) and bias 1.0 give
+    1 + 2^-8 + 2^-23 exactly, above the bf16 tie: 0x3F81; the bias first would give 1.0."""
+    idx = np.array([[0, 1, 2]], np.int64)
+    y = np.zeros((3, 1, 8), np.uint16)
+    for r, v in enumerate((_2M24, _2M24, _2M8)):
+        y[r, 0, :] = v
+    st, out = oracle.combine_by_rank(idx, np.zeros((1, 3), np.int32), y, 3, 3,
+                                     bias_bits=np.full((1, 8), _ONE, np.uint16))
+    assert st == oracle.OK and (out == 0x3F81).all()
+
+
 def test_combine_adds_the_bias_last():
     """Rows 2^-24, 2^-24, 2^-8 and bias 1.0: the rows sum exactly to 2^-8 + 2^-23, then the bias
     gives 1 + 2^-8 + 2^-23 exactly, above the bf16 tie: 0x3F81.  Had the bias come first, 1 +
@@ -478,6 +499,18 @@ def test_combine_backward_unweighted_is_the_bf16_dispatch_of_grad_out():
     st2, ref, _ = oracle.dispatch_bf16(lay, idx, w, g, E, R, A, cap, True)
     assert st == st2 == oracle.OK
     assert (gy == ref).all()
+
+
+def test_combine_backward_rounds_w_times_g_once_in_fp32():
+    """w = 11228502 * 2^-24 and g = 1.5: w * g is exactly 1 + 2^-8 + 2^-24, half an fp32 ulp
+    above 1 + 2^-8, so the fp32 product rounds to even, 1 + 2^-8, a bf16 tie that rounds to
+    even: 1.0 (0x3F80).  Rounding the exact product straight to bf16 would give 0x3F81."""
+    w = np.array([[11228502 * 2.0 ** -24]], np.float32)
+    assert float(w[0, 0]) == 11228502 * 2.0 ** -24
+    idx = np.array([[0]], np.int64)
+    lay = oracle.layout(idx, w, 1, 1, 1)
+    st, gy = oracle.combine_backward(lay, idx, np.full((1, 8), 0x3FC0, np.uint16), 1, 1, 1, 1, w=w)
+    assert st == oracle.OK and (gy[0, 0] == 0x3F80).all()
 
 
 def test_combine_backward_is_the_adjoint_of_combine():
