@@ -652,8 +652,8 @@ bool layout_fits_fused(int num_chunks, int chunk, int k, int E, int sm_budget) {
 // E <= kSmallMaxExperts): membership and id checks, per-warp histograms of token-aligned pair
 // ranges, cross-warp scan, psum, slots and row maps, all through shared memory, in one launch
 // and with no scratch beyond the handle's arrays.  The allocation-free entry point uses it; the
-// handle path runs count -> scan -> assign, which spreads a small batch over more SMs and is
-// faster.  The results are the same.
+// handle path runs the one-launch layout (or count -> scan -> assign), which spreads a small
+// batch over more SMs and is faster.  The results are the same.
 __global__ void __launch_bounds__(kSmallThreads) k_layout_small(LayoutLaunch L, int64_t cap_check) {
   extern __shared__ int32_t sm[];
   const int E = L.E, tid = threadIdx.x, warp = tid >> 5;
