@@ -621,6 +621,17 @@ def test_by_rank_dispatch_copies_and_topk_views():
     members = np.array([[tr[t, r] >= 0 for r in range(R)] for t in range(wl.tokens)]).sum(1)
     expect = bits((x.float() * torch.from_numpy(members).float()[:, None]).to(torch.bfloat16))
     assert (out == expect).all()
+    # FP8: each member row holds the token's 1x128 block codes and scales, at its own row
+    st, codes, scales, _, _ = oracle.dispatch_by_rank(idx, w, tr, xb, E, R, cap, fp8=True)
+    assert st == oracle.OK
+    for t in range(wl.tokens):
+        blocks = [oracle.quantize_block(xb[t, b:b + 128]) for b in range(0, wl.hidden, 128)]
+        want_c = np.concatenate([c for c, _ in blocks])
+        want_s = np.array([sc for _, sc in blocks], np.float32)
+        for r in range(R):
+            if tr[t, r] >= 0:
+                assert (codes[r, tr[t, r]] == want_c).all()
+                assert (scales[r, tr[t, r]].view(np.uint32) == want_s.view(np.uint32)).all()
 
 
 # ----------------------------------------------------------------------------- expert GEMM

@@ -59,6 +59,8 @@ MUTATIONS = [
      '            float acc = bias ? oracle_bf16_to_float(bias[t * H + h]) : 0.0f;\n            for (int j = 0; j < k; ++j) {\n                int64_t e = idx[t * k + j];\n                if (e < 0 || e >= E) continue;\n                int r = (int)(e / E_loc);\n                if (seen[r]) continue;\n                seen[r] = 1;\n                int32_t row = token_row[t * R + r];\n                if (row >= cap) { status = ORC_ERR_CAPACITY; continue; }\n                acc = acc + oracle_bf16_to_float(y[((int64_t)r * cap + row) * H + h]);\n            }'),
     ("row weights without topk_weights read 1", "row_w[(int64_t)r * cap + row] = w ? w[t * k + j] : 0.0f;",
      "row_w[(int64_t)r * cap + row] = w ? w[t * k + j] : 1.0f;"),
+    ("by-rank FP8 scales written at the row index", "                memcpy(recv_scales + g * nb, scales, sizeof(float) * (size_t)nb);",
+     "                memcpy(recv_scales + g, scales, sizeof(float) * (size_t)nb);"),
     ("expert GEMM reads the weights transposed",
      "dot += oracle_e4m3_to_double(x[h]) * oracle_e4m3_to_double(wr[h]);",
      "dot += oracle_e4m3_to_double(x[h]) * oracle_e4m3_to_double(qw[((int64_t)e * H + h) * N + n]);"),
