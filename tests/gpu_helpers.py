@@ -56,20 +56,3 @@ def compare_layout(h: moe.Handle, lay: oracle.Layout, wl: W.Workload):
         n = int(lay.rows_per_rank[r])
         assert (src[r, :n] == lay.row_src[r, :n]).all(), r
         assert (rw[r, :n].view(np.uint32) == lay.row_w[r, :n].view(np.uint32)).all(), r
-
-
-def pair_rows(lay: oracle.Layout, idx: np.ndarray, wl: W.Workload):
-    """(t, j, rank, slot) of every valid pair."""
-    t, j = np.nonzero(idx >= 0)
-    r = idx[t, j] // wl.experts_per_rank
-    return t, j, r, lay.slot[t, j]
-
-
-def padding_rows(lay: oracle.Layout, wl: W.Workload):
-    """(rank, row) of every padding row."""
-    out = []
-    for r in range(wl.ranks):
-        n = int(lay.rows_per_rank[r])
-        rows = np.nonzero(lay.row_src[r, :n] == -1)[0]
-        out.append(np.stack([np.full_like(rows, r), rows], 1))
-    return np.concatenate(out) if out else np.zeros((0, 2), np.int64)

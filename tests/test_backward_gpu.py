@@ -21,6 +21,10 @@ def _f32(b):
     return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
+def bf16_f32(b):
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
 def _grad_w_bound(H, g_rows, y_rows):
     return (8 * math.ceil(H / 256) + 6) * 2.0 ** -24 * np.abs(g_rows * y_rows).sum(axis=-1) + 1e-30
 
@@ -90,37 +94,42 @@ def test_combine_backward_small(weighted, zero_padding, hidden):
     assert moe.moe_handle_status(h) == moe.MOE_OK
 
 
-def test_combine_backward_full_size_sampled():
+def test_combine_backward_full_size():
+    """DeepSeek-V3 prefill, weighted: every element of grad_y (one logical rank at a time) bit-exact
+    against the oracle's backward over the whole batch, and every grad_w within its bound."""
     wl = W.WORKLOADS["deepseek"]
     idx, w, _ = inputs(wl)
     E, R, A, k, H = wl.experts, wl.ranks, wl.alignment, wl.topk, wl.hidden
-    lay = oracle.layout(idx.numpy(), w.numpy(), E, R, A)
-    cap = int(lay.rows_per_rank.max())
+    idx_n, w_n = idx.numpy(), w.numpy()
+    cap = int(oracle.layout(idx_n, w_n, E, R, A).rows_per_rank.max())
+    lay = oracle.layout(idx_n, w_n, E, R, A, cap=cap)
     h = gpu_layout(wl, idx, w, cap=0)
+    compare_layout(h, lay, wl)
     y = W.gen_y_device(wl, cap)
-    g = W.gen_bias(wl).cuda()
-    gy = torch.empty(R, cap, H, dtype=torch.bfloat16, device="cuda")
-    gw = torch.empty(wl.tokens, k, device="cuda")
-    moe.moe_combine_backward(h, g, gy, topk_weights=w.cuda(), y=y, grad_weights=gw, cap=cap)
+    g = W.gen_bias(wl)
+    gy = torch.full((R, cap, H), -23131, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+    gw = torch.full((wl.tokens, k), float("nan"), device="cuda")
+    moe.moe_combine_backward(h, g.cuda(), gy, topk_weights=w.cuda(), y=y, grad_weights=gw, cap=cap)
+    gb = bits(g)
+    st, ref = oracle.combine_backward(lay, idx_n, gb, E, R, A, cap, w=w_n, zero_padding=True)
+    assert st == oracle.OK
     torch.cuda.synchronize()
     assert moe.moe_handle_status(h) == moe.MOE_OK
-    rng = np.random.default_rng(4)
-    ts = np.unique(rng.integers(0, wl.tokens, 64))
-    n = len(ts)
-    # the sampled tokens as a problem of their own: expert j of token i is "expert" j on one rank
-    sub_idx = np.tile(np.arange(k, dtype=np.int64), (n, 1))
-    sub_lay = oracle.layout(sub_idx, w.numpy()[ts], E=k, R=1, A=1)
-    gs = bits(g[torch.from_numpy(ts).cuda()])
-    st, sub_gy = oracle.combine_backward(sub_lay, sub_idx, gs, k, 1, 1, n * k, w=w.numpy()[ts])
-    rr = torch.from_numpy(idx.numpy()[ts] // wl.experts_per_rank).cuda()
-    ss = torch.from_numpy(lay.slot[ts]).cuda()
-    got = bits(gy[rr, ss])                                  # [n, k, H]
-    for i in range(n):
-        for j in range(k):
-            assert (got[i, j] == sub_gy[0, sub_lay.slot[i, j]]).all()
-    ys = bits(y[rr, ss]).reshape(1, n * k, H)
-    sub_slot = (np.arange(n)[:, None] * k + np.arange(k)[None, :]).astype(np.int32)
-    ref_w = oracle.grad_weights_f64(sub_idx, sub_slot, gs, ys, k, 1)
-    got_w = gw[torch.from_numpy(ts).cuda()].cpu().numpy().astype(np.float64)
-    tol = _grad_w_bound(H, _f32(gs)[:, None, :], _f32(ys.reshape(n, k, H)))
-    assert (np.abs(got_w - ref_w) <= tol).all()
+    for r in range(R):
+        bad = bits(gy[r]) != ref[r]
+        assert not bad.any(), f"rank {r}: {bad.sum()} elements differ, first at (row, col) {np.argwhere(bad)[0]}"
+    del gy, ref
+    yb = bits(y)
+    del y
+    ref_w = oracle.grad_weights_f64(idx_n, lay.slot, gb, yb, E, R)
+    got_w = gw.cpu().numpy().astype(np.float64)
+    e_loc = wl.experts_per_rank
+    gf = bf16_f32(gb)
+    for t0 in range(0, wl.tokens, 1024):           # the bound needs sum |g * y| of every pair
+        t1 = min(wl.tokens, t0 + 1024)
+        rows = yb[idx_n[t0:t1] // e_loc, lay.slot[t0:t1]]            # [n, k, H]
+        # a bf16 x bf16 product is exact in binary32; the sum is taken in binary64
+        mag = np.abs(gf[t0:t1, None, :] * bf16_f32(rows)).sum(axis=-1, dtype=np.float64)
+        tol = (8 * math.ceil(H / 256) + 6) * 2.0 ** -24 * mag + 1e-30
+        bad = np.abs(got_w[t0:t1] - ref_w[t0:t1]) > tol
+        assert not bad.any(), f"grad_w outside the bound at {np.argwhere(bad)[0] + [t0, 0]}"

@@ -99,35 +99,47 @@ def test_by_rank_needs_at_most_64_ranks():
     assert e.value.status == moe.MOE_ERR_UNSUPPORTED
 
 
-def test_by_rank_full_size_sampled():
+def test_by_rank_full_size():
+    """DeepSeek-V3 prefill without expansion: token rows, every byte of the FP8 rows and scales, the
+    per-row top-k ids and weights (one logical rank at a time), and every combined token, against
+    the oracle over the whole batch."""
     wl = W.WORKLOADS["deepseek"]
     idx, w, x = inputs(wl)
     E, R, k, H = wl.experts, wl.ranks, wl.topk, wl.hidden
-    st, tr, rows = oracle.layout_by_rank(idx.numpy(), E, R)
+    idx_n, w_n = idx.numpy(), w.numpy()
+    st, tr, rows = oracle.layout_by_rank(idx_n, E, R)
+    assert st == oracle.OK
     cap = int(rows.max())
     h = gpu_layout(wl, idx, w, cap=0, by_rank=True)
     torch.cuda.synchronize()
     assert (h.token_rows().cpu().numpy() == tr).all()
+    assert (h.tokens_per_rank().cpu().numpy() == rows).all()
     recv = torch.full((R, cap, H), 0xA5, dtype=torch.uint8, device="cuda")
     sc = torch.full((R, cap, H // 128), float("nan"), device="cuda")
     ti = torch.full((R, cap, k), -7, dtype=torch.int32, device="cuda")
+    tw = torch.full((R, cap, k), float("nan"), device="cuda")
     moe.moe_dispatch_by_rank(h, x.cuda(), moe.MOE_DTYPE_FP8_E4M3, recv, sc, topk_idx=idx.cuda(), recv_topk_idx=ti,
-                             cap=cap)
+                             recv_topk_weights=tw, cap=cap)
+    st, r_recv, r_sc, r_ti, r_tw = oracle.dispatch_by_rank(idx_n, w_n, tr, bits(x), E, R, cap, True)
+    assert st == oracle.OK
     torch.cuda.synchronize()
-    rng = np.random.default_rng(6)
-    ts = np.unique(rng.integers(0, wl.tokens, 48))
-    xb = bits(x)
-    e_loc = wl.experts_per_rank
-    for t in ts:
-        blocks = [oracle.quantize_block(xb[t, b:b + 128]) for b in range(0, H, 128)]
-        codes = np.concatenate([c for c, _ in blocks])
-        scal = np.array([s for _, s in blocks], np.float32)
-        for r in range(R):
-            if tr[t, r] < 0:
-                continue
-            assert (recv[r, tr[t, r]].cpu().numpy() == codes).all()
-            assert (sc[r, tr[t, r]].cpu().numpy().view(np.uint32) == scal.view(np.uint32)).all()
-            got = ti[r, tr[t, r]].cpu().numpy()
-            exp = [int(e) - r * e_loc if e >= 0 and e // e_loc == r else -1 for e in idx[t].tolist()]
-            assert got.tolist() == exp
+    for r in range(R):
+        bad = recv[r].cpu().numpy() != r_recv[r]
+        assert not bad.any(), f"rank {r}: {bad.sum()} code bytes differ, first at (row, col) {np.argwhere(bad)[0]}"
+    assert (sc.cpu().numpy().view(np.uint32) == r_sc.view(np.uint32)).all()
+    assert (ti.cpu().numpy() == r_ti).all()
+    assert (tw.cpu().numpy().view(np.uint32) == r_tw.view(np.uint32)).all()
+    del recv, sc, ti, tw, r_recv, r_sc, r_ti, r_tw
+    # combine of per-rank partial sums, with the shared-expert bias
+    y = W.gen_y_device(wl, cap)
+    bias = W.gen_bias(wl)
+    out = torch.empty(wl.tokens, H, dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine_by_rank(h, y, out, bias=bias.cuda(), cap=cap)
+    yb = bits(y)
+    del y
+    st, ref = oracle.combine_by_rank(idx_n, tr, yb, E, R, bias_bits=bits(bias))
+    assert st == oracle.OK
+    got = bits(out)
+    assert (got == ref).all(), f"{(got != ref).sum()} elements differ"
     assert moe.moe_handle_status(h) == moe.MOE_OK
+    moe.moe_handle_free(h)
