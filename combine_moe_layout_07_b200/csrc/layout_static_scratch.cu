@@ -16,10 +16,17 @@
 //
 // Host code cannot use the array's name as a device address: the first call on each device,
 // with that device current, asks the runtime for the address (cudaGetSymbolAddress) and caches
-// it.  That first call should come before any stream capture.
+// it by device ordinal.  That first call should come before any stream capture.  The cache
+// assumes the runtime's primary context: after cudaDeviceReset, or from a context the caller
+// created through the driver API, the cached address is stale, and neither case is supported.
+//
+// Kernels: the one-CTA layout (k_layout_small) when T * k <= 8192 and E <= 1024, otherwise
+// count -> scan -> assign over 256-token chunks.  moe_layout picks its kernels by other rules
+// (the one-launch cooperative layout, adaptive chunks), but the layout is integer work with one
+// correct result, so the outputs are the same.
 //
 // Nothing here calls cudaMalloc, cudaMallocAsync, cudaMallocHost, cudaFree or any allocating
-// library routine; the layout kernels are the ones moe_layout launches.
+// library routine.
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -74,6 +81,8 @@ extern "C" int moe_layout_static_scratch(const moe_params_t* p, const int64_t* t
   if ((reinterpret_cast<uintptr_t>(topk_idx) & 7u) || (reinterpret_cast<uintptr_t>(topk_weights) & 3u) ||
       (reinterpret_cast<uintptr_t>(device_status) & 3u))
     return MOE_ERR_INVALID_ARG;
+  // without the host wait, device_status is the only place a bad id or an overflow can be read
+  if (!p->do_cpu_sync && !device_status) return MOE_ERR_INVALID_ARG;
 
   // scratch regions: status and scan ticket | pad prefix | chunk counts | pair rank | pair weight
   const int64_t C = (T + kChunkTokens - 1) / kChunkTokens;

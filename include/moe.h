@@ -301,16 +301,22 @@ const char* moe_status_string(int status);
  * the library holds until the process exits.  It needs
  *   256 + r(4(E+1)) + r(4*C*E) + 2*r(4*T*k) bytes, C = ceil(T/256), r = round up to 256;
  * larger problems return MOE_ERR_SCRATCH_LIMIT before any GPU work.
- *   device_status  int32, device, nullable: receives the device status flags of this call
- *                  (bit 0: an expert id outside [-1, E); bit 1: a rank needs more than cap rows);
- *                  cleared by the call.  NULL: the flags stay in the scratch array.
+ *   device_status  int32, device: receives the device status flags of this call (bit 0: an
+ *                  expert id outside [-1, E); bit 1: a rank needs more than cap rows); cleared by
+ *                  the call.  Required when do_cpu_sync = 0 (MOE_ERR_INVALID_ARG if NULL), since
+ *                  nothing else would report those conditions; may be NULL when do_cpu_sync = 1,
+ *                  where the call returns them.
  *   host_rows_per_rank  int32 [R], host, nullable: filled when do_cpu_sync = 1.
  * With do_cpu_sync = 1 the call waits for the counts and returns MOE_ERR_BAD_EXPERT /
  * MOE_ERR_CAPACITY directly; with 0 it returns after launching.
  * All calls share the scratch array and it keeps the last call's contents: calls whose GPU
  * work overlaps on the same device (two streams, two host threads) race.  The first call on a
- * device looks up the array's device address with that device current; make that first call
- * before any stream capture.  Calls no cudaMalloc, cudaFree or allocating library routine.
+ * device looks up the array's device address with that device current and caches it per
+ * device; make that first call before any stream capture.  The cache belongs to the runtime's
+ * primary context: calls after cudaDeviceReset, or under a context created through the driver
+ * API, are unsupported.  Kernels: one CTA when T*k <= 8192 and E <= 1024, else count, scan and
+ * assign over 256-token chunks; the results equal moe_layout's.  Calls no cudaMalloc, cudaFree
+ * or allocating library routine.
  */
 #define MOE_STATIC_SCRATCH_BYTES (4u << 20)
 int moe_layout_static_scratch(const moe_params_t* params, const int64_t* topk_idx,
