@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
         L.moe_recv_capacity_hint.restype = _I64
         L.moe_layout.argtypes = [PP, _P, _P, _P, ctypes.POINTER(_P), _P]
         L.moe_dispatch.argtypes = [_P, _P, _I32, _P, _P, _P, _I64, _I32, _I32, _I32, _P]
+        L.moe_layout_dispatch.argtypes = [PP, _P, _P, _P, _I32, _P, _P, _P, _I32, _P, ctypes.POINTER(_P)]
         L.moe_combine.argtypes = [_P, _P, _P, _P, _P, _I64, _I32, _P]
         L.moe_handle_status.argtypes = [_P, _P]
         L.moe_combine_backward.argtypes = [_P, _P, _P, _P, _I64, _I32, _P, _P, _I32, _P]
@@ -217,6 +218,20 @@ def moe_dispatch(handle: Handle, x: torch.Tensor, out_dtype: int, recv_x: torch.
     rc = lib().moe_dispatch(handle.ptr, _ptr(x), out_dtype, _ptr(recv_x), _ptr(recv_scales), _ptr(recv_weights),
                             cap, int(do_expand), int(do_zero_padding), num_sms, _stream(stream))
     _check(rc, "moe_dispatch")
+
+
+def moe_layout_dispatch(p: MoeParams, topk_idx: torch.Tensor, topk_weights: Optional[torch.Tensor], x: torch.Tensor,
+                        out_dtype: int, recv_x: torch.Tensor, recv_scales: Optional[torch.Tensor] = None,
+                        recv_weights: Optional[torch.Tensor] = None, do_zero_padding: bool = True,
+                        stream=None) -> Handle:
+    """Layout and expanded dispatch in one call (no host sync): the same results as moe_layout
+    followed by moe_dispatch with cap = p.recv_capacity_rows and num_sms = p.num_sms."""
+    h = ctypes.c_void_p()
+    rc = lib().moe_layout_dispatch(ctypes.byref(p), _ptr(topk_idx), _ptr(topk_weights), _ptr(x), out_dtype,
+                                   _ptr(recv_x), _ptr(recv_scales), _ptr(recv_weights), int(do_zero_padding),
+                                   _stream(stream), ctypes.byref(h))
+    _check(rc, "moe_layout_dispatch")
+    return Handle(h.value, p, None)
 
 
 def moe_combine(handle: Handle, y: torch.Tensor, out: torch.Tensor, topk_weights: Optional[torch.Tensor] = None,

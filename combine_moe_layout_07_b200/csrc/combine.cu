@@ -9,8 +9,11 @@
 // Numerics, fixed so every run is bit-identical: acc = 0 (fp32); for j = 0..k-1 in order,
 // skipping masked pairs, acc = fma(w, y, acc) or acc + y; then acc + bias; one rounding to bf16.
 //
-// B200 mapping (HBM-bound gather, one CTA per SM so num_sms caps SMs).  A work item is one token
-// and one column chunk of CW elements (CW <= 2048, chosen so that several stages fit):
+// B200 mapping (HBM-bound gather, one CTA per SM so num_sms caps SMs).  CTA b of G takes tokens
+// b, b + G, b + 2G, ..., so the grid reads neighbouring tokens together and the rows it gathers
+// from each expert's range lie close together (3-4 % faster at DeepSeek-V3 prefill than
+// contiguous token ranges per CTA).  A work item is one token and one column chunk of CW
+// elements (CW <= 2048, chosen so that several stages fit):
 //   warp 0      producer: reads the token's k (rank, slot) pairs from the handle and issues one
 //               cp.async.bulk load per valid source row segment (plus the bias segment) into a
 //               stage of a shared-memory ring, completed on the stage's mbarrier;
@@ -115,28 +118,28 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
   grid_dependents_launch();
   grid_dependency_wait();  // the expert outputs and the handle written by earlier kernels
 
-  int64_t t_begin, t_end;
-  cta_token_range(L.T, t_begin, t_end);
-  const int64_t n_items = (t_end - t_begin) * g.nch;
+  // CTA b of G takes tokens b, b + G, ... (token index q of this CTA is token b + q * G): the
+  // grid reads neighbouring tokens together, so the rows it gathers from each expert's range
+  // lie close together
+  const int64_t n_tok = cta_tokens(L.T);
+  const int64_t n_items = n_tok * g.nch;
   bool overflow = false;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     const int tpb = 32 / L.k, lanes_used = tpb * L.k;
-    const int64_t p_end = t_end * L.k;
     const uint32_t slot_bytes = (uint32_t)(g.cw * 2);
-    PairBatch cur = load_pair_batch(L.pair_rank, L.slot, kWeighted ? L.w : nullptr, t_begin * L.k, p_end, lane,
-                                    lanes_used);
+    PairBatch cur = load_cta_pairs(L.pair_rank, L.slot, kWeighted ? L.w : nullptr, 0, n_tok, L.k, lane, lanes_used);
     int64_t i = 0;
     int s = 0;
     uint32_t par = 0;  // parity of the stage's current use: (i / S) & 1
     bool stop = false;
-    for (int64_t tb = t_begin; tb < t_end && !stop; tb += tpb) {
-      const PairBatch nxt = load_pair_batch(L.pair_rank, L.slot, kWeighted ? L.w : nullptr, (tb + tpb) * L.k,
-                                            p_end, lane, lanes_used);
-      const int nt = (int)min((int64_t)tpb, t_end - tb);
+    for (int64_t qb = 0; qb < n_tok && !stop; qb += tpb) {
+      const PairBatch nxt =
+          load_cta_pairs(L.pair_rank, L.slot, kWeighted ? L.w : nullptr, qb + tpb, n_tok, L.k, lane, lanes_used);
+      const int nt = (int)min((int64_t)tpb, n_tok - qb);
       for (int q = 0; q < nt && !stop; ++q) {
-        const int64_t t = tb + q;
+        const int64_t t = cta_token(qb + q);
         int64_t src = -1;
         if (lane >= q * L.k && lane < (q + 1) * L.k && cur.rank >= 0 && cur.slot >= 0) {  // by-rank rows: -1 on repeats
           if (cur.slot < L.cap) src = ((int64_t)cur.rank * L.cap + cur.slot) * H;
@@ -197,11 +200,11 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
     const int grp = cwarp / kCombGroupWarps;
     const int gtid = tid - 32 - grp * kCombGroupThreads;
     const uint32_t slot_bytes = (uint32_t)(g.cw * 2);
-    // item i = (t - t_begin) * nch + chunk; this group takes i = grp, grp + G, ...
-    int64_t i = grp, t = t_begin, c = grp;
+    // item i = q * nch + chunk (q: the CTA's token index); this group takes i = grp, grp + G, ...
+    int64_t i = grp, q = 0, c = grp;
     while (c >= g.nch) {
       c -= g.nch;
-      ++t;
+      ++q;
     }
     int s = grp % S;
     uint32_t par = (uint32_t)((grp / S) & 1);
@@ -261,7 +264,8 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
             acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16hi(wb[q]));
           }
         }
-        if (!dbg_ok(t >= t_begin && t < t_end && c0 + e + 8 <= H && n <= L.k &&
+        const int64_t t = cta_token(q);
+        if (!dbg_ok(q < n_tok && t < L.T && c0 + e + 8 <= H && n <= L.k &&
                         g.data + (uint32_t)s * g.stage_bytes + (uint32_t)(n > 0 ? n - 1 : 0) * slot_bytes +
                                 (uint32_t)e * 2 + 16 <= g.total,
                     L.status, 103, t * 65536 + e))
@@ -279,7 +283,7 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
       c += kCombGroups;
       while (c >= g.nch) {
         c -= g.nch;
-        ++t;
+        ++q;
       }
       s += kCombGroups;
       while (s >= S) {

@@ -7,8 +7,11 @@
 // do_expand / do_zero_padding of "Why MoE gets stuck on communication" (locsic.com) section 1 and
 // FP8 dispatch of "DeepEP expert-parallel communication" (blog.hotdry.top), key techniques.
 //
-// B200 mapping (HBM-bound data movement, one CTA per SM so num_sms caps SMs).  Two kernels share
-// the producer (dispatch_producer) and the padding pass (zero_padding_rows):
+// B200 mapping (HBM-bound data movement, one CTA per SM so num_sms caps SMs).  CTA b of G takes
+// tokens b, b + G, b + 2G, ...: at any moment the grid works on neighbouring tokens, so the rows
+// it writes into each expert's range lie close together (consecutive tokens of an expert own
+// consecutive rows), and x is read front to back.  Two kernels share the producer
+// (dispatch_producer):
 //   k_dispatch_bulk   every dispatch except the weight-scaled rows of the combine backward.  A
 //                     storer warp writes each row to its destinations with cp.async.bulk stores
 //                     from shared memory (BF16: straight from the loaded stage; FP8: from an
@@ -22,10 +25,12 @@
 //                     registers, to each destination with 16-byte evict-first stores.
 //   FP8 (both): eight lanes own a 1x128 block, amax by three xor-shuffles, inv = 448/a and a/448
 //   as IEEE divisions, codes by cvt.rn.satfinite.e4m3x2.
-//   Padding rows are zeroed by the consumer warps after the tokens, a warp per row.
+//   Padding rows: k_dispatch_bulk's consumer groups zero one row of the CTA's share after each
+//   token they quantise (the rest after the tokens); k_dispatch zeroes them after the tokens, a
+//   warp per row.
 // Every wait is an mbarrier try_wait bounded by wall-clock time (status kStatusTimeout on
 // expiry); there are no named barriers.
-#include "moe_internal.cuh"
+#include "layout_body.cuh"
 
 namespace moe {
 
@@ -69,42 +74,42 @@ __host__ __device__ inline DispSmem disp_smem(int64_t H, int stages) {
   return s;
 }
 
+// Reads of the layout's arrays go through L2 (ld.global.cg): the one-launch layout + dispatch
+// kernel reads them in the same launch that wrote them, after its grid barrier.
 __device__ __forceinline__ int find_padding_expert(const int32_t* pad_excl, int E, int32_t i) {
   int lo = 0, hi = E;  // largest e with pad_excl[e] <= i
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (__ldg(pad_excl + mid) <= i) lo = mid;
+    if (__ldcg(pad_excl + mid) <= i) lo = mid;
     else hi = mid;
   }
   return lo;
 }
 
-// The producer warp of both dispatch kernels: pair metadata for tpb tokens per warp-wide load,
-// prefetched one batch ahead; per token, waits for its stage to be free, writes the destination
+// The producer warp of both dispatch kernels: pair metadata for tpb items per warp-wide load,
+// prefetched one batch ahead; per item, waits for its stage to be free, writes the destination
 // rows into the stage's DispMeta (and, by rank, the per-row top-k views) and issues one bulk load
-// of the bf16 row.  Stage s of token i is i % S, phase (i / S) & 1.
+// of the token's bf16 row.  Stage s of item i is i % S, phase (i / S) & 1.
 __device__ __forceinline__ void dispatch_producer(const DispatchLaunch& L, int S, uint32_t full0, uint32_t empty0,
-                                                  DispMeta* meta, uint32_t in_smem, int64_t t_begin,
-                                                  int64_t t_end, int lane, bool& overflow) {
+                                                  DispMeta* meta, uint32_t in_smem, int64_t n_items, int lane,
+                                                  bool& overflow) {
   const int64_t H = L.H;
   const uint32_t in_bytes = (uint32_t)(2 * H);
   const uint16_t* x = static_cast<const uint16_t*>(L.x);
   const int tpb = 32 / L.k, lanes_used = tpb * L.k;
-  const int64_t p_end = t_end * L.k;
   const float* wsrc = L.scale_w ? L.scale_w : L.pair_w;
   const bool views = L.recv_topk_idx || L.recv_topk_w;  // by-rank per-row top-k views
   const int64_t* ids = views ? L.topk_idx : nullptr;
-  PairBatch cur = load_pair_batch(L.pair_rank, L.slot, wsrc, t_begin * L.k, p_end, lane, lanes_used, ids);
+  PairBatch cur = load_cta_pairs(L.pair_rank, L.slot, wsrc, 0, n_items, L.k, lane, lanes_used, ids);
   int64_t i = 0;
   int s = 0;
   uint32_t par = 0;  // (i / S) & 1
   bool stop = false;
-  for (int64_t tb = t_begin; tb < t_end && !stop; tb += tpb) {
-    const PairBatch nxt =
-        load_pair_batch(L.pair_rank, L.slot, wsrc, (tb + tpb) * L.k, p_end, lane, lanes_used, ids);
-    const int nt = (int)min((int64_t)tpb, t_end - tb);
+  for (int64_t ib = 0; ib < n_items && !stop; ib += tpb) {
+    const PairBatch nxt = load_cta_pairs(L.pair_rank, L.slot, wsrc, ib + tpb, n_items, L.k, lane, lanes_used, ids);
+    const int nt = (int)min((int64_t)tpb, n_items - ib);
     for (int q = 0; q < nt; ++q) {
-      const int64_t t = tb + q;
+      const int64_t t = cta_token(ib + q);
       if (i >= S) {
         bool ok = true;
         if (lane == 0) ok = mbar_wait(empty0 + 8 * s, par ^ 1u, L.status);
@@ -198,6 +203,44 @@ __device__ __forceinline__ void zero_padding_rows(const DispatchLaunch& L, int64
   }
 }
 
+// An L2 policy that marks lines for eviction first: the receive rows are written once and read
+// only by a later kernel, so their lines go back to HBM soon after they are written, in about
+// the order the grid writes them.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ void bulk_store_hinted(void* dst, uint32_t src_smem, uint32_t bytes, uint64_t pol) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(dst),
+               "r"(src_smem), "r"(bytes), "l"(pol)
+               : "memory");
+}
+
+// Padding row i of all experts (0 <= i < pad_excl[E]), zeroed by the nth threads gtid of a
+// group: codes or bf16 row in 16-byte stores, FP8 scales, receive weight 0.  Returns false (and
+// writes nothing) when the row lies at or beyond cap.
+template <bool kFp8>
+__device__ __forceinline__ bool zero_padding_row(const DispatchLaunch& L, int32_t i, int gtid, int nth) {
+  const int64_t H = L.H, nblk = H / 128;
+  const int64_t row_bytes = kFp8 ? H : 2 * H;
+  const int e = find_padding_expert(L.pad_excl, L.E, i);
+  const int32_t pad_e = __ldcg(L.pad_excl + e + 1) - __ldcg(L.pad_excl + e);
+  const int32_t row = __ldcg(L.psum + e) - pad_e + (i - __ldcg(L.pad_excl + e));
+  if (row >= L.cap) return false;
+  const int64_t grow = (int64_t)(e / L.E_loc) * L.cap + row;
+  if (!dbg_ok(row >= 0 && grow < L.R * L.cap, L.status, 204, grow)) return true;
+  if (L.zero_padding) {
+    uint8_t* dst = static_cast<uint8_t*>(L.recv_x) + grow * row_bytes;
+    for (int64_t o = (int64_t)gtid * 16; o < row_bytes; o += (int64_t)nth * 16) st_stream_v4(dst + o, make_uint4(0, 0, 0, 0));
+    if (kFp8)
+      for (int64_t b = gtid; b < nblk; b += nth) L.recv_scales[grow * nblk + b] = 0.0f;
+  }
+  if (L.recv_w && gtid == 0) L.recv_w[grow] = 0.0f;
+  return true;
+}
+
 // FP8 E4M3 codes of the 16 bf16 values of unit u (bytes 32u .. 32u + 31) of a staged row.  Eight
 // consecutive lanes hold one 1x128 block: amax over the block by three xor-shuffles, a =
 // max(amax, 1e-4), inv = 448 / a and scale = a / 448 as IEEE divisions, codes =
@@ -258,13 +301,11 @@ __global__ void __launch_bounds__(kDispThreads, 1) k_dispatch(DispatchLaunch L, 
   grid_dependents_launch();
   grid_dependency_wait();  // the handle written by the layout kernels
 
-  int64_t t_begin, t_end;
-  cta_token_range(L.T, t_begin, t_end);
-  const int64_t n_items = t_end - t_begin;
+  const int64_t n_items = cta_tokens(L.T);
   bool overflow = false;
 
   if (warp == 0) {
-    dispatch_producer(L, S, full0, empty0, meta, base + lay.in, t_begin, t_end, lane, overflow);
+    dispatch_producer(L, S, full0, empty0, meta, base + lay.in, n_items, lane, overflow);
   } else {
     // ---------------------------------------------------------------- consumers
     const int ctid = tid - 32;
@@ -339,8 +380,10 @@ __global__ void __launch_bounds__(kDispThreads, 1) k_dispatch(DispatchLaunch L, 
 //               kBulkLag places back has been read and is handed back;
 //   warps 2..17 FP8: two consumer groups quantise alternate tokens from the input stage into an
 //               output stage (ring of O) and write the 1x128 scales with plain stores (a scale
-//               row of H / 128 floats need not be 16-byte aligned).  Then every warp zeroes
-//               padding rows; BF16 has nothing to compute, so its consumer warps start there.
+//               row of H / 128 floats need not be 16-byte aligned).  Each group also zeroes its
+//               part of the CTA's padding rows, spread evenly between its tokens; BF16 has
+//               nothing to compute, so its groups zero their padding rows from the start.
+// The row stores carry an L2 evict-first policy.
 // Barriers: full[S] (producer expect_tx, count 1); empty[S] (BF16: the storer; FP8: the group's
 // warps + the storer, which reads the stage's metadata); ofull[O] (the group's warps, after
 // fence.proxy.async so the bulk engine sees their shared-memory writes); oempty[O] (the storer).
@@ -406,16 +449,15 @@ __global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunc
   grid_dependents_launch();
   grid_dependency_wait();  // the handle written by the layout kernels
 
-  int64_t t_begin, t_end;
-  cta_token_range(L.T, t_begin, t_end);
-  const int64_t n_items = t_end - t_begin;
+  const int64_t n_items = cta_tokens(L.T);
   bool overflow = false;
 
   if (warp == 0) {
-    dispatch_producer(L, S, full0, empty0, meta, base + lay.in, t_begin, t_end, lane, overflow);
+    dispatch_producer(L, S, full0, empty0, meta, base + lay.in, n_items, lane, overflow);
   } else if (warp == 1) {
     // ---------------------------------------------------------------- storer
     uint8_t* recv = static_cast<uint8_t*>(L.recv_x);
+    const uint64_t pol = l2_evict_first_policy();
     int s = 0, o = 0;
     uint32_t par = 0, opar = 0;
     for (int64_t i = 0; i < n_items; ++i) {
@@ -431,7 +473,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunc
       }
       if (row >= 0 && dbg_ok(row < L.R * L.cap, L.status, 207, row)) {
         const uint32_t src = kFp8 ? base + lay.out + (uint32_t)o * row_bytes : base + lay.in + (uint32_t)s * in_bytes;
-        bulk_store(recv + row * row_bytes, src, row_bytes);
+        bulk_store_hinted(recv + row * row_bytes, src, row_bytes, pol);
         if (L.recv_w) L.recv_w[row] = w;
       }
       bulk_commit();
@@ -455,11 +497,20 @@ __global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunc
     bulk_wait_all();  // no store may still read shared memory when the CTA exits
   } else {
     const int ctid = tid - 64;
+    const int grp = (warp - 2) / kDispGroupWarps;
+    const int gtid = ctid - grp * kDispGroupThreads;
+    // the CTA's share [pb, pe) of the padding rows; group grp zeroes rows pb + grp, pb + grp + G, ..
+    // (G groups), paced over its tokens so that they go out among the token rows
+    const int32_t P = (L.zero_padding || L.recv_w) ? __ldg(L.pad_excl + L.E) : 0;
+    const int32_t pb = (int32_t)((int64_t)P * blockIdx.x / gridDim.x);
+    const int32_t pe = (int32_t)((int64_t)P * (blockIdx.x + 1) / gridDim.x);
+    int32_t pn = pb + grp;
     if constexpr (kFp8) {
       // ---------------------------------------------------------------- FP8 consumers
-      const int grp = (warp - 2) / kDispGroupWarps;
-      const int gtid = ctid - grp * kDispGroupThreads;
       const int64_t nblk = H / 128, nunits = H / 16;
+      const int64_t npad = pn < pe ? (pe - pn + kDispGroups - 1) / kDispGroups : 0;
+      const int64_t ntok = n_items > grp ? (n_items - grp + kDispGroups - 1) / kDispGroups : 0;
+      int64_t m = 0, pdone = 0;  // tokens and padding rows of this group so far
       int s = grp % S, o = grp % O;
       uint32_t par = (uint32_t)((grp / S) & 1), opar = (uint32_t)((grp / O) & 1);
       for (int64_t i = grp; i < n_items; i += kDispGroups) {
@@ -500,12 +551,260 @@ __global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunc
           o -= O;
           opar ^= 1u;
         }
+        for (const int64_t target = ++m * npad / ntok; pdone < target; ++pdone, pn += kDispGroups)
+          if (!zero_padding_row<kFp8>(L, pn, gtid, kDispGroupThreads)) overflow = true;
       }
     }
-    zero_padding_rows<kFp8>(L, blockIdx.x * kDispConsumerWarps + (ctid >> 5), gridDim.x * kDispConsumerWarps, lane,
-                            overflow);
+    // BF16 (nothing to compute per token): every padding row of the group from the start; FP8: the
+    // rows the pacing left
+    for (; pn < pe; pn += kDispGroups)
+      if (!zero_padding_row<kFp8>(L, pn, gtid, kDispGroupThreads)) overflow = true;
   }
   if (overflow) atomicOr(L.status, kStatusCapacity);
+}
+
+// ------------------------------------------------------------------------------------------------
+// One-launch layout + dispatch (moe_layout_dispatch without host sync, small batches): the
+// layout's notify work and the dispatch in one kernel, as the dispatch kernel of "From DeepEP to
+// Mega MoE" 2.2 runs notify warps beside its dispatch warps.  One cooperative launch of G CTAs
+// (every one resident), 576 threads each; CTA b owns items i < n_b (token b + i * G, a stage
+// each: n_b <= kLdMaxItems, no ring), and CTAs below C each own one layout chunk:
+//   warp 0       producer: at once, one bulk load of each item's bf16 row (x does not depend on
+//                the layout); after the second grid barrier (all C chunks assigned), the item's
+//                destination rows into its DispMeta, then an arrive on meta[i];
+//   warp 1       storer: per item, once its row (BF16: the input stage; FP8: the codes) and its
+//                metadata are ready, lanes 0..n-1 each issue one bulk store to a destination and
+//                write recv_w;
+//   warps 2..9   the layout of chunk b (layout_body.cuh, on named barrier 1), then an arrive on
+//                the second grid barrier; then, in every CTA, the CTA's share of padding rows
+//                once every chunk is assigned;
+//   warps 10..17 FP8: quantise each item into its output stage as soon as its row lands (while
+//                the layout runs), the 1x128 scales into shared memory; once the metadata is
+//                there, the scales to every destination.
+// The second grid barrier is the handle's status[5] (cleared with the status block before the
+// launch), raised by each layout chunk after a fence once its slots and row maps are written;
+// every wait is bounded by wall-clock time.  The layout's arrays written in this launch are read
+// through L2 (ld.global.cg).
+constexpr int kLdMaxItems = 8;     // items (tokens) per CTA
+constexpr int kLdThreads = 576;
+constexpr int kLdLayoutBar = 1;    // named barrier of the layout warps
+
+struct LdSmem {
+  uint32_t full, qdone, mready, meta, scales, layout, in, out, total;
+};
+
+__host__ __device__ inline LdSmem ld_smem(int64_t H, bool fp8, int n, int E, int R) {
+  LdSmem l;
+  uint32_t off = 0;
+  l.full = off;
+  off += 8 * n;
+  l.qdone = off;
+  off += 8 * n;
+  l.mready = off;
+  off += 8 * n;
+  off = round_to(off, 16);
+  l.meta = off;
+  off += (uint32_t)sizeof(DispMeta) * n;
+  l.scales = off;
+  off += fp8 ? (uint32_t)(4 * (H / 128) * n) : 0;
+  off = round_to(off, 16);
+  l.layout = off;
+  off += (uint32_t)fused_layout_smem(E, R);
+  off = round_to(off, 128);
+  l.in = off;
+  off += (uint32_t)(2 * H) * n;
+  l.out = off;
+  off += fp8 ? (uint32_t)H * n : 0;
+  l.total = off;
+  return l;
+}
+
+template <bool kFp8, int kRounds>
+__global__ void __launch_bounds__(kLdThreads, 1)
+    k_layout_dispatch(LayoutLaunch LL, int64_t cap_check, int C, DispatchLaunch L) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int32_t base_r[kMaxByRankRanks];
+  __shared__ int32_t go, go2;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t H = L.H, nblk = H / 128;
+  const int64_t n = cta_tokens(L.T);
+  const LdSmem lay = ld_smem(H, kFp8, kLdMaxItems, LL.E, LL.R);
+  const uint32_t base = smem_u32(smem);
+  const uint32_t full0 = base + lay.full, qdone0 = base + lay.qdone, mready0 = base + lay.mready;
+  DispMeta* meta = reinterpret_cast<DispMeta*>(smem + lay.meta);
+  float* scales_s = reinterpret_cast<float*>(smem + lay.scales);
+  const uint32_t in_bytes = (uint32_t)(2 * H);
+  const uint32_t row_bytes = kFp8 ? (uint32_t)H : in_bytes;
+  int32_t* done_ctr = LL.d.status + 5;
+
+  if (tid == 0) {
+    for (int i = 0; i < kLdMaxItems; ++i) {
+      mbar_init(full0 + 8 * i, 1);
+      mbar_init(qdone0 + 8 * i, kDispGroupWarps);
+      mbar_init(mready0 + 8 * i, 1);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  grid_dependents_launch();
+  bool overflow = false;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0)
+      for (int64_t i = 0; i < n; ++i) {
+        mbar_arrive_expect_tx(full0 + 8 * i, in_bytes);
+        if (dbg_ok(i < kLdMaxItems && cta_token(i) < L.T, L.status, 211, i))
+          bulk_load(base + lay.in + (uint32_t)i * in_bytes, static_cast<const uint16_t*>(L.x) + cta_token(i) * H,
+                    in_bytes, full0 + 8 * i);
+      }
+    bool ok = true;
+    if (lane == 0) ok = wait_count_reached(done_ctr, C, L.status);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    const int tpb = 32 / L.k, lanes_used = tpb * L.k;
+    for (int64_t ib = 0; ib < n; ib += tpb) {
+      PairBatch cur{-1, -1, 0.0f, -1};
+      const int q0 = lane / L.k;
+      if (ok && lane < lanes_used && ib + q0 < n) {  // the pairs of items ib .. ib + tpb - 1
+        const int64_t p = cta_token(ib + q0) * L.k + (lane - q0 * L.k);
+        cur.rank = __ldcg(L.pair_rank + p);
+        cur.slot = __ldcg(L.slot + p);
+        cur.w = __ldcg(L.pair_w + p);
+      }
+      const int nt = (int)min((int64_t)tpb, n - ib);
+      for (int q = 0; q < nt; ++q) {
+        const int64_t i = ib + q;
+        int64_t row = -1;
+        if (lane >= q * L.k && lane < (q + 1) * L.k && cur.rank >= 0 && cur.slot >= 0) {
+          if (cur.slot < L.cap) row = (int64_t)cur.rank * L.cap + cur.slot;
+          else overflow = true;
+        }
+        const uint32_t m = __ballot_sync(0xffffffffu, row >= 0);
+        if (row >= 0) {
+          const int pos = __popc(m & lanemask_lt());
+          meta[i].row[pos] = row;
+          meta[i].w[pos] = cur.w;
+        }
+        if (lane == 0) meta[i].n = __popc(m);  // 0 when the layout gave up: nothing is written
+        __syncwarp();
+        if (lane == 0) mbar_arrive(mready0 + 8 * i);
+      }
+    }
+    // no load of this CTA may still be in flight when it exits
+    if (lane == 0)
+      for (int64_t i = 0; i < n; ++i) mbar_wait(full0 + 8 * i, 0, L.status);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- storer
+    uint8_t* recv = static_cast<uint8_t*>(L.recv_x);
+    const uint64_t pol = l2_evict_first_policy();
+    for (int64_t i = 0; i < n; ++i) {
+      if (!mbar_wait_warp(kFp8 ? qdone0 + 8 * i : full0 + 8 * i, 0, L.status)) break;
+      if (!mbar_wait_warp(mready0 + 8 * i, 0, L.status)) break;
+      const int nd = meta[i].n;
+      if (!dbg_ok(nd >= 0 && nd <= L.k, L.status, 212, nd)) break;
+      const int64_t row = lane < nd ? meta[i].row[lane] : -1;
+      if (row >= 0 && dbg_ok(row < L.R * L.cap, L.status, 213, row)) {
+        const uint32_t src = kFp8 ? base + lay.out + (uint32_t)i * row_bytes : base + lay.in + (uint32_t)i * in_bytes;
+        bulk_store_hinted(recv + row * row_bytes, src, row_bytes, pol);
+        if (L.recv_w) L.recv_w[row] = meta[i].w[lane];
+      }
+      bulk_commit();
+    }
+    bulk_wait_all();  // no store may still read shared memory when the CTA exits
+  } else if (warp < 10) {
+    // ---------------------------------------------------------------- layout, then padding rows
+    const ThreadGroup g{tid - 64, kLayoutThreads, kLdLayoutBar};
+    bool ok = true;
+    if ((int)blockIdx.x < C) {
+      int32_t* lsm = reinterpret_cast<int32_t*>(smem + lay.layout);
+      ok = fused_layout_chunk<kRounds>(LL, cap_check, blockIdx.x, C, g, lsm, base_r, &go);
+      if (ok) {
+        __threadfence();  // the chunk's slots, pair data and row maps before the arrival
+        g.sync();
+        if (g.tid == 0) atomicAdd(done_ctr, 1);
+      }
+    }
+    const int32_t P = ok && (L.zero_padding || L.recv_w) ? 1 : 0;
+    if (P) {
+      if (g.tid == 0) go2 = wait_count_reached(done_ctr, C, L.status);
+      g.sync();
+      if (go2) {
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");
+        const int32_t total = __ldcg(L.pad_excl + L.E);
+        const int32_t pb = (int32_t)((int64_t)total * blockIdx.x / gridDim.x);
+        const int32_t pe = (int32_t)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
+        for (int32_t r = pb + (warp - 2); r < pe; r += kLayoutWarps)  // a warp per row
+          if (!zero_padding_row<kFp8>(L, r, lane, 32)) overflow = true;
+      }
+    }
+  } else if (kFp8) {
+    // ---------------------------------------------------------------- FP8 quantisers
+    const int gtid = tid - 320;
+    const int64_t nunits = H / 16;
+    for (int64_t i = 0; i < n; ++i) {
+      if (!mbar_wait_warp(full0 + 8 * i, 0, L.status)) break;
+      const uint32_t in_s = base + lay.in + (uint32_t)i * in_bytes;
+      const uint32_t out_s = base + lay.out + (uint32_t)i * row_bytes;
+      for (int64_t u = gtid; u - gtid < nunits; u += kDispGroupThreads) {
+        const bool act = u < nunits;
+        float scale;
+        const uint4 qv = quantize_unit(in_s, u, act, scale);
+        if (act) {
+          sts_v4(out_s + (uint32_t)u * 16, qv);
+          if ((gtid & 7) == 0) scales_s[i * nblk + u / 8] = scale;
+        }
+      }
+      fence_proxy_async_smem();  // the codes are read next by the bulk engine (async proxy)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qdone0 + 8 * i);
+    }
+    for (int64_t i = 0; i < n; ++i) {  // the scales, once the destinations are known
+      if (!mbar_wait_warp(qdone0 + 8 * i, 0, L.status)) break;  // every warp's scales are in
+      if (!mbar_wait_warp(mready0 + 8 * i, 0, L.status)) break;
+      const int nd = meta[i].n;
+      if (!dbg_ok(nd >= 0 && nd <= L.k, L.status, 214, nd)) break;
+      for (int64_t x = gtid; x < nd * nblk; x += kDispGroupThreads) {
+        const int j = (int)(x / nblk);
+        const int64_t b = x - j * nblk;
+        const int64_t row = meta[i].row[j];
+        if (dbg_ok(row >= 0 && row < L.R * L.cap, L.status, 215, row)) L.recv_scales[row * nblk + b] = scales_s[i * nblk + b];
+      }
+    }
+  }
+  if (overflow) atomicOr(L.status, kStatusCapacity);
+}
+
+// Whether a batch takes the one-launch layout + dispatch: at most kLdMaxItems tokens per CTA of
+// the grid, layout chunks whose pairs fit kFusedRounds rounds per warp, and shared memory (the
+// layout's arrays, a stage per item) that fits.
+bool layout_dispatch_fits(int64_t T, int64_t H, bool fp8, int E, int R, int grid, int chunk, int k) {
+  if (grid < 1 || (T + grid - 1) / grid > kLdMaxItems) return false;
+  if ((int64_t)chunk * k > (int64_t)kLayoutThreads * kFusedRounds) return false;
+  return ld_smem(H, fp8, kLdMaxItems, E, R).total <= 227u * 1024u - 1024u;
+}
+
+cudaError_t launch_layout_dispatch(const LayoutLaunch& LL, int64_t cap_check, const DispatchLaunch& L, bool fp8,
+                                   cudaStream_t st) {
+  const uint32_t smem = ld_smem(L.H, fp8, kLdMaxItems, LL.E, LL.R).total;
+  if ((int64_t)LL.chunk * LL.k > (int64_t)kLayoutThreads * kFusedRounds) return cudaErrorInvalidValue;
+  auto kern = fp8 ? k_layout_dispatch<true, kFusedRounds> : k_layout_dispatch<false, kFusedRounds>;
+  static unsigned long long done[2] = {0, 0};
+  cudaError_t err = set_smem_limit_once(kern, 227 * 1024 - 1024, &done[fp8 ? 1 : 0]);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(L.grid);
+  cfg.blockDim = dim3(kLdThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, kern, LL, cap_check, LL.num_chunks, L);
+  note_launch();
+  return err;
 }
 
 // The stage count is a multiple of the consumer-group count: stage s is then always consumed by

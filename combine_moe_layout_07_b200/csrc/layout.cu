@@ -16,111 +16,11 @@
 //   assign : per chunk, each warp takes a contiguous run of (t, j) pairs; per-warp histograms
 //            are scanned across warps, and inside a warp __match_any_sync + popc give each pair
 //            its rank among equal experts -- so rows keep ascending (t, j) order.
-#include "moe_internal.cuh"
+// Batches of at most one chunk per SM take the one-launch layout instead (k_layout_fused).  The
+// device code it shares with the one-launch layout + dispatch kernel lives in layout_body.cuh.
+#include "layout_body.cuh"
 
 namespace moe {
-
-__device__ __forceinline__ int32_t align_up_dev(int32_t n, int32_t a) { return ((n + a - 1) / a) * a; }
-
-// Expert id of a routing entry as int32: the id if in [0, E), -1 when masked, -2 when the
-// entry lies outside [-1, E) (an error the count kernel reports).
-__device__ __forceinline__ int32_t expert_of(int64_t e, int E) {
-  return (e >= 0 && e < E) ? (int32_t)e : (e == -1 ? -1 : -2);
-}
-
-// ------------------------------------------------------------------------------------ helpers
-// Membership of token t (when `valid`): writes token_in_rank[t, :] and counts the token for every
-// rank holding one of its experts into tok[r] (shared memory).  Called by whole warps: with R <= 64
-// the per-rank counts are aggregated over the warp (one ballot per rank, one atomic from lane 0),
-// which keeps shared-memory atomics off a handful of hot addresses.  When `hist` is given, every
-// valid id is also counted into it.  Returns false if one of the token's ids lies outside [-1, E).
-__device__ __forceinline__ bool token_membership(const LayoutLaunch& L, int64_t t, bool valid, int32_t* hist,
-                                                 int32_t* tok) {
-  bool bad = false;
-  const int64_t* ids = L.idx + t * L.k;
-  uint8_t* member = L.d.token_in_rank + t * L.R;
-  if (L.R <= 64) {
-    uint64_t mask = 0;
-    if (valid) {
-#pragma unroll 4
-      for (int j = 0; j < L.k; ++j) {
-        const int32_t e = expert_of(__ldg(ids + j), L.E);
-        bad |= e == -2;
-        if (e >= 0) {
-          if (hist) atomicAdd_block(&hist[e], 1);
-          mask |= 1ull << ((uint32_t)e / (uint32_t)L.E_loc);
-        }
-      }
-      for (int r = 0; r < L.R; ++r) member[r] = (uint8_t)((mask >> r) & 1);
-    }
-    const int lane = threadIdx.x & 31;
-    for (int r = 0; r < L.R; ++r) {
-      const int c = __popc(__ballot_sync(0xffffffffu, (mask >> r) & 1));
-      if (lane == 0 && c) atomicAdd_block(&tok[r], c);
-    }
-  } else if (valid) {
-    for (int r = 0; r < L.R; ++r) member[r] = 0;
-    for (int j = 0; j < L.k; ++j) {
-      const int32_t e = expert_of(__ldg(ids + j), L.E);
-      bad |= e == -2;
-      if (e < 0) continue;
-      if (hist) atomicAdd_block(&hist[e], 1);
-      const int r = (int)((uint32_t)e / (uint32_t)L.E_loc);
-      bool first = true;  // the token's first id on rank r counts it there
-      for (int j2 = 0; j2 < j; ++j2) {
-        const int32_t e2 = expert_of(__ldg(ids + j2), L.E);
-        if (e2 >= 0 && (int)((uint32_t)e2 / (uint32_t)L.E_loc) == r) first = false;
-      }
-      if (first) {
-        member[r] = 1;
-        atomicAdd_block(&tok[r], 1);
-      }
-    }
-  }
-  return !bad;
-}
-
-constexpr int kAssignBatch = 8;  // rounds of 32 pairs a warp loads before it works on them
-
-// One round of 32 pairs of a warp's run (lane = pair, e = expert id or -1): the group of lanes
-// with equal ids adds its size to h[e] through its first lane.
-__device__ __forceinline__ void histogram_round(int32_t e, int32_t* h) {
-  const int lane = threadIdx.x & 31;
-  const uint32_t peers = __match_any_sync(0xffffffffu, e);
-  if (e >= 0 && lane == __ffs(peers) - 1) h[e] += __popc(peers);
-  __syncwarp();
-}
-
-// One round of the assignment: pair p (when in_range) with expert e (or -1) and weight w gets
-// row h[e] + (lanes below it with the same id); h[e] advances by the group's size.  Writes slot,
-// pair rank, pair weight and the row maps.  Returns true on a row >= row_cap.
-__device__ __forceinline__ bool assign_round(const LayoutLaunch& L, int64_t p, bool in_range, int32_t e, float w,
-                                             int32_t* h) {
-  const int lane = threadIdx.x & 31;
-  const uint32_t peers = __match_any_sync(0xffffffffu, e);
-  int32_t row = -1;
-  if (e >= 0) row = h[e] + __popc(peers & lanemask_lt());
-  __syncwarp();
-  if (e >= 0 && lane == __ffs(peers) - 1) h[e] += __popc(peers);
-  __syncwarp();
-  bool overflow = false;
-  if (in_range) {
-    // 32-bit divisions: e < E and p < T * k < 2^31
-    const int rk = e >= 0 ? (int)((uint32_t)e / (uint32_t)L.E_loc) : -1;
-    L.d.slot[p] = row;
-    L.d.pair_rank[p] = rk;
-    L.d.pair_w[p] = w;
-    if (e >= 0) {
-      if (row < L.row_cap) {
-        L.d.row_src[(int64_t)rk * L.row_cap + row] = (int32_t)((uint32_t)p / (uint32_t)L.k);
-        L.d.row_w[(int64_t)rk * L.row_cap + row] = w;
-      } else {
-        overflow = true;
-      }
-    }
-  }
-  return overflow;
-}
 
 // Phase 1 of the slot assignment: histogram h[E] of the warp's pairs [wp0, wp1) (h zeroed).
 __device__ __forceinline__ void warp_histogram(const LayoutLaunch& L, int64_t wp0, int64_t wp1, int32_t* h) {
@@ -159,30 +59,6 @@ __device__ __forceinline__ bool warp_assign(const LayoutLaunch& L, int64_t wp0, 
       if (base + r * 32 >= wp1) break;  // warp-uniform: the rest of the batch is empty
       const int64_t p = base + r * 32 + lane;
       overflow |= assign_round(L, p, p < wp1, ev[r], wv[r], h);
-    }
-  }
-  return overflow;
-}
-
-// Padding rows of the row maps: warp w0, w0 + wstride, ... takes experts in turn and its lanes
-// stride over the expert's padding rows [psum - pad, psum) (pad from pad_excl, psum and pad_excl
-// in global or shared memory).  Returns true on a row >= row_cap.
-__device__ __forceinline__ bool row_map_padding(const LayoutLaunch& L, const int32_t* pad_excl, const int32_t* psum,
-                                                int64_t w0, int64_t wstride) {
-  const int lane = threadIdx.x & 31;
-  bool overflow = false;
-  for (int64_t e = w0; e < L.E; e += wstride) {
-    const int32_t pad_e = pad_excl[e + 1] - pad_excl[e];
-    if (pad_e == 0) continue;
-    const int32_t end = psum[e];
-    const int64_t base = (int64_t)((uint32_t)e / (uint32_t)L.E_loc) * L.row_cap;
-    for (int32_t row = end - pad_e + lane; row < end; row += 32) {
-      if (row < L.row_cap) {
-        L.d.row_src[base + row] = -1;
-        L.d.row_w[base + row] = 0.0f;
-      } else {
-        overflow = true;
-      }
     }
   }
   return overflow;
@@ -240,108 +116,6 @@ __device__ __forceinline__ void token_rows_group(const LayoutLaunch& L, int64_t 
     }
   }
   __syncthreads();
-}
-
-// Block-wide exclusive scan of one value per thread (warp shuffles + one smem pass).
-__device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_tot, int32_t* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  int32_t incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int32_t n = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += n;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int32_t w = lane < nwarps ? warp_tot[lane] : 0;
-    int32_t wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int32_t n = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += n;
-    }
-    if (lane < nwarps) warp_tot[lane] = wi - w;  // exclusive warp offsets
-    if (lane == 31) *total = wi;
-  }
-  __syncthreads();
-  const int32_t r = warp_tot[warp] + incl - v;
-  __syncthreads();
-  return r;
-}
-
-// Given cnt[] (global memory written by other CTAs when kCntGlobal, else this CTA's shared
-// memory), one CTA computes, with al / pad / gincl / pad_s as [E] or [E + 1] shared arrays:
-// align_up(cnt, A), the padding prefix over all experts (to pad_excl and pad_s), psum restarted
-// at every rank (to psum and psum_s), rows_per_rank and the capacity flag.  With publish = false
-// only the shared arrays are written (CTAs that compute the same values for their own use).
-template <bool kCntGlobal>
-__device__ __forceinline__ void block_psum(const LayoutLaunch& L, const int32_t* cnt, int64_t cap_check, int32_t* al,
-                                           int32_t* pad, int32_t* gincl, int32_t* pad_s, int32_t* psum_s,
-                                           bool publish = true) {
-  __shared__ int32_t warp_tot[32];
-  __shared__ int32_t totals[2];
-  const int E = L.E, tid = threadIdx.x;
-  for (int x = tid; x < E; x += blockDim.x) {
-    const int32_t n = kCntGlobal ? __ldcg(cnt + x) : cnt[x];  // L2: values other CTAs wrote
-    al[x] = align_up_dev(n, L.A);
-    pad[x] = al[x] - n;
-  }
-  __syncthreads();
-  const int per = (E + blockDim.x - 1) / blockDim.x;
-  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
-  int32_t sa = 0, sp = 0;
-  for (int x = e0; x < e1; ++x) {
-    sa += al[x];
-    sp += pad[x];
-  }
-  int32_t ra = block_exclusive_scan(sa, warp_tot, &totals[0]);
-  int32_t rp = block_exclusive_scan(sp, warp_tot, &totals[1]);
-  for (int x = e0; x < e1; ++x) {
-    if (publish) L.d.pad_excl[x] = rp;
-    if (pad_s) pad_s[x] = rp;
-    rp += pad[x];
-    ra += al[x];
-    gincl[x] = ra;
-  }
-  if (tid == 0) {
-    if (publish) L.d.pad_excl[E] = totals[1];
-    if (pad_s) pad_s[E] = totals[1];
-  }
-  __syncthreads();
-  for (int x = tid; x < E; x += blockDim.x) {
-    const int first = (x / L.E_loc) * L.E_loc;
-    const int32_t v = gincl[x] - (gincl[first] - al[first]);
-    if (publish) L.d.psum[x] = v;
-    if (psum_s) psum_s[x] = v;
-  }
-  for (int r = tid; publish && r < L.R; r += blockDim.x) {
-    const int first = r * L.E_loc, last = first + L.E_loc - 1;
-    const int32_t nrows = gincl[last] - (gincl[first] - al[first]);
-    L.d.rows_per_rank[r] = nrows;
-    if (cap_check > 0 && nrows > cap_check) atomicOr(L.d.status, kStatusCapacity);
-  }
-  __syncthreads();
-}
-
-// With do_cpu_sync: hand the status flags and the per-rank counts to the host as soon as they
-// are final (after psum), through mapped pinned memory, so the host's wait overlaps the rest of
-// the layout.  Words: [0] status flags, [7] ready = 1 (written last, after a system-scope fence),
-// [8, 8 + R) tokens_per_rank, [8 + R, 8 + 2R) rows_per_rank.  Called by every thread of the CTA
-// that published psum / rows_per_rank, after block_psum.
-__device__ __forceinline__ void publish_host_counts(const LayoutLaunch& L) {
-  int32_t* hc = L.d.host_counts;
-  if (hc == nullptr) return;
-  for (int r = threadIdx.x; r < L.R; r += blockDim.x) {
-    hc[8 + r] = __ldcg(L.d.tokens_per_rank + r);
-    hc[8 + L.R + r] = __ldcg(L.d.rows_per_rank + r);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    hc[0] = atomicOr(L.d.status, 0);
-    __threadfence_system();  // the counts reach host memory before the flag
-    *reinterpret_cast<volatile int32_t*>(hc + 7) = 1;
-  }
 }
 
 // ------------------------------------------------------------------------------------ count
@@ -438,8 +212,8 @@ __global__ void __launch_bounds__(kScanThreads) k_layout_scan(LayoutLaunch L, in
   if (!is_last) return;
   __threadfence();
   if (tid == 0) *L.d.ticket = 0;  // ready for the next layout on this scratch
-  block_psum<true>(L, L.d.cnt, cap_check, sm, sm + E, sm + 2 * E, nullptr, nullptr);
-  publish_host_counts(L);
+  block_psum<true>(L, L.d.cnt, cap_check, sm, sm + E, sm + 2 * E, nullptr, nullptr, true, whole_cta());
+  publish_host_counts(L, whole_cta());
 }
 
 // ------------------------------------------------------------------------------------ assign
@@ -493,158 +267,31 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L
 }
 
 // ------------------------------------------------------------------------------------ fused
-// Batches of at most one chunk per SM in one cooperative launch (every CTA resident at once), a
-// CTA per chunk of 256 threads:
-//   1. count: each warp loads its contiguous run of the chunk's pairs into registers (at most
-//      kFusedRounds rounds of 32) and histograms it; token membership as k_layout_count; chunk
-//      counts to global memory and added atomically into the expert totals cnt; then the CTA
-//      arrives at a grid barrier (the ticket word; ticket and cnt cleared before the launch) and
-//      waits, bounded, until every CTA has arrived;
-//   2. every CTA reads the totals and sums the counts of the chunks before its own (its offsets
-//      inside each expert); then align / padding prefix / psum as the scan kernel's last CTA
-//      (CTA 0 alone publishes psum, pad_excl, rows_per_rank);
-//   3. assign: as k_layout_assign for its chunk (pairs from registers), based at those offsets;
-//      padding rows of the row maps over all CTAs' warps; by rank, the token rows based at the
-//      chunk's rank offsets.
-// One launch and one global handoff instead of three kernels; the results are the same.
-__device__ __forceinline__ bool wait_count_reached(const int32_t* p, int32_t target, int32_t* status) {
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t n = 0;; ++n) {
-    int32_t v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    if (v >= target) return true;
-    if ((n & 63) == 63 && globaltimer_ns() - t0 > kWaitLimitNs) break;
-  }
-  atomicOr(status, kStatusTimeout);
-  return false;
-}
-
+// The one-launch layout (layout_body.cuh, fused_layout_chunk): a CTA of 256 threads per chunk, in
+// one cooperative launch; by rank, then the token rows of the chunk, in groups of blockDim tokens
+// based at the chunk's per-rank offsets.  One launch and one global handoff instead of three
+// kernels; the results are the same.
+template <int kRounds>
 __global__ void __launch_bounds__(kLayoutThreads, 1) k_layout_fused(LayoutLaunch L, int64_t cap_check) {
   extern __shared__ int32_t sm[];
-  const int E = L.E, R = L.R, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int c = blockIdx.x, C = gridDim.x;
-  int32_t* whist = sm;                        // [kLayoutWarps][E]
-  int32_t* hist = whist + kLayoutWarps * E;   // [E]  expert totals
-  int32_t* off = hist + E;                    // [E]  rows of each expert in the chunks before c
-  int32_t* al = off + E;                      // [E]
-  int32_t* pad = al + E;                      // [E]
-  int32_t* gincl = pad + E;                   // [E]
-  int32_t* psum_s = gincl + E;                // [E]
-  int32_t* pad_s = psum_s + E;                // [E + 1]
-  int32_t* tok = pad_s + E + 1;               // [R]
   __shared__ int32_t base_r[kMaxByRankRanks];
   __shared__ int32_t wcnt[kLayoutWarps * kMaxByRankRanks];
   __shared__ int32_t go;
   grid_dependents_launch();
-
-  // the warp's contiguous run of the chunk's pairs, held in registers for counting and assigning
-  const int64_t t0 = (int64_t)c * L.chunk, t1 = min(L.T, t0 + L.chunk);
-  const int64_t p0 = t0 * L.k, np = (t1 - t0) * L.k;
-  const int64_t per = (np + kLayoutWarps - 1) / kLayoutWarps;
-  const int64_t wp0 = p0 + min(np, warp * per), wp1 = p0 + min(np, (warp + 1) * per);
-  int32_t ev[kFusedRounds];
-  float wv[kFusedRounds];
-  bool ok = true;
-#pragma unroll
-  for (int r = 0; r < kFusedRounds; ++r) {
-    const int64_t p = wp0 + r * 32 + lane;
-    const int32_t e = p < wp1 ? expert_of(__ldg(L.idx + p), L.E) : -1;
-    ok &= e != -2;
-    ev[r] = max(e, -1);
-    wv[r] = (p < wp1 && L.w) ? __ldg(L.w + p) : 0.0f;
-  }
-  int32_t* h = whist + warp * E;
-  for (int e = lane; e < E; e += 32) h[e] = 0;
-  for (int r = tid; r < R; r += blockDim.x) tok[r] = 0;
-  __syncthreads();
-  // 1. count: per-warp histograms, token membership (ids now in L1), chunk counts
-#pragma unroll
-  for (int r = 0; r < kFusedRounds; ++r)
-    if (wp0 + r * 32 < wp1) histogram_round(ev[r], h);
-  for (int64_t tb = t0; tb < t1; tb += blockDim.x) {  // same trip count for every thread
-    const int64_t t = tb + tid;
-    ok &= token_membership(L, t, t < t1, nullptr, tok);
-  }
-  if (!ok) atomicOr(L.d.status, kStatusBadExpert);
-  __syncthreads();
-  for (int e = tid; e < E; e += blockDim.x) {
-    int32_t n = 0;
-    for (int w = 0; w < kLayoutWarps; ++w) n += whist[w * E + e];
-    L.d.chunk_cnt[(int64_t)c * E + e] = n;
-    if (n) atomicAdd(L.d.cnt + e, n);  // expert totals (cleared before the launch): order-free
-  }
-  for (int r = tid; r < R; r += blockDim.x) {
-    if (tok[r]) atomicAdd(L.d.tokens_per_rank + r, tok[r]);  // integer sum: order-free
-    if (L.by_rank) L.d.chunk_tok[(int64_t)c * R + r] = tok[r];
-  }
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    atomicAdd(L.d.ticket, 1);
-    go = wait_count_reached(L.d.ticket, C, L.d.status);
-  }
-  __syncthreads();
-  if (!go) return;
-
-  // 2. the expert totals, and the chunk's offsets from the counts of the chunks before it
-  // (kFusedLoads loads in flight); then psum.  CTA 0 needs no offsets, so the counts reach the
-  // host right after the barrier.
-  for (int e = tid; e < E; e += blockDim.x) {
-    const int32_t total = __ldcg(L.d.cnt + e);  // issued first: in flight with the chunk loads
-    int32_t before = 0;
-    for (int cb = 0; cb < c; cb += kFusedLoads) {
-      int32_t v[kFusedLoads];
-#pragma unroll
-      for (int q = 0; q < kFusedLoads; ++q)
-        v[q] = cb + q < c ? __ldcg(L.d.chunk_cnt + (int64_t)(cb + q) * E + e) : 0;
-#pragma unroll
-      for (int q = 0; q < kFusedLoads; ++q) before += v[q];
-    }
-    off[e] = before;
-    hist[e] = total;
-  }
-  if (L.by_rank)
-    for (int r = tid; r < R; r += blockDim.x) {
-      int32_t before = 0;
-      for (int cc = 0; cc < c; ++cc) before += __ldcg(L.d.chunk_tok + (int64_t)cc * R + r);
-      base_r[r] = before;
-    }
-  __syncthreads();
-  block_psum<false>(L, hist, cap_check, al, pad, gincl, pad_s, psum_s, c == 0);
-  if (c == 0) publish_host_counts(L);
-
-  // 3. assign: warp bases (exclusive over warps, from the expert's segment start and the chunk's
-  // offset), then the warp's pairs from registers
-  for (int e = tid; e < E; e += blockDim.x) {
-    int32_t base = psum_s[e] - al[e] + off[e];
-    for (int w = 0; w < kLayoutWarps; ++w) {
-      const int32_t v = whist[w * E + e];
-      whist[w * E + e] = base;
-      base += v;
-    }
-  }
-  __syncthreads();
-  bool overflow = false;
-#pragma unroll
-  for (int r = 0; r < kFusedRounds; ++r) {
-    const int64_t p = wp0 + r * 32 + lane;
-    if (wp0 + r * 32 < wp1) overflow |= assign_round(L, p, p < wp1, ev[r], wv[r], h);
-  }
-  overflow |= row_map_padding(L, pad_s, psum_s, (int64_t)c * kLayoutWarps + warp, (int64_t)C * kLayoutWarps);
-  if (overflow) atomicOr(L.d.status, kStatusCapacity);
-  if (L.by_rank) {
+  if (!fused_layout_chunk<kRounds>(L, cap_check, blockIdx.x, gridDim.x, whole_cta(), sm, base_r, &go)) return;
+  if (L.by_rank) {  // groups of blockDim tokens (a chunk may hold several), based at the chunk's offsets
     __syncthreads();
-    token_rows_group(L, t0, t1, base_r, wcnt);
+    const int64_t t0 = (int64_t)blockIdx.x * L.chunk, t1 = min(L.T, t0 + L.chunk);
+    for (int64_t tg = t0; tg < t1; tg += blockDim.x) token_rows_group(L, tg, t1, base_r, wcnt);
   }
 }
-
-size_t fused_layout_smem(int E, int R) { return sizeof(int32_t) * ((size_t)(kLayoutWarps + 7) * E + 1 + R); }
 
 // At most one chunk per SM of the budget (so every CTA can be resident), the chunk's pairs in
 // the warps' registers, and bounded redundant summing.
 bool layout_fits_fused(int num_chunks, int chunk, int k, int E, int sm_budget) {
   return num_chunks >= 1 && num_chunks <= sm_budget && E <= kFusedMaxExperts &&
-         (int64_t)chunk * k <= (int64_t)kLayoutThreads * kFusedRounds && (int64_t)num_chunks * E <= kFusedMaxChunkCounts;
+         (int64_t)chunk * k <= (int64_t)kLayoutThreads * kFusedMaxRounds &&
+         (int64_t)num_chunks * E <= kFusedMaxChunkCounts;
 }
 
 // ------------------------------------------------------------------------------------ small
@@ -698,7 +345,7 @@ __global__ void __launch_bounds__(kSmallThreads) k_layout_small(LayoutLaunch L, 
   }
   for (int r = tid; r < L.R; r += blockDim.x) L.d.tokens_per_rank[r] = tok[r];
   __syncthreads();
-  block_psum<false>(L, cnt_s, cap_check, al, pad, gincl, pad_s, psum_s);
+  block_psum<false>(L, cnt_s, cap_check, al, pad, gincl, pad_s, psum_s, true, whole_cta());
 
   for (int e = tid; e < E; e += blockDim.x) {  // base every warp's rows at the segment start
     const int32_t seg = psum_s[e] - al[e];
@@ -742,8 +389,11 @@ static cudaError_t ensure_smem_attrs() {
     err = cudaFuncSetAttribute(k_layout_assign, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(sizeof(int32_t) * kLayoutWarps * kMaxExperts));
   if (err == cudaSuccess)
-    err = cudaFuncSetAttribute(k_layout_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(k_layout_fused<kFusedRounds>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)fused_layout_smem(kFusedMaxExperts, kFusedMaxExperts));  // R <= E
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(k_layout_fused<kFusedMaxRounds>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)fused_layout_smem(kFusedMaxExperts, kFusedMaxExperts));
   if (err == cudaSuccess && dev < 64) done |= 1ull << dev;
   return err;
 }
@@ -779,7 +429,11 @@ cudaError_t launch_layout_fused(const LayoutLaunch& L, int64_t cap_check, cudaSt
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, k_layout_fused, L, cap_check);
+  // pairs per warp: ceil(chunk * k / warps), held in rounds of 32
+  const int64_t per_warp = ((int64_t)L.chunk * L.k + kLayoutWarps - 1) / kLayoutWarps;
+  if (per_warp > 32 * kFusedMaxRounds) return cudaErrorInvalidValue;
+  if (per_warp <= 32 * kFusedRounds) err = cudaLaunchKernelEx(&cfg, k_layout_fused<kFusedRounds>, L, cap_check);
+  else err = cudaLaunchKernelEx(&cfg, k_layout_fused<kFusedMaxRounds>, L, cap_check);
   note_launch();
   return err;
 }

@@ -216,31 +216,11 @@ static bool wait_host_counts(const moe_handle_t* h, cudaStream_t s) {
   return true;
 }
 
-}  // namespace moe
-
-using namespace moe;
-
-extern "C" {
-
-int64_t moe_recv_capacity_hint(const moe_params_t* p, int64_t max_tokens_per_rank) {
-  if (check_params(p) == MOE_ERR_INVALID_ARG || max_tokens_per_rank < 0) return -1;
-  const int64_t e_loc = p->num_experts / p->num_logical_ranks;
-  const int64_t per_token = p->topk < e_loc ? p->topk : e_loc;
-  return (int64_t)p->num_logical_ranks * max_tokens_per_rank * per_token + e_loc * (p->expert_alignment - 1);
-}
-
-int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk_weights, void* stream,
-               moe_handle_t** out_handle, int32_t* host_rows_per_rank) {
-  TraceRange trace("moe_layout");
-  if (!out_handle) return MOE_ERR_INVALID_ARG;
-  *out_handle = nullptr;
-  int rc = check_params(p);
-  if (rc != MOE_OK) return rc;
-  if (!topk_idx && p->num_tokens > 0) return MOE_ERR_INVALID_ARG;
-  if (!aligned4(topk_weights)) return MOE_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(topk_idx) & 7u) != 0) return MOE_ERR_INVALID_ARG;
-
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+// Everything moe_layout does before its launches: the handle and its arrays (one stream-ordered
+// allocation), the mapped count block under do_cpu_sync, the chunking and the launch description.
+// The arguments are checked by the caller.  On failure nothing is left allocated.
+static int layout_prepare(const moe_params_t* p, const int64_t* topk_idx, const float* topk_weights, cudaStream_t s,
+                          moe_handle_t** out_handle, LayoutLaunch* out_launch, bool* out_fused) {
   moe_handle_t* h = new (std::nothrow) moe_handle_t();
   if (!h) return MOE_ERR_OOM;
   h->p = *p;
@@ -251,14 +231,24 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   }
   const int64_t T = p->num_tokens, k = p->topk, E = p->num_experts, R = p->num_logical_ranks;
   // Chunks.  The one-launch layout takes the smallest chunk of 32..256 tokens that leaves at most
-  // one chunk per SM the layout may use, if its other limits hold (layout_fits_fused).
+  // one chunk per SM the layout may use, if its other limits hold (layout_fits_fused).  Under a
+  // num_sms cap, when 256-token chunks still outnumber the SMs, it takes one chunk per SM of
+  // ceil(T / SMs) tokens rounded up to a warp, if the pairs still fit the warps' registers.
   // Otherwise the count / assign kernels halve the chunk from kChunkTokens down to 32 tokens
   // while the batch gives fewer than two chunks per SM, so it still spreads over many CTAs
   // (a warp's run of pairs, chunk * k / 8, sets the assign kernel's serial work).
   const int sm_budget = grid_for(p->num_sms, h->device);
   int chunk = 32;
   while ((T + chunk - 1) / chunk > sm_budget && chunk < kChunkTokens) chunk *= 2;
-  const bool fused = layout_fits_fused((int)((T + chunk - 1) / chunk), chunk, (int)k, (int)E, sm_budget);
+  bool fused = layout_fits_fused((int)((T + chunk - 1) / chunk), chunk, (int)k, (int)E, sm_budget);
+  if (!fused && sm_budget < sm_count(h->device) && (T + chunk - 1) / chunk > sm_budget) {
+    const int64_t wide = align_up64((T + sm_budget - 1) / sm_budget, 32);
+    if (wide < ((int64_t)1 << 30) &&
+        layout_fits_fused((int)((T + wide - 1) / wide), (int)wide, (int)k, (int)E, sm_budget)) {
+      chunk = (int)wide;
+      fused = true;
+    }
+  }
   if (!fused) {
     const int64_t want_chunks = 2 * (int64_t)sm_count(h->device);
     chunk = kChunkTokens;
@@ -348,10 +338,17 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
   L.by_rank = by_rank ? 1 : 0;
   L.d = d;
 
-  // count -> scan -> assign back to back, or all three in one cooperative launch when there is
-  // at most a chunk per SM; with do_cpu_sync one host wait at the end.  (Small batches take
-  // 32-token chunks over many CTAs: faster than one CTA whose warps each walk hundreds of pairs.)
-  cudaError_t err = cudaMemsetAsync(d.status, 0, (size_t)(32 + 8 * R + 4 * E), s);
+  *out_handle = h;
+  *out_launch = L;
+  *out_fused = fused;
+  return MOE_OK;
+}
+
+// The layout's launches: the status block cleared, then the one-launch layout or count -> scan ->
+// assign.  (Small batches take 32-token chunks over many CTAs: faster than one CTA whose warps
+// each walk hundreds of pairs.)
+static cudaError_t layout_enqueue(const moe_params_t* p, const LayoutLaunch& L, bool fused, cudaStream_t s) {
+  cudaError_t err = cudaMemsetAsync(L.d.status, 0, (size_t)(32 + 8 * (int64_t)L.R + 4 * (int64_t)L.E), s);
   if (fused) {
     if (err == cudaSuccess) err = launch_layout_fused(L, p->recv_capacity_rows, s);
   } else {
@@ -359,6 +356,69 @@ int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk
     if (err == cudaSuccess) err = launch_layout_scan(L, p->recv_capacity_rows, s);
     if (err == cudaSuccess) err = launch_layout_assign(L, s);
   }
+  return err;
+}
+
+// The launch description of an expanded dispatch on handle h.
+static DispatchLaunch expanded_dispatch(const moe_handle_t* h, const void* x, void* recv_x, float* recv_scales,
+                                        float* recv_weights, int64_t cap, int do_zero_padding, int num_sms) {
+  const moe_params_t& p = h->p;
+  DispatchLaunch L{};
+  L.x = x;
+  L.recv_x = recv_x;
+  L.recv_scales = recv_scales;
+  L.recv_w = recv_weights;
+  L.T = p.num_tokens;
+  L.cap = cap;
+  L.H = p.hidden;
+  L.k = p.topk;
+  L.E = p.num_experts;
+  L.E_loc = p.num_experts / p.num_logical_ranks;
+  L.zero_padding = do_zero_padding;
+  L.R = p.num_logical_ranks;
+  L.grid = grid_for(num_sms, h->device);
+  L.pair_rank = h->d.pair_rank;
+  L.slot = h->d.slot;
+  L.pair_w = h->d.pair_w;
+  L.psum = h->d.psum;
+  L.pad_excl = h->d.pad_excl;
+  L.status = h->d.status;
+  return L;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int64_t moe_recv_capacity_hint(const moe_params_t* p, int64_t max_tokens_per_rank) {
+  if (check_params(p) == MOE_ERR_INVALID_ARG || max_tokens_per_rank < 0) return -1;
+  const int64_t e_loc = p->num_experts / p->num_logical_ranks;
+  const int64_t per_token = p->topk < e_loc ? p->topk : e_loc;
+  return (int64_t)p->num_logical_ranks * max_tokens_per_rank * per_token + e_loc * (p->expert_alignment - 1);
+}
+
+int moe_layout(const moe_params_t* p, const int64_t* topk_idx, const float* topk_weights, void* stream,
+               moe_handle_t** out_handle, int32_t* host_rows_per_rank) {
+  TraceRange trace("moe_layout");
+  if (!out_handle) return MOE_ERR_INVALID_ARG;
+  *out_handle = nullptr;
+  int rc = check_params(p);
+  if (rc != MOE_OK) return rc;
+  if (!topk_idx && p->num_tokens > 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned4(topk_weights)) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(topk_idx) & 7u) != 0) return MOE_ERR_INVALID_ARG;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  moe_handle_t* h = nullptr;
+  LayoutLaunch L{};
+  bool fused = false;
+  rc = layout_prepare(p, topk_idx, topk_weights, s, &h, &L, &fused);
+  if (rc != MOE_OK) return rc;
+  const int64_t R = p->num_logical_ranks;
+  const bool publish = p->do_cpu_sync && !(p->flags & MOE_DEFER_EPILOGUE);
+  cudaError_t err = layout_enqueue(p, L, fused, s);
   if (err != cudaSuccess) {
     release(h);
     return MOE_ERR_CUDA;
@@ -436,27 +496,57 @@ int moe_dispatch(const moe_handle_t* h, const void* x, int out_dtype, void* recv
       if (v > cap) return MOE_ERR_CAPACITY;
   }
   if (p.num_tokens == 0) return MOE_OK;
-  DispatchLaunch L{};
-  L.x = x;
-  L.recv_x = recv_x;
-  L.recv_scales = recv_scales;
-  L.recv_w = recv_weights;
-  L.T = p.num_tokens;
-  L.cap = cap;
-  L.H = p.hidden;
-  L.k = p.topk;
-  L.E = p.num_experts;
-  L.E_loc = p.num_experts / p.num_logical_ranks;
-  L.zero_padding = do_zero_padding;
-  L.R = p.num_logical_ranks;
-  L.grid = grid_for(num_sms, h->device);
-  L.pair_rank = h->d.pair_rank;
-  L.slot = h->d.slot;
-  L.pair_w = h->d.pair_w;
-  L.psum = h->d.psum;
-  L.pad_excl = h->d.pad_excl;
-  L.status = h->d.status;
+  const DispatchLaunch L = expanded_dispatch(h, x, recv_x, recv_scales, recv_weights, cap, do_zero_padding, num_sms);
   return launch_dispatch(L, fp8, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_layout_dispatch(const moe_params_t* p, const int64_t* topk_idx, const float* topk_weights, const void* x,
+                        int out_dtype, void* recv_x, float* recv_scales, float* recv_weights, int do_zero_padding,
+                        void* stream, moe_handle_t** out_handle) {
+  TraceRange trace("moe_layout_dispatch");
+  if (!out_handle) return MOE_ERR_INVALID_ARG;
+  *out_handle = nullptr;
+  int rc = check_params(p);
+  if (rc != MOE_OK) return rc;
+  if (p->do_cpu_sync != 0 || p->flags != 0) return MOE_ERR_INVALID_ARG;
+  if (!topk_idx && p->num_tokens > 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned4(topk_weights) || (reinterpret_cast<uintptr_t>(topk_idx) & 7u) != 0) return MOE_ERR_INVALID_ARG;
+  if (do_zero_padding != 0 && do_zero_padding != 1) return MOE_ERR_INVALID_ARG;
+  if (out_dtype != MOE_DTYPE_BF16 && out_dtype != MOE_DTYPE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+  const bool fp8 = out_dtype == MOE_DTYPE_FP8_E4M3;
+  if (fp8 && (p->hidden % 128 != 0 || !recv_scales || !aligned4(recv_scales))) return MOE_ERR_INVALID_ARG;
+  if (p->num_tokens > 0 && (!x || !recv_x)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(recv_x) || !aligned4(recv_weights)) return MOE_ERR_INVALID_ARG;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  moe_handle_t* h = nullptr;
+  LayoutLaunch L{};
+  bool fused = false;
+  rc = layout_prepare(p, topk_idx, topk_weights, s, &h, &L, &fused);
+  if (rc != MOE_OK) return rc;
+  cudaError_t err = cudaSuccess;
+  if (p->num_tokens > 0) {
+    const int64_t cap = p->recv_capacity_rows;
+    const DispatchLaunch D =
+        expanded_dispatch(h, x, recv_x, recv_scales, recv_weights, cap, do_zero_padding, p->num_sms);
+    if (fused && L.num_chunks <= D.grid &&
+        layout_dispatch_fits(p->num_tokens, p->hidden, fp8, p->num_experts, p->num_logical_ranks, D.grid, L.chunk,
+                             L.k)) {
+      err = cudaMemsetAsync(L.d.status, 0, (size_t)(32 + 8 * (int64_t)L.R + 4 * (int64_t)L.E), s);
+      if (err == cudaSuccess) err = launch_layout_dispatch(L, cap, D, fp8, s);
+    } else {  // the same results from the layout's launches and the dispatch kernel
+      err = layout_enqueue(p, L, fused, s);
+      if (err == cudaSuccess) err = launch_dispatch(D, fp8, s);
+    }
+  } else {
+    err = layout_enqueue(p, L, fused, s);
+  }
+  if (err != cudaSuccess) {
+    release(h);
+    return MOE_ERR_CUDA;
+  }
+  *out_handle = h;
+  return MOE_OK;
 }
 
 int moe_combine(const moe_handle_t* h, const void* y, const float* topk_weights, const void* bias, void* out,

@@ -141,6 +141,9 @@ struct DispatchLaunch {
 };
 
 cudaError_t launch_dispatch(const DispatchLaunch& L, bool fp8, cudaStream_t s);
+bool layout_dispatch_fits(int64_t T, int64_t H, bool fp8, int E, int R, int grid, int chunk, int k);
+cudaError_t launch_layout_dispatch(const LayoutLaunch& LL, int64_t cap_check, const DispatchLaunch& L, bool fp8,
+                                   cudaStream_t s);
 
 struct CombineLaunch {
   const void* y;
@@ -394,32 +397,36 @@ __device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
 // ------------------------------------------------------------------------------ pair metadata
 namespace moe {
 
-// One warp-wide load of the (rank, slot, weight) of up to 32 consecutive (token, j) pairs:
-// lane l holds pair p0 + l (p0 = first token of the batch * k), if it lies before p_end.
+// The (rank, slot, weight[, expert]) of one (token, j) pair.
 struct PairBatch {
   int32_t rank, slot;
   float w;
   int32_t e;  // expert id (only when `ids` is given), else -1
 };
 
-__device__ __forceinline__ PairBatch load_pair_batch(const int32_t* pair_rank, const int32_t* slot,
-                                                     const float* w, int64_t p0, int64_t p_end, int lane,
-                                                     int lanes_used, const int64_t* ids = nullptr) {
+// Tokens of CTA b of G in the dispatch and combine kernels: its q-th token is b + q * G, so the
+// grid works on neighbouring tokens at any moment.  cta_tokens = how many the CTA has.
+__device__ __forceinline__ int64_t cta_tokens(int64_t T) {
+  return (int64_t)blockIdx.x < T ? (T - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+}
+
+__device__ __forceinline__ int64_t cta_token(int64_t q) { return (int64_t)blockIdx.x + q * gridDim.x; }
+
+// One warp-wide load of the pairs of the CTA's tokens q0 .. q0 + 32 / k - 1 (lane l: token q0 +
+// l / k, pair l % k; lanes_used = (32 / k) * k), for token indices below n_tok.
+__device__ __forceinline__ PairBatch load_cta_pairs(const int32_t* pair_rank, const int32_t* slot, const float* w,
+                                                    int64_t q0, int64_t n_tok, int k, int lane, int lanes_used,
+                                                    const int64_t* ids = nullptr) {
   PairBatch b{-1, -1, 0.0f, -1};
-  const int64_t p = p0 + lane;
-  if (lane < lanes_used && p < p_end) {
+  const int q = lane / k, j = lane - q * k;
+  if (lane < lanes_used && q0 + q < n_tok) {
+    const int64_t p = cta_token(q0 + q) * k + j;
     b.rank = __ldg(pair_rank + p);
     b.slot = __ldg(slot + p);
     if (w) b.w = __ldg(w + p);
     if (ids && b.rank >= 0) b.e = (int32_t)__ldg(ids + p);
   }
   return b;
-}
-
-// The contiguous token range [begin, end) of CTA b out of G (balanced split of T tokens).
-__device__ __forceinline__ void cta_token_range(int64_t T, int64_t& begin, int64_t& end) {
-  begin = T * blockIdx.x / gridDim.x;
-  end = T * (blockIdx.x + 1) / gridDim.x;
 }
 
 }  // namespace moe

@@ -143,6 +143,24 @@ int moe_dispatch(const moe_handle_t* handle, const void* x, int out_dtype, void*
                  int do_zero_padding, int num_sms, void* stream);
 
 /*
+ * Layout and expanded dispatch in one call ("From DeepEP to Mega MoE" 2.2: the dispatch kernel
+ * runs its notify warps, which count the routing and build psum, beside the dispatch warps that
+ * move the tokens; "deepep-expert-parallel-dispatch-combine", arithmetic intensity:
+ * do_cpu_sync = False sizes the outputs to capacity and consumers read the device-side psum).
+ * Computes exactly moe_layout followed by moe_dispatch(do_expand = 1) with
+ * cap = params->recv_capacity_rows and num_sms = params->num_sms, and returns the handle as
+ * moe_layout does.  params->do_cpu_sync must be 0 and params->flags 0 (MOE_ERR_INVALID_ARG
+ * otherwise); the other arguments are those of moe_layout and moe_dispatch.  A bad expert id or
+ * a capacity overflow is reported by moe_handle_status.  Small batches (at most 8 tokens per SM
+ * of the budget, with the one-launch layout's limits) run as one cooperative kernel whose
+ * dispatch warps load and quantise the tokens while its layout warps assign the rows; other
+ * batches run the layout's launches and then the dispatch kernel.
+ */
+int moe_layout_dispatch(const moe_params_t* params, const int64_t* topk_idx, const float* topk_weights,
+                        const void* x, int out_dtype, void* recv_x, float* recv_scales, float* recv_weights,
+                        int do_zero_padding, void* stream, moe_handle_t** out_handle);
+
+/*
  * Non-expanded dispatch ("Why MoE gets stuck on communication" 1: without do_expand a destination
  * rank receives each token once; "Chapter 2: repository map" 2.1: token -> rank membership).
  * Rank r receives one row per token that has at least one expert on r, in ascending token order

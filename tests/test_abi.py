@@ -103,3 +103,24 @@ def test_wait_and_event_calls_reject_null_on_the_host():
     assert L.moe_event_record(None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_event_free(None) == moe.MOE_OK
     assert moe.status_string(moe.MOE_NOT_READY) == "not complete yet"
+
+
+def test_layout_dispatch_rejects_bad_arguments_on_the_host():
+    L = moe.lib()
+    h = ctypes.c_void_p(123)
+    ok = moe.params(64, 2, 8, 2, 256, 16, recv_capacity_rows=64, do_cpu_sync=False)
+
+    def call(p, x=0x1000, dtype=moe.MOE_DTYPE_BF16, recv=0x2000, scales=None, zp=1, out=ctypes.byref(h)):
+        return L.moe_layout_dispatch(ctypes.byref(p), ctypes.c_void_p(0x3000), None, ctypes.c_void_p(x), dtype,
+                                     ctypes.c_void_p(recv), scales, None, zp, None, out)
+
+    assert call(moe.params(64, 2, 8, 2, 256, 16, recv_capacity_rows=64, do_cpu_sync=True)) == moe.MOE_ERR_INVALID_ARG
+    assert h.value is None                                   # *out_handle cleared
+    assert call(moe.params(64, 2, 8, 2, 256, 16, recv_capacity_rows=64, do_cpu_sync=False,
+                           by_rank=True)) == moe.MOE_ERR_INVALID_ARG
+    assert call(moe.params(64, 2, 8, 2, 256, 16, recv_capacity_rows=0, do_cpu_sync=False)) == moe.MOE_ERR_INVALID_ARG
+    assert call(ok, dtype=7) == moe.MOE_ERR_INVALID_ARG
+    assert call(ok, x=0x1008) == moe.MOE_ERR_INVALID_ARG      # rows must be 16-byte aligned
+    assert call(ok, zp=2) == moe.MOE_ERR_INVALID_ARG
+    assert call(ok, dtype=moe.MOE_DTYPE_FP8_E4M3) == moe.MOE_ERR_INVALID_ARG   # FP8 needs scales
+    assert call(ok, out=None) == moe.MOE_ERR_INVALID_ARG

@@ -13,13 +13,13 @@ from gpu_helpers import bits, gpu_layout, inputs
 pytestmark = pytest.mark.gpu
 
 
-def _round_trip(wl, mask=0.1, with_bias=True, via_moe_dispatch=False):
+def _round_trip(wl, mask=0.1, with_bias=True, via_moe_dispatch=False, num_sms=0):
     idx, w, x = inputs(wl, mask)
     E, R = wl.experts, wl.ranks
     st, tr, rows = oracle.layout_by_rank(idx.numpy(), E, R)
     assert st == oracle.OK
     cap = int(rows.max()) + 2
-    h = gpu_layout(wl, idx, w, cap=0, by_rank=True)
+    h = gpu_layout(wl, idx, w, cap=0, by_rank=True, num_sms=num_sms)
     torch.cuda.synchronize()
     assert (h.token_rows().cpu().numpy() == tr).all()
     assert (h.tokens_per_rank().cpu().numpy() == rows).all()
@@ -71,6 +71,13 @@ def _round_trip(wl, mask=0.1, with_bias=True, via_moe_dispatch=False):
 def test_by_rank_round_trip(fp8, kw):
     wl = W.WORKLOADS["tiny"].with_(hidden=512, fp8=fp8, **kw)
     _round_trip(wl)
+
+
+def test_by_rank_wide_chunks_under_an_sm_cap():
+    """num_sms = 24 over 8192 tokens: the one-launch layout's chunks of 352 tokens hold several
+    groups of token rows each."""
+    wl = W.WORKLOADS["tiny"].with_(hidden=256, tokens_per_rank=512, ranks=16, experts=128, topk=8)
+    _round_trip(wl, num_sms=24)
 
 
 def test_moe_dispatch_without_expansion():

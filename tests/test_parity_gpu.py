@@ -142,6 +142,22 @@ def test_fused_layout_respects_the_sm_budget():
     _roundtrip_small(wl, idx, w, x, weighted=True, num_sms=32)
 
 
+@pytest.mark.parametrize("num_sms,kw", [
+    (24, dict(tokens_per_rank=512, ranks=16, experts=128, topk=8)),   # skewed shape: 24 chunks of 352 tokens
+    (16, dict(tokens_per_rank=512, ranks=16, experts=128, topk=8)),   # 512-token chunks: 4096 pairs, the limit
+    (16, dict(tokens_per_rank=512, ranks=16, experts=144, topk=9)),   # 4608 pairs per chunk: three kernels
+    (3, dict(tokens_per_rank=300, ranks=3, experts=12, topk=3, alignment=5)),   # chunks of 320, 320, 260 tokens
+])
+def test_wide_chunk_layout_under_an_sm_cap(num_sms, kw):
+    """Under a num_sms cap the one-launch layout takes one chunk per SM of the budget, wider than
+    256 tokens, while a warp's pairs fit its registers (16 rounds of 32); beyond that, the three
+    kernels.  Both sides, with and without host sync, every byte."""
+    wl = W.WORKLOADS["tiny"].with_(hidden=64, **kw)
+    idx, w, x = inputs(wl, 0.05)
+    _roundtrip_small(wl, idx, w, x, weighted=True, with_bias=True, num_sms=num_sms)
+    _roundtrip_small(wl, idx, w, x, cpu_sync=False, num_sms=num_sms)
+
+
 @pytest.mark.parametrize("kw", [
     dict(tokens_per_rank=64, ranks=8, experts=2048, topk=8, alignment=1, hidden=64),   # E at the fused limit
     dict(tokens_per_rank=64, ranks=8, experts=4096, topk=8, alignment=1, hidden=64),   # beyond it: three kernels
