@@ -100,14 +100,19 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
+        self.sink = None
         self.out = ""
         self.t0 = self.t1 = None
 
     def start(self):
+        import tempfile
+        # samples go to a file: a pipe left unread until the end fills (64 KiB, about 30 s of
+        # samples) and stalls the sampler
+        self.sink = tempfile.TemporaryFile(mode="w+")
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}",
                                           "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                                         stdout=self.sink, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
         time.sleep(0.5)   # let the sampler come up before the timed region
@@ -119,18 +124,27 @@ class ClockSampler:
     def mark_stop(self):
         self.t1 = time.time()
 
-    def stop(self):
+    def stop(self, log_path: str | None = None):
         if self.proc is not None:
             time.sleep(2 * self.PERIOD_MS / 1000)
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                self.proc.wait()
+            self.sink.seek(0)
+            self.out = self.sink.read()
+            self.sink.close()
+        if log_path:
+            with open(log_path, "w") as f:
+                f.write(self.out)
 
-    def summary(self):
+    def summary(self, t0: float | None = None, t1: float | None = None):
+        """Clock record of the window [t0, t1] (default: the marked timed region)."""
         import datetime
+        t0 = self.t0 if t0 is None else t0
+        t1 = self.t1 if t1 is None else t1
         rows = []
         for r in self.out.strip().splitlines():
             f = [c.strip() for c in r.split(",")]
@@ -144,13 +158,19 @@ class ClockSampler:
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         pad = self.PERIOD_MS / 1000 * 1.5
-        inside = [r for r in rows if self.t0 is not None and self.t0 - pad <= r[0] <= self.t1 + pad]
-        use = inside or rows
+        inside = [r for r in rows if t0 is not None and t0 - pad <= r[0] <= t1 + pad]
+        if inside:
+            use, where = inside, "timed region"
+        elif t0 is not None:  # a gap in the sampler's output: the two samples nearest the window
+            mid = 0.5 * (t0 + t1)
+            use = sorted(rows, key=lambda r: abs(r[0] - mid))[:2]
+            where = "nearest samples (none inside the timed region)"
+        else:
+            use, where = rows, "whole run (no timed region marked)"
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in use for i in range(4) if r[3][i] == "Active"})
         return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
-                "reasons": reasons, "samples": len(use),
-                "window": "timed region" if inside else "whole run (no sample inside the timed region)"}
+                "reasons": reasons, "samples": len(use), "window": where}
 
 
 # --------------------------------------------------------------------------- distributed plumbing
@@ -321,9 +341,13 @@ def run_e2e(args, world, dev, stream, step, step_bytes, x, idx, w, y, bias, out,
 
 
 # --------------------------------------------------------------------------- workload extras
-def decode_latency(step_parts, stream, dev, n: int = 50) -> dict:
-    """Per-call latency of layout, dispatch and combine, median over n steps, warm (back to back)
-    and cold (L2 flushed by writing a buffer of twice the L2 size before every step)."""
+def decode_latency(step_parts, stream, dev, one_call: bool, n: int = 50) -> dict:
+    """Per-call device time of layout, dispatch and combine, median over n steps, warm (the
+    previous step's data still in L2) and cold (L2 flushed by writing a buffer of twice the L2
+    size before every step).  Each step starts behind a device-side spin of about 200 us, so the
+    host has enqueued the three calls before the first event fires: the intervals hold device
+    time only, not the host's enqueue time (which an idle GPU would otherwise expose in the
+    layout's interval)."""
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
 
@@ -332,6 +356,7 @@ def decode_latency(step_parts, stream, dev, n: int = 50) -> dict:
         for _ in range(n):
             if cold:
                 flush.fill_(1)
+            torch.cuda._sleep(400_000)
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
             step_parts(ev, stream)
             torch.cuda.synchronize()
@@ -339,7 +364,10 @@ def decode_latency(step_parts, stream, dev, n: int = 50) -> dict:
             rec["dispatch"].append(ev[1].elapsed_time(ev[2]) * 1e3)
             rec["combine"].append(ev[2].elapsed_time(ev[3]) * 1e3)
             rec["total"].append(ev[0].elapsed_time(ev[3]) * 1e3)
-        return {k: round(statistics.median(v), 2) for k, v in rec.items()}
+        med = {k: round(statistics.median(v), 2) for k, v in rec.items()}
+        if one_call:  # layout and dispatch are one launch: its time is the first interval
+            med = {"layout_dispatch": med["layout"], "combine": med["combine"], "total": med["total"]}
+        return med
 
     res = {"unit": "us", "warm": run(False), "cold_l2_flushed": run(True), "samples": n}
     # the same round trip captured once in a CUDA graph (do_cpu_sync=0 path), replayed warm
@@ -462,15 +490,19 @@ def expert_gemm_measurement(moe, wl, h, x, cap: int, N: int, stream, dev, iters:
             "iters": iters}
 
 
-def run_ours(args) -> int:
-    world, rank, local = dist_setup("nccl")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    import combine_moe_layout_07_b200 as moe
+# steps and CPU-baseline sample of the configurations measured beside the headline one: each
+# timed region lasts about 0.3 s (several clock samples), each oracle pass a few seconds at most
+SIDE_WORKLOADS = {"decode": {"steps": 4000, "cpu_tokens": 1024},
+                  "large": {"steps": 600, "cpu_tokens": 4096},
+                  "skewed": {"steps": 300, "cpu_tokens": 8192}}
 
-    wl = W.WORKLOADS[args.workload]
-    if args.tokens_per_rank:
-        wl = wl.with_(tokens_per_rank=args.tokens_per_rank)
+
+def measure_workload(moe, wl: W.Workload, args, world: int, rank: int, dev, stream, clk: ClockSampler,
+                     steps: int, warmup: int, cpu_tokens: int, want_e2e: bool) -> dict:
+    """Times `steps` round trips (layout -> dispatch -> combine -> handle free) of one workload
+    after `warmup` untimed ones, bracketed by barrier + synchronize, max over ranks; returns the
+    measurement with its per-kernel times, roofline, clocks, CPU-oracle baseline (rank 0, one
+    GPU) and the workload's own extras (decode latency, skewed overlap)."""
     stream = torch.cuda.current_stream()
     idx_c, w_c = W.gen_routing(wl)
     x_c = W.gen_x(wl)
@@ -511,115 +543,183 @@ def run_ours(args) -> int:
     out = torch.empty(wl.tokens, wl.hidden, dtype=torch.bfloat16, device=dev)
 
     ev = {k: [] for k in ("l0", "l1", "d1", "c1")}
+    # without host sync the layout and the dispatch are one call (moe_layout_dispatch)
+    one_call = not wl.cpu_sync
 
-    def step(record: bool):
-        if record:
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-            e[0].record(stream)
-        h = moe.moe_layout(make_params(p_cap), idx, w, stream=stream)
-        if record:
-            e[1].record(stream)
-        moe.moe_dispatch(h, x, dtype_out, recv, scales, None, cap=cap, do_zero_padding=wl.zero_padding,
-                         num_sms=wl.num_sms, stream=stream)
-        if record:
-            e[2].record(stream)
-        moe.moe_combine(h, y, out, topk_weights=weights_for_combine, bias=bias, cap=cap, num_sms=wl.num_sms,
-                        stream=stream)
-        if record:
-            e[3].record(stream)
-            for key, val in zip(ev, e):
-                ev[key].append(val)
-        moe.moe_handle_free(h)
-
-    clk = ClockSampler(local).start()
-    def step_parts(ev, st):
-        ev[0].record(st)
-        h = moe.moe_layout(make_params(p_cap), idx, w, stream=st)
-        ev[1].record(st)
-        moe.moe_dispatch(h, x, dtype_out, recv, scales, None, cap=cap, do_zero_padding=wl.zero_padding,
-                         num_sms=wl.num_sms, stream=st)
-        ev[2].record(st)
+    def step_parts(e, st):
+        if e is not None:
+            e[0].record(st)
+        if one_call:
+            h = moe.moe_layout_dispatch(make_params(p_cap), idx, w, x, dtype_out, recv, scales, None,
+                                        do_zero_padding=wl.zero_padding, stream=st)
+            if e is not None:
+                e[1].record(st)
+        else:
+            h = moe.moe_layout(make_params(p_cap), idx, w, stream=st)
+            if e is not None:
+                e[1].record(st)
+            moe.moe_dispatch(h, x, dtype_out, recv, scales, None, cap=cap, do_zero_padding=wl.zero_padding,
+                             num_sms=wl.num_sms, stream=st)
+        if e is not None:
+            e[2].record(st)
         moe.moe_combine(h, y, out, topk_weights=weights_for_combine, bias=bias, cap=cap, num_sms=wl.num_sms,
                         stream=st)
-        ev[3].record(st)
+        if e is not None:
+            e[3].record(st)
         moe.moe_handle_free(h)
 
-    for _ in range(args.warmup):
+    def step(record: bool):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if record else None
+        step_parts(e, stream)
+        if record:
+            for key, val in zip(ev, e):
+                ev[key].append(val)
+
+    for _ in range(warmup):
         step(False)
     torch.cuda.synchronize()
-    assert moe.moe_handle_status(moe.moe_layout(make_params(p_cap), idx, w)) == moe.MOE_OK
+    hc = moe.moe_layout(make_params(p_cap), idx, w)
+    assert moe.moe_handle_status(hc) == moe.MOE_OK
+    moe.moe_handle_free(hc)
 
     barrier()
     torch.cuda.synchronize()
     launches0 = moe.moe_kernel_launch_count()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clk.mark_start()
+    w0 = time.time()
     t_start.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         step(True)
     t_end.record(stream)
     torch.cuda.synchronize()
-    clk.mark_stop()
-    clk.stop()
+    w1 = time.time()
     barrier()
     launches = moe.moe_kernel_launch_count() - launches0
-    ms = reduce_max(t_start.elapsed_time(t_end), dev) / args.steps
+    ms = reduce_max(t_start.elapsed_time(t_end), dev) / steps
     layout_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["l0"], ev["l1"]))
     dispatch_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["l1"], ev["d1"]))
     combine_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["d1"], ev["c1"]))
     value = world * step_bytes / (ms * 1e-3) / 1e9
 
+    kernels_ms = ({"layout_dispatch": layout_ms + dispatch_ms, "combine": combine_ms} if one_call else
+                  {"layout": layout_ms, "dispatch": dispatch_ms, "combine": combine_ms})
+    rec = {"value": value, "ms_per_step": ms, "steps": steps, "warmup": warmup, "cap": cap,
+           "window": (w0, w1), "launches": launches, "nb": nb, "valid_pairs": valid_pairs, "pad_rows": pad_rows,
+           "rows": rows, "kernels_ms": kernels_ms, "one_call": one_call}
     # end to end through the public API: pinned host inputs -> device, round trip, result -> host
-    e2e = None if args.no_e2e else run_e2e(args, world, dev, stream, step, step_bytes, x, idx, w, y, bias, out,
-                                           x_c, idx_c, w_c, bias_c)
+    rec["e2e"] = run_e2e(args, world, dev, stream, step, step_bytes, x, idx, w, y, bias, out, x_c, idx_c, w_c,
+                         bias_c) if want_e2e else None
     extras = {}
-    if args.expert_gemm:
+    if args.expert_gemm and want_e2e:
         if not wl.fp8 or wl.alignment % 128 or wl.hidden % 128 or args.expert_gemm % 128:
             raise SystemExit("--expert-gemm needs an FP8 workload, expert_alignment and N multiples of 128")
         hg = moe.moe_layout(make_params(cap), idx, w, stream=stream)
         extras["expert_gemm"] = expert_gemm_measurement(moe, wl, hg, x, cap, args.expert_gemm, stream, dev)
         moe.moe_handle_free(hg)
     if wl.name == "decode":
-        extras["latency"] = decode_latency(step_parts, stream, dev)
+        extras["latency"] = decode_latency(step_parts, stream, dev, one_call)
     if wl.name == "skewed":
         extras["overlap"] = skewed_overlap(step, stream, dev)
         extras["rows_per_rank"] = {"max": int(rows.max()), "mean": float(rows.mean()), "min": int(rows.min())}
+    rec["extras"] = extras
+
     peak, peak_kind = hbm_peak()
-    kern = {"dispatch": (dispatch_ms, nb["dispatch"]), "combine": (combine_ms, nb["combine"])}
+    kern = {("layout_dispatch" if one_call else "dispatch"): (kernels_ms.get("layout_dispatch", dispatch_ms),
+                                                              nb["dispatch"]),
+            "combine": (combine_ms, nb["combine"])}
     dom = max(kern, key=lambda k: kern[k][0])
     achieved = kern[dom][1] / (kern[dom][0] * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "kernel": f"k_{dom}", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
-                if peak_kind == "measured" else "fallback 6.65 TB/s",
-                "algorithmic_bytes_per_launch": kern[dom][1],
-                "traffic": measured_traffic(dom, args.workload)}
+    rec["peak"] = peak
+    rec["roofline"] = {"bound": "hbm", "kernel": f"k_{dom}", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                       "frac": achieved / peak,
+                       "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                       if peak_kind == "measured" else "fallback 6.65 TB/s",
+                       "algorithmic_bytes_per_launch": kern[dom][1],
+                       "traffic": measured_traffic(dom, wl.name) if dom in KERNEL_SOURCES else None}
 
     cpu = None
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        run = oracle_sample(wl, args.cpu_tokens)
+    if world == 1 and rank == 0 and cpu_tokens > 0:
+        run = oracle_sample(wl, cpu_tokens)
         passes = [run() for _ in range(3)]
         dt, cb, desc = min(passes)
         cpu = {"value": cb / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": desc + "; best of 3 passes", "host": host_cpu()}
+    rec["cpu_baseline"] = cpu
+    del recv, scales, y, out, x, idx, w, bias
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
+def side_record(wl: W.Workload, rec: dict, clk: ClockSampler) -> dict:
+    """The compact record of a configuration measured beside the headline one."""
+    k = rec["kernels_ms"]
+    nb = rec["nb"]
+    out = {"value": rec["value"], "unit": UNIT, "us_per_step": rec["ms_per_step"] * 1e3, "steps": rec["steps"],
+           "warmup": rec["warmup"], "frac_of_hbm_peak": rec["value"] / rec["peak"],
+           "kernels_us": {key: val * 1e3 for key, val in k.items()},
+           "kernels_gbs": {("layout_dispatch" if rec["one_call"] else "dispatch"):
+                           nb["dispatch"] / k["layout_dispatch" if rec["one_call"] else "dispatch"] / 1e6,
+                           "combine": nb["combine"] / k["combine"] / 1e6},
+           "bytes_per_step": nb, "valid_rows": rec["valid_pairs"], "padding_rows": rec["pad_rows"],
+           "rows_per_rank_max_over_mean": float(rec["rows"].max() / max(rec["rows"].mean(), 1e-9)),
+           "roofline": rec["roofline"], "cpu_baseline": rec["cpu_baseline"],
+           "clocks": clk.summary(*rec["window"]), "timed_window_unix_s": [round(v, 3) for v in rec["window"]],
+           "config": workload_config(wl, rec["cap"]), **rec["extras"]}
+    return out
+
+
+def run_ours(args) -> int:
+    world, rank, local = dist_setup("nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import combine_moe_layout_07_b200 as moe
+
+    wl = W.WORKLOADS[args.workload]
+    if args.tokens_per_rank:
+        wl = wl.with_(tokens_per_rank=args.tokens_per_rank)
+    stream = torch.cuda.current_stream()
+    clk = ClockSampler(local).start()
+    rec = measure_workload(moe, wl, args, world, rank, dev, stream, clk, args.steps, args.warmup,
+                           0 if args.no_cpu_baseline else args.cpu_tokens, want_e2e=not args.no_e2e)
+    side = {}
+    if not args.no_side_workloads:
+        for name, spec in SIDE_WORKLOADS.items():
+            if name == wl.name:
+                continue
+            swl = W.WORKLOADS[name]
+            srec = measure_workload(moe, swl, args, world, rank, dev, stream, clk, spec["steps"],
+                                    max(3, args.warmup), 0 if args.no_cpu_baseline else spec["cpu_tokens"],
+                                    want_e2e=False)
+            side[name] = srec
+    clk.stop(args.clock_log)
+    clk.t0, clk.t1 = rec["window"]
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        nb, k = rec["nb"], rec["kernels_ms"]
+        rows, peak = rec["rows"], rec["peak"]
+        line = {"metric": METRIC, "value": rec["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "data_types": {"x": "bf16", "recv": "e4m3 + f32 scales" if wl.fp8 else "bf16", "y,out": "bf16"},
-                "config": workload_config(wl, cap, {"parallelism": f"{world} independent replica(s), "
-                                                                   f"{wl.ranks} logical EP ranks each"}),
-                "frac_of_hbm_peak": value / world / peak,
-                "frac_of_8tbs_nominal": value / world / 8000.0,
-                "kernels_ms": {"layout": layout_ms, "dispatch": dispatch_ms, "combine": combine_ms},
-                "kernels_gbs": {"dispatch": nb["dispatch"] / dispatch_ms / 1e6, "combine": nb["combine"] / combine_ms / 1e6},
-                "bytes_per_step": nb, "valid_rows": valid_pairs, "padding_rows": pad_rows,
-                "A_pad": (valid_pairs + pad_rows) / max(valid_pairs, 1),
+                "config": workload_config(wl, rec["cap"], {"parallelism": f"{world} independent replica(s), "
+                                                                          f"{wl.ranks} logical EP ranks each"}),
+                "frac_of_hbm_peak": rec["value"] / world / peak,
+                "frac_of_8tbs_nominal": rec["value"] / world / 8000.0,
+                "kernels_ms": k,
+                "kernels_gbs": {("layout_dispatch" if rec["one_call"] else "dispatch"):
+                                nb["dispatch"] / k["layout_dispatch" if rec["one_call"] else "dispatch"] / 1e6,
+                                "combine": nb["combine"] / k["combine"] / 1e6},
+                "bytes_per_step": nb, "valid_rows": rec["valid_pairs"], "padding_rows": rec["pad_rows"],
+                "A_pad": (rec["valid_pairs"] + rec["pad_rows"]) / max(rec["valid_pairs"], 1),
                 "rows_per_rank_max_over_mean": float(rows.max() / max(rows.mean(), 1e-9)),
-                "roofline": roofline, "cpu_baseline": cpu,
-                "e2e": e2e,
-                "gpu_launches": launches, "clocks": clk.summary(),
-                "library": os.path.relpath(moe.library_path(), ROOT), **extras}
+                "roofline": rec["roofline"], "cpu_baseline": rec["cpu_baseline"],
+                "e2e": rec["e2e"],
+                "gpu_launches": rec["launches"], "clocks": clk.summary(*rec["window"]),
+                "library": os.path.relpath(moe.library_path(), ROOT), **rec["extras"]}
+        if side:
+            line["workloads"] = {WORKLOAD_NAMES[name]: side_record(W.WORKLOADS[name], srec, clk)
+                                 for name, srec in side.items()}
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized():
@@ -641,6 +741,9 @@ def main() -> int:
     ap.add_argument("--expert-gemm", type=int, default=0, metavar="N",
                     help="also time the first expert GEMM (E4M3, K = hidden, N output columns) on the dispatch output")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--clock-log", default=None, metavar="FILE", help="write the raw nvidia-smi clock samples to FILE")
+    ap.add_argument("--no-side-workloads", action="store_true",
+                    help="measure only the headline workload (not decode, large and skewed beside it)")
     ap.add_argument("--tokens-per-rank", type=int, default=0, help="override the workload's tokens per rank "
                     "(smaller cases for profiling)")
     args = ap.parse_args()

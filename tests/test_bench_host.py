@@ -75,3 +75,17 @@ def test_clock_summary_without_samples():
     c.out = ""
     s = c.summary()
     assert s["samples"] == 0 and s["reasons"] == ["unavailable"]
+
+
+def test_clock_summary_falls_back_to_the_nearest_samples():
+    c = bench.ClockSampler(0)
+    t0 = 1_700_000_000.0
+    lines = [_sample_line(t0 + 0.1 * i, 1000 + i) for i in range(10)]          # a gap after t0 + 0.9
+    lines += [_sample_line(t0 + 5.0, 1900), _sample_line(t0 + 5.1, 1901, ("Active",) + ("Not Active",) * 3)]
+    c.out = "\n".join(lines)
+    s = c.summary(t0 + 2.0, t0 + 2.1)                   # nothing inside: t0 + 0.9 and t0 + 0.8 are nearest
+    assert s["samples"] == 2 and s["window"].startswith("nearest")
+    assert s["sm_mhz"] == float(np.median([1009, 1008]))
+    assert s["reasons"] == []
+    s = c.summary(t0 + 4.0, t0 + 4.1)                   # t0 + 5.0 and t0 + 5.1, one with hw_slowdown
+    assert s["sm_mhz"] == float(np.median([1900, 1901])) and s["reasons"] == ["hw_slowdown"]
