@@ -153,31 +153,49 @@ struct ThreadGroup {
 
 __device__ __forceinline__ ThreadGroup whole_cta() { return ThreadGroup{(int)threadIdx.x, (int)blockDim.x, 0}; }
 
-// Exclusive scan of one value per thread of the group (warp shuffles + one smem pass).
-__device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_tot, int32_t* total,
-                                                        const ThreadGroup& g) {
+// Exclusive scans of two values per thread of the group at once (warp shuffles + one smem pass);
+// warp_tot holds 2 x 32 entries, total 2.  Returns the two exclusive prefixes.
+__device__ __forceinline__ int2 block_exclusive_scan2(int32_t v0, int32_t v1, int32_t* warp_tot, int32_t* total,
+                                                      const ThreadGroup& g) {
   const int lane = g.tid & 31, warp = g.tid >> 5, nwarps = g.n >> 5;
-  int32_t incl = v;
+  int32_t a = v0, b = v1;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int32_t n = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += n;
+    const int32_t na = __shfl_up_sync(0xffffffffu, a, o);
+    const int32_t nb = __shfl_up_sync(0xffffffffu, b, o);
+    if (lane >= o) {
+      a += na;
+      b += nb;
+    }
   }
-  if (lane == 31) warp_tot[warp] = incl;
+  if (lane == 31) {
+    warp_tot[warp] = a;
+    warp_tot[32 + warp] = b;
+  }
   g.sync();
   if (warp == 0) {
-    int32_t w = lane < nwarps ? warp_tot[lane] : 0;
-    int32_t wi = w;
+    const int32_t wa = lane < nwarps ? warp_tot[lane] : 0, wb = lane < nwarps ? warp_tot[32 + lane] : 0;
+    int32_t ia = wa, ib = wb;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int32_t n = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += n;
+      const int32_t na = __shfl_up_sync(0xffffffffu, ia, o);
+      const int32_t nb = __shfl_up_sync(0xffffffffu, ib, o);
+      if (lane >= o) {
+        ia += na;
+        ib += nb;
+      }
     }
-    if (lane < nwarps) warp_tot[lane] = wi - w;  // exclusive warp offsets
-    if (lane == 31) *total = wi;
+    if (lane < nwarps) {  // exclusive warp offsets
+      warp_tot[lane] = ia - wa;
+      warp_tot[32 + lane] = ib - wb;
+    }
+    if (lane == 31) {
+      total[0] = ia;
+      total[1] = ib;
+    }
   }
   g.sync();
-  const int32_t r = warp_tot[warp] + incl - v;
+  const int2 r = make_int2(warp_tot[warp] + a - v0, warp_tot[32 + warp] + b - v1);
   g.sync();
   return r;
 }
@@ -191,7 +209,7 @@ template <bool kCntGlobal>
 __device__ __forceinline__ void block_psum(const LayoutLaunch& L, const int32_t* cnt, int64_t cap_check, int32_t* al,
                                            int32_t* pad, int32_t* gincl, int32_t* pad_s, int32_t* psum_s,
                                            bool publish, const ThreadGroup& g) {
-  __shared__ int32_t warp_tot[32];
+  __shared__ int32_t warp_tot[64];
   __shared__ int32_t totals[2];
   const int E = L.E, tid = g.tid;
   for (int x = tid; x < E; x += g.n) {
@@ -207,8 +225,8 @@ __device__ __forceinline__ void block_psum(const LayoutLaunch& L, const int32_t*
     sa += al[x];
     sp += pad[x];
   }
-  int32_t ra = block_exclusive_scan(sa, warp_tot, &totals[0], g);
-  int32_t rp = block_exclusive_scan(sp, warp_tot, &totals[1], g);
+  const int2 rr = block_exclusive_scan2(sa, sp, warp_tot, totals, g);
+  int32_t ra = rr.x, rp = rr.y;
   for (int x = e0; x < e1; ++x) {
     if (publish) L.d.pad_excl[x] = rp;
     if (pad_s) pad_s[x] = rp;
