@@ -25,10 +25,12 @@
 //               tile of weights (128-byte swizzle) into a ring of stages (full/empty mbarriers);
 //   warp 1      allocates all 512 tensor-memory columns; one lane issues the MMAs and commits
 //               them to the stage's empty barrier and to the accumulator's full barrier;
-//   warps 2..9  epilogue: warp w reads tensor-memory lanes 32 * (w % 4) .. (one output row per
-//               thread) and half (w - 2) / 4 of the tile's kN columns (kN / 2 accumulators per
-//               thread): per K-block, 32-column loads in rounds of kRoundCols with one wait per
-//               round, then the promotions; a bf16 store of its kN / 2 columns per tile.
+//   warps 2, 3  set-up only (row tiles per rank, psum into shared memory);
+//   warps 4..11 epilogue (warpgroups 1 and 2, which take the registers warpgroup 0 gives back):
+//               warp w reads tensor-memory lanes 32 * (w % 4) .. (one output row per thread) and
+//               half (w - 4) / 4 of the tile's kN columns (kN / 2 accumulators per thread): per
+//               K-block, 32-column loads in rounds of kRoundCols with one wait per round, then
+//               the promotions; a bf16 store of its kN / 2 columns per tile.
 // Every wait is an mbarrier wait bounded by wall-clock time (status kStatusTimeout).  No TMA
 // load here uses cluster multicast.
 #include <cuda.h>
@@ -39,7 +41,15 @@ namespace moe {
 
 constexpr int kGemmM = 128;                            // rows of a tile = the K-block width
 constexpr int kGemmEpiWarps = 8;                       // two per tensor-memory lane quarter
-constexpr int kGemmThreads = 64 + 32 * kGemmEpiWarps;  // producer, MMA, epilogue warps
+constexpr int kGemmEpiWarp0 = 4;                       // the epilogue is warpgroups 1 and 2
+constexpr int kGemmThreads = 128 + 32 * kGemmEpiWarps;  // warpgroup 0 (producer, MMA, set-up), epilogue
+// Register split (setmaxnreg): warpgroup 0 gives registers back, the epilogue warpgroups take them
+// for their 128 accumulators per thread.  The launch holds kGemmThreads x (registers at launch);
+// the split needs 128 x kGemmCtlRegs + 256 x kGemmEpiRegs of them, which the host checks against
+// the kernel's register count before it launches.
+constexpr int kGemmCtlRegs = 112;
+constexpr int kGemmEpiRegs = 192;
+static_assert(kGemmCtlRegs % 8 == 0 && kGemmEpiRegs % 8 == 0, "setmaxnreg counts are multiples of 8");
 constexpr uint32_t kGemmTmemCols = 512;                // all of tensor memory (one CTA per SM)
 constexpr uint32_t kGemmStageBudget = 192 * 1024;      // shared memory for the operand ring
 
@@ -244,73 +254,77 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int64_t n_tiles = (int64_t)tiles[L.R] * NT;
   const int KB = L.KB;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
-      int64_t g = 0;
-      bool ok = true;
-      for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const GemmTile tl = gemm_tile(L.R, L.E_loc, NT, tiles, psum_s, t);
-        const int32_t y_rows = (int32_t)((int64_t)tl.r * L.cap + tl.row0);
-        const int32_t y_cols = (int32_t)((int64_t)tl.e * L.N + (int64_t)tl.nb * kN);
-        for (int kb = 0; kb < KB; ++kb, ++g) {
-          if (g >= C::kStages && !(ok = mbar_wait(empty0 + 8 * s, ph ^ 1u, L.status))) break;
-          const uint32_t a = base + lay.stage0 + (uint32_t)s * C::kStageBytes;
-          mbar_arrive_expect_tx(full0 + 8 * s, C::kStageBytes);
-          tma_load_2d(a, &map_x, kb * 128, y_rows, full0 + 8 * s);
-          tma_load_2d(a + C::kBytesA, &map_w, kb * 128, y_cols, full0 + 8 * s);
-          if (++s == C::kStages) {
-            s = 0;
-            ph ^= 1u;
+  if (warp < kGemmEpiWarp0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kGemmCtlRegs));
+    if (warp == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        int s = 0;
+        uint32_t ph = 0;
+        int64_t g = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+          const GemmTile tl = gemm_tile(L.R, L.E_loc, NT, tiles, psum_s, t);
+          const int32_t y_rows = (int32_t)((int64_t)tl.r * L.cap + tl.row0);
+          const int32_t y_cols = (int32_t)((int64_t)tl.e * L.N + (int64_t)tl.nb * kN);
+          for (int kb = 0; kb < KB; ++kb, ++g) {
+            if (g >= C::kStages && !(ok = mbar_wait(empty0 + 8 * s, ph ^ 1u, L.status))) break;
+            const uint32_t a = base + lay.stage0 + (uint32_t)s * C::kStageBytes;
+            mbar_arrive_expect_tx(full0 + 8 * s, C::kStageBytes);
+            tma_load_2d(a, &map_x, kb * 128, y_rows, full0 + 8 * s);
+            tma_load_2d(a + C::kBytesA, &map_w, kb * 128, y_cols, full0 + 8 * s);
+            if (++s == C::kStages) {
+              s = 0;
+              ph ^= 1u;
+            }
           }
         }
-      }
-      // no load may still be landing when the CTA exits: the last stages must have filled
-      for (int64_t j = 0; j < (g < C::kStages ? g : C::kStages); ++j) {
-        if (--s < 0) {
-          s = C::kStages - 1;
-          ph ^= 1u;
-        }
-        mbar_wait(full0 + 8 * s, ph, L.status);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
-      int64_t g = 0;
-      bool ok = true;
-      for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        for (int kb = 0; kb < KB; ++kb, ++g) {
-          const int b = (int)(g % C::kAccBufs);
-          const uint32_t tph = (uint32_t)((g / C::kAccBufs) & 1);
-          if (!(ok = mbar_wait(full0 + 8 * s, ph, L.status))) break;
-          if (g >= C::kAccBufs && !(ok = mbar_wait(tempty0 + 8 * b, tph ^ 1u, L.status))) break;
-          tc_fence_after();
-          const uint32_t a = base + lay.stage0 + (uint32_t)s * C::kStageBytes;
-          const uint64_t ad = kmajor_sw128_desc(a), bd = kmajor_sw128_desc(a + C::kBytesA);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)  // K = 32 E4M3 = 32 bytes = 2 descriptor units per step
-            mma_e4m3(tmem + (uint32_t)(b * kN), ad + 2 * k, bd + 2 * k, C::kIdesc, k > 0 ? 1u : 0u);
-          mma_commit(empty0 + 8 * s);  // the stage is free once these MMAs have read it
-          mma_commit(tfull0 + 8 * b);  // the accumulator is ready for the epilogue
-          if (++s == C::kStages) {
-            s = 0;
+        // no load may still be landing when the CTA exits: the last stages must have filled
+        for (int64_t j = 0; j < (g < C::kStages ? g : C::kStages); ++j) {
+          if (--s < 0) {
+            s = C::kStages - 1;
             ph ^= 1u;
           }
+          mbar_wait(full0 + 8 * s, ph, L.status);
         }
       }
-      mma_commit(done);  // every MMA of this CTA has completed when `done` flips
-      mbar_wait(done, 0, L.status);
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        int s = 0;
+        uint32_t ph = 0;
+        int64_t g = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+          for (int kb = 0; kb < KB; ++kb, ++g) {
+            const int b = (int)(g % C::kAccBufs);
+            const uint32_t tph = (uint32_t)((g / C::kAccBufs) & 1);
+            if (!(ok = mbar_wait(full0 + 8 * s, ph, L.status))) break;
+            if (g >= C::kAccBufs && !(ok = mbar_wait(tempty0 + 8 * b, tph ^ 1u, L.status))) break;
+            tc_fence_after();
+            const uint32_t a = base + lay.stage0 + (uint32_t)s * C::kStageBytes;
+            const uint64_t ad = kmajor_sw128_desc(a), bd = kmajor_sw128_desc(a + C::kBytesA);
+  #pragma unroll
+            for (int k = 0; k < 4; ++k)  // K = 32 E4M3 = 32 bytes = 2 descriptor units per step
+              mma_e4m3(tmem + (uint32_t)(b * kN), ad + 2 * k, bd + 2 * k, C::kIdesc, k > 0 ? 1u : 0u);
+            mma_commit(empty0 + 8 * s);  // the stage is free once these MMAs have read it
+            mma_commit(tfull0 + 8 * b);  // the accumulator is ready for the epilogue
+            if (++s == C::kStages) {
+              s = 0;
+              ph ^= 1u;
+            }
+          }
+        }
+        mma_commit(done);  // every MMA of this CTA has completed when `done` flips
+        mbar_wait(done, 0, L.status);
+      }
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kGemmEpiRegs));
     // ------------------------------------------------------------------ epilogue
     constexpr int W = C::kWarpCols;
     const int q = warp & 3;                       // tensor-memory lane quarter of this warp
-    const int col0 = ((warp - 2) >> 2) * W;       // the half of the tile's columns it owns
+    const int col0 = ((warp - kGemmEpiWarp0) >> 2) * W;  // the half of the tile's columns it owns
     const int my_row = q * 32 + lane;             // row of the tile this thread owns
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     uint16_t* out = static_cast<uint16_t*>(L.out);
@@ -435,6 +449,12 @@ static cudaError_t launch_gemm_n(const GemmLaunch& L, const void* x, const void*
   static unsigned long long done = 0;
   cudaError_t err = set_smem_limit_once(k_expert_gemm<kN>, 227 * 1024, &done);
   if (err != cudaSuccess) return err;
+  // the register split must fit the registers the launch holds (else setmaxnreg.inc would wait)
+  cudaFuncAttributes fa{};
+  err = cudaFuncGetAttributes(&fa, k_expert_gemm<kN>);
+  if (err != cudaSuccess) return err;
+  if ((int64_t)fa.numRegs * kGemmThreads < 128 * kGemmCtlRegs + 32 * kGemmEpiWarps * kGemmEpiRegs)
+    return cudaErrorInvalidConfiguration;
   err = launch_pdl(k_expert_gemm<kN>, dim3(L.grid), dim3(kGemmThreads), smem, st, mx, mw, L);
   note_launch();
   return err;
