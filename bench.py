@@ -498,7 +498,7 @@ SIDE_WORKLOADS = {"decode": {"steps": 4000, "cpu_tokens": 1024},
 
 
 def measure_workload(moe, wl: W.Workload, args, world: int, rank: int, dev, stream, clk: ClockSampler,
-                     steps: int, warmup: int, cpu_tokens: int, want_e2e: bool) -> dict:
+                     steps: int, warmup: int, cpu_tokens: int, want_e2e: bool, headline: bool) -> dict:
     """Times `steps` round trips (layout -> dispatch -> combine -> handle free) of one workload
     after `warmup` untimed ones, bracketed by barrier + synchronize, max over ranks; returns the
     measurement with its per-kernel times, roofline, clocks, CPU-oracle baseline (rank 0, one
@@ -610,7 +610,7 @@ def measure_workload(moe, wl: W.Workload, args, world: int, rank: int, dev, stre
     rec["e2e"] = run_e2e(args, world, dev, stream, step, step_bytes, x, idx, w, y, bias, out, x_c, idx_c, w_c,
                          bias_c) if want_e2e else None
     extras = {}
-    if args.expert_gemm and want_e2e:
+    if args.expert_gemm and headline:
         if not wl.fp8 or wl.alignment % 128 or wl.hidden % 128 or args.expert_gemm % 128:
             raise SystemExit("--expert-gemm needs an FP8 workload, expert_alignment and N multiples of 128")
         hg = moe.moe_layout(make_params(cap), idx, w, stream=stream)
@@ -681,7 +681,7 @@ def run_ours(args) -> int:
     stream = torch.cuda.current_stream()
     clk = ClockSampler(local).start()
     rec = measure_workload(moe, wl, args, world, rank, dev, stream, clk, args.steps, args.warmup,
-                           0 if args.no_cpu_baseline else args.cpu_tokens, want_e2e=not args.no_e2e)
+                           0 if args.no_cpu_baseline else args.cpu_tokens, want_e2e=not args.no_e2e, headline=True)
     side = {}
     if not args.no_side_workloads:
         for name, spec in SIDE_WORKLOADS.items():
@@ -690,7 +690,7 @@ def run_ours(args) -> int:
             swl = W.WORKLOADS[name]
             srec = measure_workload(moe, swl, args, world, rank, dev, stream, clk, spec["steps"],
                                     max(3, args.warmup), 0 if args.no_cpu_baseline else spec["cpu_tokens"],
-                                    want_e2e=False)
+                                    want_e2e=False, headline=False)
             side[name] = srec
     clk.stop(args.clock_log)
     clk.t0, clk.t1 = rec["window"]

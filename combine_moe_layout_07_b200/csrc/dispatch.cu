@@ -74,16 +74,45 @@ __host__ __device__ inline DispSmem disp_smem(int64_t H, int stages) {
   return s;
 }
 
-// Reads of the layout's arrays go through L2 (ld.global.cg): the one-launch layout + dispatch
-// kernel reads them in the same launch that wrote them, after its grid barrier.
-__device__ __forceinline__ int find_padding_expert(const int32_t* pad_excl, int E, int32_t i) {
-  int lo = 0, hi = E;  // largest e with pad_excl[e] <= i
+// A walk over the padding rows of all experts in increasing index i (0 <= i < pad_excl[E], the
+// padding prefix over experts): one binary search for the first row, then a step per expert
+// crossed.  kCoherent reads the layout's arrays through L2 (ld.global.cg), for the one-launch
+// layout + dispatch kernel that reads them in the launch that wrote them; otherwise through L1.
+struct PadCursor {
+  int e;                     // expert of the current row
+  int32_t begin, end, last;  // pad_excl[e], pad_excl[e + 1], psum[e]
+};
+
+template <bool kCoherent>
+__device__ __forceinline__ int32_t ld_layout(const int32_t* p) {
+  if constexpr (kCoherent) return __ldcg(p);
+  else return __ldg(p);
+}
+
+template <bool kCoherent>
+__device__ __forceinline__ PadCursor pad_seek(const DispatchLaunch& L, int32_t i) {
+  int lo = 0, hi = L.E;  // largest e with pad_excl[e] <= i
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (__ldcg(pad_excl + mid) <= i) lo = mid;
+    if (ld_layout<kCoherent>(L.pad_excl + mid) <= i) lo = mid;
     else hi = mid;
   }
-  return lo;
+  return PadCursor{lo, ld_layout<kCoherent>(L.pad_excl + lo), ld_layout<kCoherent>(L.pad_excl + lo + 1),
+                   ld_layout<kCoherent>(L.psum + lo)};
+}
+
+// Receive-buffer row (rank * cap + row) of padding row i, at or after the cursor's row; -1 when it
+// lies at or beyond cap.  Expert e's padding rows are [psum[e] - pad_e, psum[e]) of its rank.
+template <bool kCoherent>
+__device__ __forceinline__ int64_t pad_row(const DispatchLaunch& L, PadCursor& c, int32_t i) {
+  while (i >= c.end) {
+    ++c.e;
+    c.begin = c.end;
+    c.end = ld_layout<kCoherent>(L.pad_excl + c.e + 1);
+    c.last = ld_layout<kCoherent>(L.psum + c.e);
+  }
+  const int32_t row = c.last - (c.end - c.begin) + (i - c.begin);
+  return row < L.cap ? (int64_t)(c.e / L.E_loc) * L.cap + row : -1;
 }
 
 // The producer warp of both dispatch kernels: pair metadata for tpb items per warp-wide load,
@@ -174,35 +203,6 @@ __device__ __forceinline__ void dispatch_producer(const DispatchLaunch& L, int S
   }
 }
 
-// Padding rows (zero_padding: zero codes and scales; recv_w: weight 0), a warp per row: warp gw of
-// nw warps in the grid takes padding rows gw, gw + nw, ...
-template <bool kFp8>
-__device__ __forceinline__ void zero_padding_rows(const DispatchLaunch& L, int64_t gw, int64_t nw, int lane,
-                                                  bool& overflow) {
-  if (!L.zero_padding && !L.recv_w) return;
-  const int64_t H = L.H, nblk = H / 128;
-  const int32_t total_pad = __ldg(L.pad_excl + L.E);
-  const int64_t row_bytes = kFp8 ? H : 2 * H;
-  for (int64_t i = gw; i < total_pad; i += nw) {
-    const int e = find_padding_expert(L.pad_excl, L.E, (int32_t)i);
-    const int32_t pad_e = __ldg(L.pad_excl + e + 1) - __ldg(L.pad_excl + e);
-    const int32_t row = __ldg(L.psum + e) - pad_e + ((int32_t)i - __ldg(L.pad_excl + e));
-    if (row >= L.cap) {
-      overflow = true;
-      continue;
-    }
-    const int64_t grow = (int64_t)(e / L.E_loc) * L.cap + row;
-    if (!dbg_ok(row >= 0 && grow < L.R * L.cap, L.status, 204, grow)) continue;
-    if (L.zero_padding) {
-      uint8_t* dst = static_cast<uint8_t*>(L.recv_x) + grow * row_bytes;
-      for (int64_t o = lane * 16; o < row_bytes; o += 32 * 16) st_stream_v4(dst + o, make_uint4(0, 0, 0, 0));
-      if (kFp8)
-        for (int64_t b = lane; b < nblk; b += 32) L.recv_scales[grow * nblk + b] = 0.0f;
-    }
-    if (L.recv_w && lane == 0) L.recv_w[grow] = 0.0f;
-  }
-}
-
 // An L2 policy that marks lines for eviction first: the receive rows are written once and read
 // only by a later kernel, so their lines go back to HBM soon after they are written, in about
 // the order the grid writes them.
@@ -218,19 +218,13 @@ __device__ __forceinline__ void bulk_store_hinted(void* dst, uint32_t src_smem, 
                : "memory");
 }
 
-// Padding row i of all experts (0 <= i < pad_excl[E]), zeroed by the nth threads gtid of a
-// group: codes or bf16 row in 16-byte stores, FP8 scales, receive weight 0.  Returns false (and
-// writes nothing) when the row lies at or beyond cap.
+// Receive-buffer row grow (a padding row), zeroed by the nth threads gtid of a group: codes or
+// bf16 row in 16-byte stores, FP8 scales, receive weight 0.
 template <bool kFp8>
-__device__ __forceinline__ bool zero_padding_row(const DispatchLaunch& L, int32_t i, int gtid, int nth) {
+__device__ __forceinline__ void zero_padding_row(const DispatchLaunch& L, int64_t grow, int gtid, int nth) {
   const int64_t H = L.H, nblk = H / 128;
   const int64_t row_bytes = kFp8 ? H : 2 * H;
-  const int e = find_padding_expert(L.pad_excl, L.E, i);
-  const int32_t pad_e = __ldcg(L.pad_excl + e + 1) - __ldcg(L.pad_excl + e);
-  const int32_t row = __ldcg(L.psum + e) - pad_e + (i - __ldcg(L.pad_excl + e));
-  if (row >= L.cap) return false;
-  const int64_t grow = (int64_t)(e / L.E_loc) * L.cap + row;
-  if (!dbg_ok(row >= 0 && grow < L.R * L.cap, L.status, 204, grow)) return true;
+  if (!dbg_ok(grow >= 0 && grow < L.R * L.cap, L.status, 204, grow)) return;
   if (L.zero_padding) {
     uint8_t* dst = static_cast<uint8_t*>(L.recv_x) + grow * row_bytes;
     for (int64_t o = (int64_t)gtid * 16; o < row_bytes; o += (int64_t)nth * 16) st_stream_v4(dst + o, make_uint4(0, 0, 0, 0));
@@ -238,7 +232,23 @@ __device__ __forceinline__ bool zero_padding_row(const DispatchLaunch& L, int32_
       for (int64_t b = gtid; b < nblk; b += nth) L.recv_scales[grow * nblk + b] = 0.0f;
   }
   if (L.recv_w && gtid == 0) L.recv_w[grow] = 0.0f;
-  return true;
+}
+
+// Padding rows (zero_padding: zero codes and scales; recv_w: weight 0), a warp per row: warp gw of
+// nw warps in the grid takes the contiguous run [gw * P / nw, (gw + 1) * P / nw) of the P rows.
+template <bool kFp8>
+__device__ __forceinline__ void zero_padding_rows(const DispatchLaunch& L, int64_t gw, int64_t nw, int lane,
+                                                  bool& overflow) {
+  if (!L.zero_padding && !L.recv_w) return;
+  const int64_t P = __ldg(L.pad_excl + L.E);
+  const int32_t i0 = (int32_t)(P * gw / nw), i1 = (int32_t)(P * (gw + 1) / nw);
+  if (i0 >= i1) return;
+  PadCursor c = pad_seek<false>(L, i0);
+  for (int32_t i = i0; i < i1; ++i) {
+    const int64_t grow = pad_row<false>(L, c, i);
+    if (grow < 0) overflow = true;
+    else zero_padding_row<kFp8>(L, grow, lane, 32);
+  }
 }
 
 // FP8 E4M3 codes of the 16 bf16 values of unit u (bytes 32u .. 32u + 31) of a staged row.  Eight
@@ -499,12 +509,15 @@ __global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunc
     const int ctid = tid - 64;
     const int grp = (warp - 2) / kDispGroupWarps;
     const int gtid = ctid - grp * kDispGroupThreads;
-    // the CTA's share [pb, pe) of the padding rows; group grp zeroes rows pb + grp, pb + grp + G, ..
-    // (G groups), paced over its tokens so that they go out among the token rows
+    // the CTA's share [pb, pe) of the padding rows: FP8, group grp zeroes rows pb + grp, pb + grp +
+    // G, .. (G groups), paced over its tokens so that they go out among the token rows; BF16 (no
+    // work per token), a warp per row from the start
     const int32_t P = (L.zero_padding || L.recv_w) ? __ldg(L.pad_excl + L.E) : 0;
     const int32_t pb = (int32_t)((int64_t)P * blockIdx.x / gridDim.x);
     const int32_t pe = (int32_t)((int64_t)P * (blockIdx.x + 1) / gridDim.x);
     int32_t pn = pb + grp;
+    PadCursor pc{0, 0, 0, 0};
+    if (kFp8 && pn < pe) pc = pad_seek<false>(L, pn);
     if constexpr (kFp8) {
       // ---------------------------------------------------------------- FP8 consumers
       const int64_t nblk = H / 128, nunits = H / 16;
@@ -551,14 +564,30 @@ __global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunc
           o -= O;
           opar ^= 1u;
         }
-        for (const int64_t target = ++m * npad / ntok; pdone < target; ++pdone, pn += kDispGroups)
-          if (!zero_padding_row<kFp8>(L, pn, gtid, kDispGroupThreads)) overflow = true;
+        for (const int64_t target = ++m * npad / ntok; pdone < target; ++pdone, pn += kDispGroups) {
+          const int64_t grow = pad_row<false>(L, pc, pn);
+          if (grow < 0) overflow = true;
+          else zero_padding_row<kFp8>(L, grow, gtid, kDispGroupThreads);
+        }
+      }
+      for (; pn < pe; pn += kDispGroups) {  // the rows the pacing left
+        const int64_t grow = pad_row<false>(L, pc, pn);
+        if (grow < 0) overflow = true;
+        else zero_padding_row<kFp8>(L, grow, gtid, kDispGroupThreads);
+      }
+    } else {  // BF16: warp w of the 16 takes the contiguous run w of the CTA's share
+      const int w = ctid >> 5;
+      const int32_t i0 = pb + (int32_t)((int64_t)(pe - pb) * w / kDispConsumerWarps);
+      const int32_t i1 = pb + (int32_t)((int64_t)(pe - pb) * (w + 1) / kDispConsumerWarps);
+      if (i0 < i1) {
+        PadCursor c = pad_seek<false>(L, i0);
+        for (int32_t i = i0; i < i1; ++i) {
+          const int64_t grow = pad_row<false>(L, c, i);
+          if (grow < 0) overflow = true;
+          else zero_padding_row<kFp8>(L, grow, lane, 32);
+        }
       }
     }
-    // BF16 (nothing to compute per token): every padding row of the group from the start; FP8: the
-    // rows the pacing left
-    for (; pn < pe; pn += kDispGroups)
-      if (!zero_padding_row<kFp8>(L, pn, gtid, kDispGroupThreads)) overflow = true;
   }
   if (overflow) atomicOr(L.status, kStatusCapacity);
 }
@@ -734,8 +763,17 @@ __global__ void __launch_bounds__(kLdThreads, 1)
         const int32_t total = __ldcg(L.pad_excl + L.E);
         const int32_t pb = (int32_t)((int64_t)total * blockIdx.x / gridDim.x);
         const int32_t pe = (int32_t)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
-        for (int32_t r = pb + (warp - 2); r < pe; r += kLayoutWarps)  // a warp per row
-          if (!zero_padding_row<kFp8>(L, r, lane, 32)) overflow = true;
+        const int w = warp - 2;  // warp w of the 8 takes the contiguous run w of the CTA's share
+        const int32_t i0 = pb + (int32_t)((int64_t)(pe - pb) * w / kLayoutWarps);
+        const int32_t i1 = pb + (int32_t)((int64_t)(pe - pb) * (w + 1) / kLayoutWarps);
+        if (i0 < i1) {
+          PadCursor c = pad_seek<true>(L, i0);
+          for (int32_t i = i0; i < i1; ++i) {
+            const int64_t grow = pad_row<true>(L, c, i);
+            if (grow < 0) overflow = true;
+            else zero_padding_row<kFp8>(L, grow, lane, 32);
+          }
+        }
       }
     }
   } else if (kFp8) {
