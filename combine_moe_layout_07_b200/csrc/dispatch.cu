@@ -236,6 +236,35 @@ __device__ __forceinline__ void zero_padding_row(const DispatchLaunch& L, int64_
 
 // Padding rows (zero_padding: zero codes and scales; recv_w: weight 0), a warp per row: warp gw of
 // nw warps in the grid takes the contiguous run [gw * P / nw, (gw + 1) * P / nw) of the P rows.
+// A block of zero bytes in shared memory from which padding rows are written by bulk (TMA)
+// stores: one instruction per kZeroBytes instead of a 16-byte store per thread and step.
+constexpr uint32_t kZeroBytes = 4096;
+
+// Receive-buffer row grow (a padding row), zeroed by one warp: lane 0 issues bulk stores of the
+// zero block for the codes or bf16 row and, when the scale row is 16-byte aligned, for the FP8
+// scales (else the lanes store them), writes the receive weight 0, and commits one bulk group.
+// The zero block stays unchanged, so the stores need no wait until the CTA exits.
+template <bool kFp8>
+__device__ __forceinline__ void zero_padding_row_bulk(const DispatchLaunch& L, int64_t grow, uint32_t zero_smem,
+                                                      int lane) {
+  const int64_t H = L.H, nblk = H / 128;
+  const int64_t row_bytes = kFp8 ? H : 2 * H;
+  if (!dbg_ok(grow >= 0 && grow < L.R * L.cap, L.status, 204, grow)) return;
+  const bool bulk_scales = kFp8 && (nblk % 4) == 0 && (reinterpret_cast<uintptr_t>(L.recv_scales) & 15) == 0;
+  if (L.zero_padding) {
+    if (lane == 0) {
+      uint8_t* dst = static_cast<uint8_t*>(L.recv_x) + grow * row_bytes;
+      for (int64_t o = 0; o < row_bytes; o += kZeroBytes)
+        bulk_store(dst + o, zero_smem, (uint32_t)min((int64_t)kZeroBytes, row_bytes - o));
+      if (bulk_scales) bulk_store(L.recv_scales + grow * nblk, zero_smem, (uint32_t)(4 * nblk));
+      bulk_commit();
+    }
+    if (kFp8 && !bulk_scales)
+      for (int64_t b = lane; b < nblk; b += 32) L.recv_scales[grow * nblk + b] = 0.0f;
+  }
+  if (L.recv_w && lane == 0) L.recv_w[grow] = 0.0f;
+}
+
 template <bool kFp8>
 __device__ __forceinline__ void zero_padding_rows(const DispatchLaunch& L, int64_t gw, int64_t nw, int lane,
                                                   bool& overflow) {
@@ -403,7 +432,7 @@ constexpr int kBulkOut = 8;     // FP8 output stages, a multiple of the consumer
 constexpr int kBulkLag = 2;     // bulk groups a storer lane leaves reading shared memory
 
 struct BulkSmem {
-  uint32_t full, empty, ofull, oempty, meta, in, out, total;
+  uint32_t full, empty, ofull, oempty, meta, in, out, zero, total;
 };
 
 __host__ __device__ inline BulkSmem bulk_smem(int64_t H, bool fp8, int S) {
@@ -426,6 +455,9 @@ __host__ __device__ inline BulkSmem bulk_smem(int64_t H, bool fp8, int S) {
   off += (uint32_t)(2 * H) * S;
   b.out = off;
   off += (uint32_t)H * O;
+  off = round_to(off, 128);
+  b.zero = off;
+  off += kZeroBytes;
   b.total = off;
   return b;
 }
@@ -455,6 +487,8 @@ __global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunc
     }
     fence_mbar_init();
   }
+  for (uint32_t o = (uint32_t)tid * 16; o < kZeroBytes; o += kBulkThreads * 16) sts_v4(base + lay.zero + o, make_uint4(0, 0, 0, 0));
+  fence_proxy_async_smem();  // the zero block is read by the bulk engine (async proxy)
   __syncthreads();
   grid_dependents_launch();
   grid_dependency_wait();  // the handle written by the layout kernels
@@ -567,13 +601,13 @@ __global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunc
         for (const int64_t target = ++m * npad / ntok; pdone < target; ++pdone, pn += kDispGroups) {
           const int64_t grow = pad_row<false>(L, pc, pn);
           if (grow < 0) overflow = true;
-          else zero_padding_row<kFp8>(L, grow, gtid, kDispGroupThreads);
+          else if (gtid < 32) zero_padding_row_bulk<kFp8>(L, grow, base + lay.zero, lane);  // the group's first warp
         }
       }
       for (; pn < pe; pn += kDispGroups) {  // the rows the pacing left
         const int64_t grow = pad_row<false>(L, pc, pn);
         if (grow < 0) overflow = true;
-        else zero_padding_row<kFp8>(L, grow, gtid, kDispGroupThreads);
+        else if (gtid < 32) zero_padding_row_bulk<kFp8>(L, grow, base + lay.zero, lane);
       }
     } else {  // BF16: warp w of the 16 takes the contiguous run w of the CTA's share
       const int w = ctid >> 5;
@@ -584,10 +618,11 @@ __global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunc
         for (int32_t i = i0; i < i1; ++i) {
           const int64_t grow = pad_row<false>(L, c, i);
           if (grow < 0) overflow = true;
-          else zero_padding_row<kFp8>(L, grow, lane, 32);
+          else zero_padding_row_bulk<kFp8>(L, grow, base + lay.zero, lane);
         }
       }
     }
+    bulk_wait_all();  // the padding rows' bulk stores read the zero block until they complete
   }
   if (overflow) atomicOr(L.status, kStatusCapacity);
 }
@@ -619,7 +654,7 @@ constexpr int kLdThreads = 576;
 constexpr int kLdLayoutBar = 1;    // named barrier of the layout warps
 
 struct LdSmem {
-  uint32_t full, qdone, mready, meta, scales, layout, in, out, total;
+  uint32_t full, qdone, mready, meta, scales, layout, in, out, zero, total;
 };
 
 __host__ __device__ inline LdSmem ld_smem(int64_t H, bool fp8, int n, int E, int R) {
@@ -638,12 +673,15 @@ __host__ __device__ inline LdSmem ld_smem(int64_t H, bool fp8, int n, int E, int
   off += fp8 ? (uint32_t)(4 * (H / 128) * n) : 0;
   off = round_to(off, 16);
   l.layout = off;
-  off += (uint32_t)fused_layout_smem(E, R);
+  off += (uint32_t)fused_layout_smem(E, R, kLayoutWarps);
   off = round_to(off, 128);
   l.in = off;
   off += (uint32_t)(2 * H) * n;
   l.out = off;
   off += fp8 ? (uint32_t)H * n : 0;
+  off = round_to(off, 128);
+  l.zero = off;
+  off += kZeroBytes;
   l.total = off;
   return l;
 }
@@ -674,6 +712,8 @@ __global__ void __launch_bounds__(kLdThreads, 1)
     }
     fence_mbar_init();
   }
+  for (uint32_t o = (uint32_t)tid * 16; o < kZeroBytes; o += kLdThreads * 16) sts_v4(base + lay.zero + o, make_uint4(0, 0, 0, 0));
+  fence_proxy_async_smem();  // the zero block is read by the bulk engine (async proxy)
   __syncthreads();
   grid_dependents_launch();
   bool overflow = false;
@@ -771,8 +811,9 @@ __global__ void __launch_bounds__(kLdThreads, 1)
           for (int32_t i = i0; i < i1; ++i) {
             const int64_t grow = pad_row<true>(L, c, i);
             if (grow < 0) overflow = true;
-            else zero_padding_row<kFp8>(L, grow, lane, 32);
+            else zero_padding_row_bulk<kFp8>(L, grow, base + lay.zero, lane);
           }
+          bulk_wait_all();  // the bulk stores read the zero block until they complete
         }
       }
     }

@@ -267,15 +267,22 @@ __global__ void __launch_bounds__(kLayoutThreads) k_layout_assign(LayoutLaunch L
 }
 
 // ------------------------------------------------------------------------------------ fused
-// The one-launch layout (layout_body.cuh, fused_layout_chunk): a CTA of 256 threads per chunk, in
-// one cooperative launch; by rank, then the token rows of the chunk, in groups of blockDim tokens
-// based at the chunk's per-rank offsets.  One launch and one global handoff instead of three
-// kernels; the results are the same.
-template <int kRounds>
-__global__ void __launch_bounds__(kLayoutThreads, 1) k_layout_fused(LayoutLaunch L, int64_t cap_check) {
+// The one-launch layout (layout_body.cuh, fused_layout_chunk): a CTA of kThreads threads per
+// chunk, in one cooperative launch; by rank, then the token rows of the chunk, in groups of
+// blockDim tokens based at the chunk's per-rank offsets.  One launch and one global handoff
+// instead of three kernels; the results are the same.  Instances: 256 threads with 8 or 16
+// register rounds of 32 pairs per warp, and 1024 threads with 4 rounds for the wide chunks of a
+// capped SM budget (32 warps take a chunk's pairs in a quarter of the rounds: the rounds' match
+// and histogram steps run one after another inside a warp).
+constexpr int kFusedWideThreads = 1024;
+constexpr int kFusedWideRounds = 4;
+constexpr int kFusedWideMaxExperts = 1024;  // 32 per-warp histograms of E counts in shared memory
+
+template <int kRounds, int kThreads>
+__global__ void __launch_bounds__(kThreads, 1) k_layout_fused(LayoutLaunch L, int64_t cap_check) {
   extern __shared__ int32_t sm[];
   __shared__ int32_t base_r[kMaxByRankRanks];
-  __shared__ int32_t wcnt[kLayoutWarps * kMaxByRankRanks];
+  __shared__ int32_t wcnt[(kThreads / 32) * kMaxByRankRanks];
   __shared__ int32_t go;
   grid_dependents_launch();
   if (!fused_layout_chunk<kRounds>(L, cap_check, blockIdx.x, gridDim.x, whole_cta(), sm, base_r, &go)) return;
@@ -389,11 +396,18 @@ static cudaError_t ensure_smem_attrs() {
     err = cudaFuncSetAttribute(k_layout_assign, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(sizeof(int32_t) * kLayoutWarps * kMaxExperts));
   if (err == cudaSuccess)
-    err = cudaFuncSetAttribute(k_layout_fused<kFusedRounds>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)fused_layout_smem(kFusedMaxExperts, kFusedMaxExperts));  // R <= E
+    err = cudaFuncSetAttribute(k_layout_fused<kFusedRounds, kLayoutThreads>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)fused_layout_smem(kFusedMaxExperts, kFusedMaxExperts, kLayoutWarps));  // R <= E
   if (err == cudaSuccess)
-    err = cudaFuncSetAttribute(k_layout_fused<kFusedMaxRounds>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)fused_layout_smem(kFusedMaxExperts, kFusedMaxExperts));
+    err = cudaFuncSetAttribute(k_layout_fused<kFusedMaxRounds, kLayoutThreads>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)fused_layout_smem(kFusedMaxExperts, kFusedMaxExperts, kLayoutWarps));
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(k_layout_fused<kFusedWideRounds, kFusedWideThreads>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)fused_layout_smem(kFusedWideMaxExperts, kFusedWideMaxExperts,
+                                                      kFusedWideThreads / 32));
   if (err == cudaSuccess && dev < 64) done |= 1ull << dev;
   return err;
 }
@@ -421,8 +435,6 @@ cudaError_t launch_layout_fused(const LayoutLaunch& L, int64_t cap_check, cudaSt
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(L.num_chunks);
-  cfg.blockDim = dim3(kLayoutThreads);
-  cfg.dynamicSmemBytes = fused_layout_smem(L.E, L.R);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
@@ -430,10 +442,23 @@ cudaError_t launch_layout_fused(const LayoutLaunch& L, int64_t cap_check, cudaSt
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   // pairs per warp: ceil(chunk * k / warps), held in rounds of 32
-  const int64_t per_warp = ((int64_t)L.chunk * L.k + kLayoutWarps - 1) / kLayoutWarps;
+  const int64_t pairs = (int64_t)L.chunk * L.k;
+  const int64_t per_warp = (pairs + kLayoutWarps - 1) / kLayoutWarps;
+  const int wide_warps = kFusedWideThreads / 32;
   if (per_warp > 32 * kFusedMaxRounds) return cudaErrorInvalidValue;
-  if (per_warp <= 32 * kFusedRounds) err = cudaLaunchKernelEx(&cfg, k_layout_fused<kFusedRounds>, L, cap_check);
-  else err = cudaLaunchKernelEx(&cfg, k_layout_fused<kFusedMaxRounds>, L, cap_check);
+  if (per_warp <= 32 * kFusedRounds) {
+    cfg.blockDim = dim3(kLayoutThreads);
+    cfg.dynamicSmemBytes = fused_layout_smem(L.E, L.R, kLayoutWarps);
+    err = cudaLaunchKernelEx(&cfg, k_layout_fused<kFusedRounds, kLayoutThreads>, L, cap_check);
+  } else if (L.E <= kFusedWideMaxExperts && (pairs + wide_warps - 1) / wide_warps <= 32 * kFusedWideRounds) {
+    cfg.blockDim = dim3(kFusedWideThreads);
+    cfg.dynamicSmemBytes = fused_layout_smem(L.E, L.R, wide_warps);
+    err = cudaLaunchKernelEx(&cfg, k_layout_fused<kFusedWideRounds, kFusedWideThreads>, L, cap_check);
+  } else {
+    cfg.blockDim = dim3(kLayoutThreads);
+    cfg.dynamicSmemBytes = fused_layout_smem(L.E, L.R, kLayoutWarps);
+    err = cudaLaunchKernelEx(&cfg, k_layout_fused<kFusedMaxRounds, kLayoutThreads>, L, cap_check);
+  }
   note_launch();
   return err;
 }

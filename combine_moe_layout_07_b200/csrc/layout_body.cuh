@@ -290,7 +290,7 @@ __device__ __forceinline__ bool wait_count_reached(const int32_t* p, int32_t tar
 
 // ------------------------------------------------------------------------------------ one launch
 // The one-launch layout, for batches of at most one chunk per SM (C chunks, every CTA that holds
-// one resident at once), chunk c by a group of kLayoutThreads threads (8 warps):
+// one resident at once), chunk c by a group of W warps (g.n = 32 W threads):
 //   1. count: each warp loads its contiguous run of the chunk's pairs into registers (at most
 //      kRounds rounds of 32) and histograms it; token membership as the count kernel; chunk
 //      counts to global memory and added atomically into the expert totals cnt; then the group
@@ -302,21 +302,21 @@ __device__ __forceinline__ bool wait_count_reached(const int32_t* p, int32_t tar
 //   3. assign: as the assign kernel for its chunk (pairs from registers), based at those offsets;
 //      padding rows of the row maps over all chunks' warps.  By rank, base_r receives the chunk's
 //      per-rank token offsets (the caller builds the token rows).
-// Shared memory: sm = fused_layout_smem(E, R) bytes; go = a shared flag.  Returns false, the same
+// Shared memory: sm = fused_layout_smem(E, R, W) bytes; go = a shared flag.  Returns false, the same
 // in every thread of the group, when the grid barrier timed out.
 constexpr int kFusedMaxRounds = 16;
 
-__host__ __device__ inline size_t fused_layout_smem(int E, int R) {
-  return sizeof(int32_t) * ((size_t)(kLayoutWarps + 7) * E + 1 + R);
+__host__ __device__ inline size_t fused_layout_smem(int E, int R, int warps) {
+  return sizeof(int32_t) * ((size_t)(warps + 7) * E + 1 + R);
 }
 
 template <int kRounds>
 __device__ __forceinline__ bool fused_layout_chunk(const LayoutLaunch& L, int64_t cap_check, int c, int C,
                                                    const ThreadGroup& g, int32_t* sm, int32_t* base_r,
                                                    int32_t* go) {
-  const int E = L.E, R = L.R, tid = g.tid, lane = tid & 31, warp = tid >> 5;
-  int32_t* whist = sm;                        // [kLayoutWarps][E]
-  int32_t* hist = whist + kLayoutWarps * E;   // [E]  expert totals
+  const int E = L.E, R = L.R, tid = g.tid, lane = tid & 31, warp = tid >> 5, W = g.n >> 5;
+  int32_t* whist = sm;                        // [W][E]  per-warp histograms, then bases
+  int32_t* hist = whist + W * E;              // [E]  expert totals
   int32_t* off = hist + E;                    // [E]  rows of each expert in the chunks before c
   int32_t* al = off + E;                      // [E]
   int32_t* pad = al + E;                      // [E]
@@ -328,7 +328,7 @@ __device__ __forceinline__ bool fused_layout_chunk(const LayoutLaunch& L, int64_
   // the warp's contiguous run of the chunk's pairs, held in registers for counting and assigning
   const int64_t t0 = (int64_t)c * L.chunk, t1 = min(L.T, t0 + L.chunk);
   const int64_t p0 = t0 * L.k, np = (t1 - t0) * L.k;
-  const int64_t per = (np + kLayoutWarps - 1) / kLayoutWarps;
+  const int64_t per = (np + W - 1) / W;
   const int64_t wp0 = p0 + min(np, warp * per), wp1 = p0 + min(np, (warp + 1) * per);
   int32_t ev[kRounds];
   float wv[kRounds];
@@ -357,7 +357,7 @@ __device__ __forceinline__ bool fused_layout_chunk(const LayoutLaunch& L, int64_
   g.sync();
   for (int e = tid; e < E; e += g.n) {
     int32_t n = 0;
-    for (int w = 0; w < kLayoutWarps; ++w) n += whist[w * E + e];
+    for (int w = 0; w < W; ++w) n += whist[w * E + e];
     L.d.chunk_cnt[(int64_t)c * E + e] = n;
     if (n) atomicAdd(L.d.cnt + e, n);  // expert totals (cleared before the launch): order-free
   }
@@ -405,7 +405,7 @@ __device__ __forceinline__ bool fused_layout_chunk(const LayoutLaunch& L, int64_
   // offset), then the warp's pairs from registers
   for (int e = tid; e < E; e += g.n) {
     int32_t base = psum_s[e] - al[e] + off[e];
-    for (int w = 0; w < kLayoutWarps; ++w) {
+    for (int w = 0; w < W; ++w) {
       const int32_t v = whist[w * E + e];
       whist[w * E + e] = base;
       base += v;
@@ -418,7 +418,7 @@ __device__ __forceinline__ bool fused_layout_chunk(const LayoutLaunch& L, int64_
     const int64_t p = wp0 + r * 32 + lane;
     if (wp0 + r * 32 < wp1) overflow |= assign_round(L, p, p < wp1, ev[r], wv[r], h);
   }
-  overflow |= row_map_padding(L, pad_s, psum_s, (int64_t)c * kLayoutWarps + warp, (int64_t)C * kLayoutWarps);
+  overflow |= row_map_padding(L, pad_s, psum_s, (int64_t)c * W + warp, (int64_t)C * W);
   if (overflow) atomicOr(L.d.status, kStatusCapacity);
   return true;
 }

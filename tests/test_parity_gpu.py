@@ -147,11 +147,13 @@ def test_fused_layout_respects_the_sm_budget():
     (16, dict(tokens_per_rank=512, ranks=16, experts=128, topk=8)),   # 512-token chunks: 4096 pairs, the limit
     (16, dict(tokens_per_rank=512, ranks=16, experts=144, topk=9)),   # 4608 pairs per chunk: three kernels
     (3, dict(tokens_per_rank=300, ranks=3, experts=12, topk=3, alignment=5)),   # chunks of 320, 320, 260 tokens
+    (16, dict(tokens_per_rank=576, ranks=8, experts=2048, topk=8, alignment=2)),  # E > 1024: 256 threads, 16 rounds
 ])
 def test_wide_chunk_layout_under_an_sm_cap(num_sms, kw):
     """Under a num_sms cap the one-launch layout takes one chunk per SM of the budget, wider than
-    256 tokens, while a warp's pairs fit its registers (16 rounds of 32); beyond that, the three
-    kernels.  Both sides, with and without host sync, every byte."""
+    256 tokens, while the chunk's pairs fit its warps' registers: 32 warps of 4 rounds of 32 pairs
+    for E <= 1024, else 8 warps of 16 rounds; beyond that, the three kernels.  Each case with and
+    without host sync, every byte."""
     wl = W.WORKLOADS["tiny"].with_(hidden=64, **kw)
     idx, w, x = inputs(wl, 0.05)
     _roundtrip_small(wl, idx, w, x, weighted=True, with_bias=True, num_sms=num_sms)
