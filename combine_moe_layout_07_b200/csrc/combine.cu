@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
       for (int64_t e = gtid * 8; e < width; e += kCombGroupThreads * 8) {
         float acc[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+        for (int v = 0; v < 8; ++v) acc[v] = 0.0f;
         int j = 0;
         for (; j + 4 <= n; j += 4) {
           uint4 d[4];
@@ -229,13 +229,13 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
             const uint32_t wd[4] = {d[u].x, d[u].y, d[u].z, d[u].w};
             const float wj = kWeighted ? meta[s].w[j + u] : 1.0f;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int v = 0; v < 4; ++v) {
               if (kWeighted) {
-                acc[2 * q] = __fmaf_rn(wj, bf16lo(wd[q]), acc[2 * q]);
-                acc[2 * q + 1] = __fmaf_rn(wj, bf16hi(wd[q]), acc[2 * q + 1]);
+                acc[2 * v] = __fmaf_rn(wj, bf16lo(wd[v]), acc[2 * v]);
+                acc[2 * v + 1] = __fmaf_rn(wj, bf16hi(wd[v]), acc[2 * v + 1]);
               } else {
-                acc[2 * q] = __fadd_rn(acc[2 * q], bf16lo(wd[q]));
-                acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16hi(wd[q]));
+                acc[2 * v] = __fadd_rn(acc[2 * v], bf16lo(wd[v]));
+                acc[2 * v + 1] = __fadd_rn(acc[2 * v + 1], bf16hi(wd[v]));
               }
             }
           }
@@ -245,13 +245,13 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
           const uint32_t wd[4] = {d.x, d.y, d.z, d.w};
           const float wj = kWeighted ? meta[s].w[j] : 1.0f;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int v = 0; v < 4; ++v) {
             if (kWeighted) {
-              acc[2 * q] = __fmaf_rn(wj, bf16lo(wd[q]), acc[2 * q]);
-              acc[2 * q + 1] = __fmaf_rn(wj, bf16hi(wd[q]), acc[2 * q + 1]);
+              acc[2 * v] = __fmaf_rn(wj, bf16lo(wd[v]), acc[2 * v]);
+              acc[2 * v + 1] = __fmaf_rn(wj, bf16hi(wd[v]), acc[2 * v + 1]);
             } else {
-              acc[2 * q] = __fadd_rn(acc[2 * q], bf16lo(wd[q]));
-              acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16hi(wd[q]));
+              acc[2 * v] = __fadd_rn(acc[2 * v], bf16lo(wd[v]));
+              acc[2 * v + 1] = __fadd_rn(acc[2 * v + 1], bf16hi(wd[v]));
             }
           }
         }
@@ -259,9 +259,9 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
           const uint4 b = lds_v4(stage + (uint32_t)L.k * slot_bytes + (uint32_t)e * 2);
           const uint32_t wb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            acc[2 * q] = __fadd_rn(acc[2 * q], bf16lo(wb[q]));
-            acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16hi(wb[q]));
+          for (int v = 0; v < 4; ++v) {
+            acc[2 * v] = __fadd_rn(acc[2 * v], bf16lo(wb[v]));
+            acc[2 * v + 1] = __fadd_rn(acc[2 * v + 1], bf16hi(wb[v]));
           }
         }
         const int64_t t = cta_token(q);
