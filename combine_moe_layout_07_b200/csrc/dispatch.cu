@@ -76,40 +76,43 @@ __host__ __device__ inline DispSmem disp_smem(int64_t H, int stages) {
 
 // A walk over the padding rows of all experts in increasing index i (0 <= i < pad_excl[E], the
 // padding prefix over experts): one binary search for the first row, then a step per expert
-// crossed.  kCoherent reads the layout's arrays through L2 (ld.global.cg), for the one-launch
-// layout + dispatch kernel that reads them in the launch that wrote them; otherwise through L1.
+// crossed.  The arrays are the handle's (global memory, read through L1) or, with kShared, a
+// CTA's own copy in shared memory (the one-launch layout + dispatch, which computes them itself).
 struct PadCursor {
   int e;                     // expert of the current row
   int32_t begin, end, last;  // pad_excl[e], pad_excl[e + 1], psum[e]
+  const int32_t* pad_excl;
+  const int32_t* psum;
 };
 
-template <bool kCoherent>
+template <bool kShared>
 __device__ __forceinline__ int32_t ld_layout(const int32_t* p) {
-  if constexpr (kCoherent) return __ldcg(p);
+  if constexpr (kShared) return *p;
   else return __ldg(p);
 }
 
-template <bool kCoherent>
-__device__ __forceinline__ PadCursor pad_seek(const DispatchLaunch& L, int32_t i) {
+template <bool kShared>
+__device__ __forceinline__ PadCursor pad_seek(const DispatchLaunch& L, const int32_t* pad_excl, const int32_t* psum,
+                                              int32_t i) {
   int lo = 0, hi = L.E;  // largest e with pad_excl[e] <= i
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (ld_layout<kCoherent>(L.pad_excl + mid) <= i) lo = mid;
+    if (ld_layout<kShared>(pad_excl + mid) <= i) lo = mid;
     else hi = mid;
   }
-  return PadCursor{lo, ld_layout<kCoherent>(L.pad_excl + lo), ld_layout<kCoherent>(L.pad_excl + lo + 1),
-                   ld_layout<kCoherent>(L.psum + lo)};
+  return PadCursor{lo, ld_layout<kShared>(pad_excl + lo), ld_layout<kShared>(pad_excl + lo + 1),
+                   ld_layout<kShared>(psum + lo), pad_excl, psum};
 }
 
 // Receive-buffer row (rank * cap + row) of padding row i, at or after the cursor's row; -1 when it
 // lies at or beyond cap.  Expert e's padding rows are [psum[e] - pad_e, psum[e]) of its rank.
-template <bool kCoherent>
+template <bool kShared>
 __device__ __forceinline__ int64_t pad_row(const DispatchLaunch& L, PadCursor& c, int32_t i) {
   while (i >= c.end) {
     ++c.e;
     c.begin = c.end;
-    c.end = ld_layout<kCoherent>(L.pad_excl + c.e + 1);
-    c.last = ld_layout<kCoherent>(L.psum + c.e);
+    c.end = ld_layout<kShared>(c.pad_excl + c.e + 1);
+    c.last = ld_layout<kShared>(c.psum + c.e);
   }
   const int32_t row = c.last - (c.end - c.begin) + (i - c.begin);
   return row < L.cap ? (int64_t)(c.e / L.E_loc) * L.cap + row : -1;
@@ -272,7 +275,7 @@ __device__ __forceinline__ void zero_padding_rows(const DispatchLaunch& L, int64
   const int64_t P = __ldg(L.pad_excl + L.E);
   const int32_t i0 = (int32_t)(P * gw / nw), i1 = (int32_t)(P * (gw + 1) / nw);
   if (i0 >= i1) return;
-  PadCursor c = pad_seek<false>(L, i0);
+  PadCursor c = pad_seek<false>(L, L.pad_excl, L.psum, i0);
   for (int32_t i = i0; i < i1; ++i) {
     const int64_t grow = pad_row<false>(L, c, i);
     if (grow < 0) overflow = true;
@@ -550,8 +553,8 @@ __global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunc
     const int32_t pb = (int32_t)((int64_t)P * blockIdx.x / gridDim.x);
     const int32_t pe = (int32_t)((int64_t)P * (blockIdx.x + 1) / gridDim.x);
     int32_t pn = pb + grp;
-    PadCursor pc{0, 0, 0, 0};
-    if (kFp8 && pn < pe) pc = pad_seek<false>(L, pn);
+    PadCursor pc{0, 0, 0, 0, L.pad_excl, L.psum};
+    if (kFp8 && pn < pe) pc = pad_seek<false>(L, L.pad_excl, L.psum, pn);
     if constexpr (kFp8) {
       // ---------------------------------------------------------------- FP8 consumers
       const int64_t nblk = H / 128, nunits = H / 16;
@@ -614,7 +617,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunc
       const int32_t i0 = pb + (int32_t)((int64_t)(pe - pb) * w / kDispConsumerWarps);
       const int32_t i1 = pb + (int32_t)((int64_t)(pe - pb) * (w + 1) / kDispConsumerWarps);
       if (i0 < i1) {
-        PadCursor c = pad_seek<false>(L, i0);
+        PadCursor c = pad_seek<false>(L, L.pad_excl, L.psum, i0);
         for (int32_t i = i0; i < i1; ++i) {
           const int64_t grow = pad_row<false>(L, c, i);
           if (grow < 0) overflow = true;
@@ -630,31 +633,31 @@ __global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunc
 // ------------------------------------------------------------------------------------------------
 // One-launch layout + dispatch (moe_layout_dispatch without host sync, small batches): the
 // layout's notify work and the dispatch in one kernel, as the dispatch kernel of "From DeepEP to
-// Mega MoE" 2.2 runs notify warps beside its dispatch warps.  One cooperative launch of G CTAs
-// (every one resident), 576 threads each; CTA b owns items i < n_b (token b + i * G, a stage
-// each: n_b <= kLdMaxItems, no ring), and CTAs below C each own one layout chunk:
+// Mega MoE" 2.2 runs notify warps beside its dispatch warps.  G CTAs of 576 threads, one per SM;
+// CTA b owns the chunk of tokens [b * chunk, (b + 1) * chunk) (chunk <= kLdMaxItems, an item and
+// a stage per token, no ring).  No CTA waits for another: each computes the layout of its own
+// chunk from the whole routing table (replicated_layout_chunk), so the tokens it dispatches are
+// the ones whose slots it has just assigned.
 //   warp 0       producer: at once, one bulk load of each item's bf16 row (x does not depend on
-//                the layout); after the second grid barrier (all C chunks assigned), the item's
-//                destination rows into its DispMeta, then an arrive on meta[i];
-//   warp 1       storer: per item, once its row (BF16: the input stage; FP8: the codes) and its
-//                metadata are ready, lanes 0..n-1 each issue one bulk store to a destination and
-//                write recv_w;
-//   warps 2..9   the layout of chunk b (layout_body.cuh, on named barrier 1), then an arrive on
-//                the second grid barrier; then, in every CTA, the CTA's share of padding rows
-//                once every chunk is assigned;
+//                the layout); once the chunk is assigned (the lready barrier), the item's
+//                destination rows from the slots the layout recorded in shared memory into its
+//                DispMeta, then an arrive on meta[i];
+//   warp 1       storer: per item, once its row (BF16: the input stage; FP8: the codes and
+//                scales) and its metadata are ready, lanes 0..n-1 each issue one bulk store of
+//                the row to a destination and write recv_w; FP8: the lanes copy the scales;
+//   warps 2..9   the layout (named barrier 1; CTA 0 publishes the handle's per-expert arrays),
+//                then an arrive on lready; then the CTA's share of the padding rows, located from
+//                its own psum and padding prefix in shared memory;
 //   warps 10..17 FP8: quantise each item into its output stage as soon as its row lands (while
-//                the layout runs), the 1x128 scales into shared memory; once the metadata is
-//                there, the scales to every destination.
-// The second grid barrier is the handle's status[5] (cleared with the status block before the
-// launch), raised by each layout chunk after a fence once its slots and row maps are written;
-// every wait is bounded by wall-clock time.  The layout's arrays written in this launch are read
-// through L2 (ld.global.cg).
+//                the layout runs), the 1x128 scales into shared memory, then exit (warps left
+//                polling a barrier would take issue slots from the storer and the producer).
+// Every wait is an mbarrier wait inside the CTA, bounded by wall-clock time.
 constexpr int kLdMaxItems = 8;     // items (tokens) per CTA
 constexpr int kLdThreads = 576;
 constexpr int kLdLayoutBar = 1;    // named barrier of the layout warps
 
 struct LdSmem {
-  uint32_t full, qdone, mready, meta, scales, layout, in, out, zero, total;
+  uint32_t full, qdone, mready, lready, meta, rec, scales, layout, in, out, zero, total;
 };
 
 __host__ __device__ inline LdSmem ld_smem(int64_t H, bool fp8, int n, int E, int R) {
@@ -666,9 +669,13 @@ __host__ __device__ inline LdSmem ld_smem(int64_t H, bool fp8, int n, int E, int
   off += 8 * n;
   l.mready = off;
   off += 8 * n;
+  l.lready = off;
+  off += 8;
   off = round_to(off, 16);
   l.meta = off;
   off += (uint32_t)sizeof(DispMeta) * n;
+  l.rec = off;                          // int32 slot[n * kMaxTopk], rank[n * kMaxTopk], fp32 w[n * kMaxTopk]
+  off += 3 * 4 * (uint32_t)(n * kMaxTopk);
   l.scales = off;
   off += fp8 ? (uint32_t)(4 * (H / 128) * n) : 0;
   off = round_to(off, 16);
@@ -686,23 +693,25 @@ __host__ __device__ inline LdSmem ld_smem(int64_t H, bool fp8, int n, int E, int
   return l;
 }
 
-template <bool kFp8, int kRounds>
+template <bool kFp8>
 __global__ void __launch_bounds__(kLdThreads, 1)
-    k_layout_dispatch(LayoutLaunch LL, int64_t cap_check, int C, DispatchLaunch L) {
+    k_layout_dispatch(LayoutLaunch LL, int64_t cap_check, int chunk, DispatchLaunch L) {
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int32_t base_r[kMaxByRankRanks];
-  __shared__ int32_t go, go2;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t H = L.H, nblk = H / 128;
-  const int64_t n = cta_tokens(L.T);
+  const int64_t t0 = min((int64_t)blockIdx.x * chunk, L.T), n = min((int64_t)chunk, L.T - t0);
   const LdSmem lay = ld_smem(H, kFp8, kLdMaxItems, LL.E, LL.R);
   const uint32_t base = smem_u32(smem);
   const uint32_t full0 = base + lay.full, qdone0 = base + lay.qdone, mready0 = base + lay.mready;
+  const uint32_t lready = base + lay.lready;
   DispMeta* meta = reinterpret_cast<DispMeta*>(smem + lay.meta);
+  int32_t* rec_slot = reinterpret_cast<int32_t*>(smem + lay.rec);
+  int32_t* rec_rank = rec_slot + kLdMaxItems * kMaxTopk;
+  float* rec_w = reinterpret_cast<float*>(rec_rank + kLdMaxItems * kMaxTopk);
   float* scales_s = reinterpret_cast<float*>(smem + lay.scales);
+  int32_t* lsm = reinterpret_cast<int32_t*>(smem + lay.layout);
   const uint32_t in_bytes = (uint32_t)(2 * H);
   const uint32_t row_bytes = kFp8 ? (uint32_t)H : in_bytes;
-  int32_t* done_ctr = LL.d.status + 5;
 
   if (tid == 0) {
     for (int i = 0; i < kLdMaxItems; ++i) {
@@ -710,12 +719,14 @@ __global__ void __launch_bounds__(kLdThreads, 1)
       mbar_init(qdone0 + 8 * i, kDispGroupWarps);
       mbar_init(mready0 + 8 * i, 1);
     }
+    mbar_init(lready, 1);
     fence_mbar_init();
   }
   for (uint32_t o = (uint32_t)tid * 16; o < kZeroBytes; o += kLdThreads * 16) sts_v4(base + lay.zero + o, make_uint4(0, 0, 0, 0));
   fence_proxy_async_smem();  // the zero block is read by the bulk engine (async proxy)
   __syncthreads();
   grid_dependents_launch();
+  grid_dependency_wait();  // the routing and x, and receive buffers earlier kernels may still read
   bool overflow = false;
 
   if (warp == 0) {
@@ -723,50 +734,45 @@ __global__ void __launch_bounds__(kLdThreads, 1)
     if (lane == 0)
       for (int64_t i = 0; i < n; ++i) {
         mbar_arrive_expect_tx(full0 + 8 * i, in_bytes);
-        if (dbg_ok(i < kLdMaxItems && cta_token(i) < L.T, L.status, 211, i))
-          bulk_load(base + lay.in + (uint32_t)i * in_bytes, static_cast<const uint16_t*>(L.x) + cta_token(i) * H,
+        if (dbg_ok(i < kLdMaxItems && t0 + i < L.T, L.status, 211, i))
+          bulk_load(base + lay.in + (uint32_t)i * in_bytes, static_cast<const uint16_t*>(L.x) + (t0 + i) * H,
                     in_bytes, full0 + 8 * i);
       }
-    bool ok = true;
-    if (lane == 0) ok = wait_count_reached(done_ctr, C, L.status);
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    asm volatile("fence.acq_rel.gpu;" ::: "memory");
-    const int tpb = 32 / L.k, lanes_used = tpb * L.k;
-    for (int64_t ib = 0; ib < n; ib += tpb) {
-      PairBatch cur{-1, -1, 0.0f, -1};
-      const int q0 = lane / L.k;
-      if (ok && lane < lanes_used && ib + q0 < n) {  // the pairs of items ib .. ib + tpb - 1
-        const int64_t p = cta_token(ib + q0) * L.k + (lane - q0 * L.k);
-        cur.rank = __ldcg(L.pair_rank + p);
-        cur.slot = __ldcg(L.slot + p);
-        cur.w = __ldcg(L.pair_w + p);
-      }
-      const int nt = (int)min((int64_t)tpb, n - ib);
-      for (int q = 0; q < nt; ++q) {
-        const int64_t i = ib + q;
-        int64_t row = -1;
-        if (lane >= q * L.k && lane < (q + 1) * L.k && cur.rank >= 0 && cur.slot >= 0) {
-          if (cur.slot < L.cap) row = (int64_t)cur.rank * L.cap + cur.slot;
+    const bool ok = mbar_wait_warp(lready, 0, L.status);  // the chunk's slots are in rec_*
+    for (int64_t i = 0; i < n; ++i) {  // shared memory only
+      int64_t row = -1;
+      float w = 0.0f;
+      if (ok && lane < L.k) {
+        const int j = (int)i * L.k + lane;
+        const int32_t rk = rec_rank[j], sl = rec_slot[j];
+        if (rk >= 0 && sl >= 0) {
+          if (sl < L.cap) row = (int64_t)rk * L.cap + sl;
           else overflow = true;
+          w = rec_w[j];
         }
-        const uint32_t m = __ballot_sync(0xffffffffu, row >= 0);
-        if (row >= 0) {
-          const int pos = __popc(m & lanemask_lt());
-          meta[i].row[pos] = row;
-          meta[i].w[pos] = cur.w;
-        }
-        if (lane == 0) meta[i].n = __popc(m);  // 0 when the layout gave up: nothing is written
-        __syncwarp();
-        if (lane == 0) mbar_arrive(mready0 + 8 * i);
       }
+      const uint32_t m = __ballot_sync(0xffffffffu, row >= 0);
+      if (row >= 0) {
+        const int pos = __popc(m & lanemask_lt());
+        meta[i].row[pos] = row;
+        meta[i].w[pos] = w;
+      }
+      if (lane == 0) meta[i].n = __popc(m);  // 0 when the layout gave up: nothing is written
+      __syncwarp();
+      if (lane == 0) mbar_arrive(mready0 + 8 * i);
     }
     // no load of this CTA may still be in flight when it exits
     if (lane == 0)
       for (int64_t i = 0; i < n; ++i) mbar_wait(full0 + 8 * i, 0, L.status);
   } else if (warp == 1) {
     // ---------------------------------------------------------------- storer
+    // codes (or bf16 rows): one bulk store per destination; FP8 scales: 16-byte stores by the
+    // lanes (4-byte ones when a row of them is not a whole number of 16-byte units or the buffer
+    // is not 16-byte aligned), which keeps the bulk-copy queue for the rows
     uint8_t* recv = static_cast<uint8_t*>(L.recv_x);
     const uint64_t pol = l2_evict_first_policy();
+    const int64_t sc_units = nblk / 4;  // 16-byte units of a row of scales
+    const bool sc_vec = kFp8 && nblk % 4 == 0 && (reinterpret_cast<uintptr_t>(L.recv_scales) & 15u) == 0;
     for (int64_t i = 0; i < n; ++i) {
       if (!mbar_wait_warp(kFp8 ? qdone0 + 8 * i : full0 + 8 * i, 0, L.status)) break;
       if (!mbar_wait_warp(mready0 + 8 * i, 0, L.status)) break;
@@ -778,43 +784,48 @@ __global__ void __launch_bounds__(kLdThreads, 1)
         bulk_store_hinted(recv + row * row_bytes, src, row_bytes, pol);
         if (L.recv_w) L.recv_w[row] = meta[i].w[lane];
       }
+      if (kFp8 && sc_vec)
+        for (int64_t x = lane; x < nd * sc_units; x += 32) {
+          const int j = (int)(x / sc_units);
+          const int64_t u = x - j * sc_units;
+          const int64_t r = meta[i].row[j];
+          const uint4 v = *reinterpret_cast<const uint4*>(scales_s + i * nblk + 4 * u);
+          if (dbg_ok(r >= 0 && r < L.R * L.cap, L.status, 215, r))
+            *reinterpret_cast<uint4*>(L.recv_scales + r * nblk + 4 * u) = v;
+        }
+      else if (kFp8)
+        for (int64_t x = lane; x < nd * nblk; x += 32) {
+          const int j = (int)(x / nblk);
+          const int64_t b = x - j * nblk;
+          const int64_t r = meta[i].row[j];
+          if (dbg_ok(r >= 0 && r < L.R * L.cap, L.status, 215, r)) L.recv_scales[r * nblk + b] = scales_s[i * nblk + b];
+        }
       bulk_commit();
     }
     bulk_wait_all();  // no store may still read shared memory when the CTA exits
   } else if (warp < 10) {
     // ---------------------------------------------------------------- layout, then padding rows
     const ThreadGroup g{tid - 64, kLayoutThreads, kLdLayoutBar};
-    bool ok = true;
-    if ((int)blockIdx.x < C) {
-      int32_t* lsm = reinterpret_cast<int32_t*>(smem + lay.layout);
-      ok = fused_layout_chunk<kRounds>(LL, cap_check, blockIdx.x, C, g, lsm, base_r, &go);
-      if (ok) {
-        __threadfence();  // the chunk's slots, pair data and row maps before the arrival
-        g.sync();
-        if (g.tid == 0) atomicAdd(done_ctr, 1);
-      }
-    }
-    const int32_t P = ok && (L.zero_padding || L.recv_w) ? 1 : 0;
-    if (P) {
-      if (g.tid == 0) go2 = wait_count_reached(done_ctr, C, L.status);
-      g.sync();
-      if (go2) {
-        asm volatile("fence.acq_rel.gpu;" ::: "memory");
-        const int32_t total = __ldcg(L.pad_excl + L.E);
-        const int32_t pb = (int32_t)((int64_t)total * blockIdx.x / gridDim.x);
-        const int32_t pe = (int32_t)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
-        const int w = warp - 2;  // warp w of the 8 takes the contiguous run w of the CTA's share
-        const int32_t i0 = pb + (int32_t)((int64_t)(pe - pb) * w / kLayoutWarps);
-        const int32_t i1 = pb + (int32_t)((int64_t)(pe - pb) * (w + 1) / kLayoutWarps);
-        if (i0 < i1) {
-          PadCursor c = pad_seek<true>(L, i0);
-          for (int32_t i = i0; i < i1; ++i) {
-            const int64_t grow = pad_row<true>(L, c, i);
-            if (grow < 0) overflow = true;
-            else zero_padding_row_bulk<kFp8>(L, grow, base + lay.zero, lane);
-          }
-          bulk_wait_all();  // the bulk stores read the zero block until they complete
+    replicated_layout_chunk(LL, cap_check, t0, t0 + n, blockIdx.x == 0, g, lsm, rec_slot, rec_rank, rec_w);
+    g.sync();  // every pair of the chunk is assigned (its slot recorded) before the arrival
+    if (g.tid == 0) mbar_arrive(lready);
+    if (L.zero_padding || L.recv_w) {
+      const int32_t* pad_s = lsm + (kLayoutWarps + 6) * LL.E;   // pad_excl[E + 1], this CTA's copy
+      const int32_t* psum_s = lsm + (kLayoutWarps + 5) * LL.E;  // psum[E]
+      const int32_t total = pad_s[LL.E];
+      const int32_t pb = (int32_t)((int64_t)total * blockIdx.x / gridDim.x);
+      const int32_t pe = (int32_t)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
+      const int w = warp - 2;  // warp w of the 8 takes the contiguous run w of the CTA's share
+      const int32_t i0 = pb + (int32_t)((int64_t)(pe - pb) * w / kLayoutWarps);
+      const int32_t i1 = pb + (int32_t)((int64_t)(pe - pb) * (w + 1) / kLayoutWarps);
+      if (i0 < i1) {
+        PadCursor c = pad_seek<true>(L, pad_s, psum_s, i0);
+        for (int32_t i = i0; i < i1; ++i) {
+          const int64_t grow = pad_row<true>(L, c, i);
+          if (grow < 0) overflow = true;
+          else zero_padding_row_bulk<kFp8>(L, grow, base + lay.zero, lane);
         }
+        bulk_wait_all();  // the bulk stores read the zero block until they complete
       }
     }
   } else if (kFp8) {
@@ -838,50 +849,32 @@ __global__ void __launch_bounds__(kLdThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(qdone0 + 8 * i);
     }
-    for (int64_t i = 0; i < n; ++i) {  // the scales, once the destinations are known
-      if (!mbar_wait_warp(qdone0 + 8 * i, 0, L.status)) break;  // every warp's scales are in
-      if (!mbar_wait_warp(mready0 + 8 * i, 0, L.status)) break;
-      const int nd = meta[i].n;
-      if (!dbg_ok(nd >= 0 && nd <= L.k, L.status, 214, nd)) break;
-      for (int64_t x = gtid; x < nd * nblk; x += kDispGroupThreads) {
-        const int j = (int)(x / nblk);
-        const int64_t b = x - j * nblk;
-        const int64_t row = meta[i].row[j];
-        if (dbg_ok(row >= 0 && row < L.R * L.cap, L.status, 215, row)) L.recv_scales[row * nblk + b] = scales_s[i * nblk + b];
-      }
-    }
   }
   if (overflow) atomicOr(L.status, kStatusCapacity);
 }
 
-// Whether a batch takes the one-launch layout + dispatch: at most kLdMaxItems tokens per CTA of
-// the grid, layout chunks whose pairs fit kFusedRounds rounds per warp, and shared memory (the
-// layout's arrays, a stage per item) that fits.
-bool layout_dispatch_fits(int64_t T, int64_t H, bool fp8, int E, int R, int grid, int chunk, int k) {
-  if (grid < 1 || (T + grid - 1) / grid > kLdMaxItems) return false;
-  if ((int64_t)chunk * k > (int64_t)kLayoutThreads * kFusedRounds) return false;
-  return ld_smem(H, fp8, kLdMaxItems, E, R).total <= 227u * 1024u - 1024u;
+// Whether a batch takes the one-launch layout + dispatch: chunks of at most kLdMaxItems tokens,
+// one per CTA of the grid, whose pairs fit one round per layout warp (chunk * k <= the layout
+// warps' threads), T * k below 2^16 (the packed per-expert counts), and shared memory (the
+// layout's arrays, a stage per item) that fits.  Returns the chunk, or 0.
+int layout_dispatch_chunk(int64_t T, int64_t H, bool fp8, int E, int R, int grid, int k) {
+  if (grid < 1 || T < 1 || T * k >= (int64_t)1 << 16) return 0;
+  const int64_t chunk = (T + grid - 1) / grid;
+  if (chunk > kLdMaxItems || chunk * k > kLayoutThreads) return 0;
+  if (ld_smem(H, fp8, kLdMaxItems, E, R).total > 227u * 1024u - 1024u) return 0;
+  return (int)chunk;
 }
 
-cudaError_t launch_layout_dispatch(const LayoutLaunch& LL, int64_t cap_check, const DispatchLaunch& L, bool fp8,
-                                   cudaStream_t st) {
+cudaError_t launch_layout_dispatch(const LayoutLaunch& LL, int64_t cap_check, int chunk, const DispatchLaunch& L,
+                                   bool fp8, cudaStream_t st) {
   const uint32_t smem = ld_smem(L.H, fp8, kLdMaxItems, LL.E, LL.R).total;
-  if ((int64_t)LL.chunk * LL.k > (int64_t)kLayoutThreads * kFusedRounds) return cudaErrorInvalidValue;
-  auto kern = fp8 ? k_layout_dispatch<true, kFusedRounds> : k_layout_dispatch<false, kFusedRounds>;
+  if (chunk < 1 || chunk > kLdMaxItems || (int64_t)chunk * LL.k > kLayoutThreads) return cudaErrorInvalidValue;
+  auto kern = fp8 ? k_layout_dispatch<true> : k_layout_dispatch<false>;
   static unsigned long long done[2] = {0, 0};
   cudaError_t err = set_smem_limit_once(kern, 227 * 1024 - 1024, &done[fp8 ? 1 : 0]);
   if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(L.grid);
-  cfg.blockDim = dim3(kLdThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, kern, LL, cap_check, LL.num_chunks, L);
+  const int grid = (int)((L.T + chunk - 1) / chunk);  // every CTA owns a chunk (<= L.grid)
+  err = launch_pdl(kern, dim3(grid), dim3(kLdThreads), (size_t)smem, st, LL, cap_check, chunk, L);
   note_launch();
   return err;
 }

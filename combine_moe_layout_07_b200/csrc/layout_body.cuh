@@ -86,9 +86,11 @@ __device__ __forceinline__ void histogram_round(int32_t e, int32_t* h) {
 
 // One round of the assignment: pair p (when in_range) with expert e (or -1) and weight w gets
 // row h[e] + (lanes below it with the same id); h[e] advances by the group's size.  Writes slot,
-// pair rank, pair weight and the row maps.  Returns true on a row >= row_cap.
+// pair rank, pair weight and the row maps (and, when rec_slot is given, the slot and rank into
+// rec_slot[rec_i] / rec_rank[rec_i] too).  Returns true on a row >= row_cap.
 __device__ __forceinline__ bool assign_round(const LayoutLaunch& L, int64_t p, bool in_range, int32_t e, float w,
-                                             int32_t* h) {
+                                             int32_t* h, int32_t* rec_slot = nullptr, int32_t* rec_rank = nullptr,
+                                             int rec_i = 0) {
   const int lane = threadIdx.x & 31;
   const uint32_t peers = __match_any_sync(0xffffffffu, e);
   int32_t row = -1;
@@ -103,6 +105,10 @@ __device__ __forceinline__ bool assign_round(const LayoutLaunch& L, int64_t p, b
     L.d.slot[p] = row;
     L.d.pair_rank[p] = rk;
     L.d.pair_w[p] = w;
+    if (rec_slot) {
+      rec_slot[rec_i] = row;
+      rec_rank[rec_i] = rk;
+    }
     if (e >= 0) {
       if (row < L.row_cap) {
         L.d.row_src[(int64_t)rk * L.row_cap + row] = (int32_t)((uint32_t)p / (uint32_t)L.k);
@@ -421,6 +427,129 @@ __device__ __forceinline__ bool fused_layout_chunk(const LayoutLaunch& L, int64_
   overflow |= row_map_padding(L, pad_s, psum_s, (int64_t)c * W + warp, (int64_t)C * W);
   if (overflow) atomicOr(L.d.status, kStatusCapacity);
   return true;
+}
+
+// ------------------------------------------------------------------------------------ replicated
+// The layout of one chunk with no grid-wide step, for the one-launch layout + dispatch of small
+// batches.  Every CTA of the launch counts all T * k pairs of the batch itself (the routing table
+// comes from DRAM once, then from L2), packing per expert (pairs << 16) | (pairs before the
+// chunk) into one shared-memory atomic, so it knows every expert's total and its chunk's offset
+// inside each expert without reading another CTA's counts; psum follows as in block_psum, and
+// the chunk's pairs are assigned from there.  The chunk is tokens [t0, t1) with (t1 - t0) * k <=
+// g.n (one round of 32 pairs per warp), and T * k < 2^16 for the packed counts.
+//   publish  (one CTA) writes cnt, psum, pad_excl, rows_per_rank and the capacity and bad-id flags;
+//   every CTA adds its chunk's per-rank token counts to tokens_per_rank (cleared before the
+//   launch), writes token_in_rank, slot, pair rank / weight and the row maps of its chunk's pairs
+//   (and the slot, rank and weight of chunk pair j into rec_slot[j] / rec_rank[j] / rec_w[j]), and
+//   the padding rows' row maps of its share (warps blockIdx.x * W + w over gridDim.x * W).
+// Shared memory: sm = fused_layout_smem(E, R, W) bytes; afterwards psum_s (sm + (W + 5) E) and
+// pad_s (sm + (W + 6) E) hold psum and pad_excl.
+constexpr int kRepLoads = 8;  // loads (of two routing ids each) in flight per thread in the batch-wide count
+
+__device__ __forceinline__ void replicated_layout_chunk(const LayoutLaunch& L, int64_t cap_check, int64_t t0,
+                                                        int64_t t1, bool publish, const ThreadGroup& g, int32_t* sm,
+                                                        int32_t* rec_slot, int32_t* rec_rank, float* rec_w) {
+  const int E = L.E, R = L.R, tid = g.tid, warp = tid >> 5, W = g.n >> 5;
+  int32_t* whist = sm;                        // [W][E]  per-warp histograms of the chunk, then bases
+  int32_t* hist = whist + W * E;              // [E]  expert totals
+  int32_t* off = hist + E;                    // [E]  packed counts, then the pairs before the chunk
+  int32_t* al = off + E;                      // [E]
+  int32_t* pad = al + E;                      // [E]
+  int32_t* gincl = pad + E;                   // [E]
+  int32_t* psum_s = gincl + E;                // [E]
+  int32_t* pad_s = psum_s + E;                // [E + 1]
+  int32_t* tok = pad_s + E + 1;               // [R]
+
+  // the chunk's pairs, one per thread (warp w: pairs p0 + 32 w + lane)
+  const int64_t p0 = t0 * L.k, np = (t1 - t0) * L.k;
+  const int64_t p = p0 + tid;
+  const bool mine = tid < np;
+  int32_t ev = -1;
+  float wv = 0.0f;
+  bool ok = true;
+  if (mine) {
+    const int32_t e = expert_of(__ldg(L.idx + p), E);
+    ok = e != -2;
+    ev = max(e, -1);
+    wv = L.w ? __ldg(L.w + p) : 0.0f;
+  }
+  if (mine) rec_w[tid] = wv;
+  for (int i = tid; i < W * E; i += g.n) whist[i] = 0;
+  for (int e = tid; e < E; e += g.n) off[e] = 0;
+  for (int r = tid; r < R; r += g.n) tok[r] = 0;
+  g.sync();
+
+  // 1. every pair of the batch: (1 << 16) | (q < p0) into off[e]; two ids per 16-byte load when
+  // the table is 16-byte aligned (kRepLoads loads in flight per thread)
+  const int64_t NP = L.T * L.k;
+  bool bad = false;
+  const bool vec = (reinterpret_cast<uintptr_t>(L.idx) & 15u) == 0;
+  const int64_t NV = vec ? NP / 2 : 0;  // ids [0, 2 NV) by pairs, the rest one by one
+  const longlong2* idx2 = reinterpret_cast<const longlong2*>(L.idx);
+  for (int64_t v0 = 0; v0 < NV; v0 += (int64_t)g.n * kRepLoads) {
+    longlong2 ii[kRepLoads];
+#pragma unroll
+    for (int u = 0; u < kRepLoads; ++u) {
+      const int64_t v = v0 + (int64_t)u * g.n + tid;
+      ii[u] = v < NV ? __ldg(idx2 + v) : make_longlong2(-1, -1);
+    }
+#pragma unroll
+    for (int u = 0; u < kRepLoads; ++u) {
+      const int64_t q = 2 * (v0 + (int64_t)u * g.n + tid);
+      const int32_t ea = expert_of(ii[u].x, E), eb = expert_of(ii[u].y, E);
+      bad |= (ea == -2) | (eb == -2);
+      if (ea >= 0) atomicAdd_block(&off[ea], (1 << 16) | (q < p0 ? 1 : 0));
+      if (eb >= 0) atomicAdd_block(&off[eb], (1 << 16) | (q + 1 < p0 ? 1 : 0));
+    }
+  }
+  for (int64_t q0 = 2 * NV; q0 < NP; q0 += (int64_t)g.n * kRepLoads) {
+    int32_t ee[kRepLoads];
+#pragma unroll
+    for (int u = 0; u < kRepLoads; ++u) {
+      const int64_t q = q0 + (int64_t)u * g.n + tid;
+      ee[u] = q < NP ? expert_of(__ldg(L.idx + q), E) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kRepLoads; ++u) {
+      const int64_t q = q0 + (int64_t)u * g.n + tid;
+      bad |= ee[u] == -2;
+      if (ee[u] >= 0) atomicAdd_block(&off[ee[u]], (1 << 16) | (q < p0 ? 1 : 0));
+    }
+  }
+  if (publish && bad) atomicOr(L.d.status, kStatusBadExpert);
+  // 2. the chunk: per-warp histograms (every warp takes part in the match), token membership
+  histogram_round(ev, whist + warp * E);
+  for (int64_t tb = t0; tb < t1; tb += g.n) {  // same trip count for every thread
+    const int64_t t = tb + tid;
+    ok &= token_membership(L, t, t < t1, nullptr, tok);
+  }
+  if (!ok) atomicOr(L.d.status, kStatusBadExpert);
+  g.sync();
+  for (int e = tid; e < E; e += g.n) {
+    const int32_t v = off[e];
+    hist[e] = v >> 16;
+    off[e] = v & 0xFFFF;
+  }
+  for (int r = tid; r < R; r += g.n)
+    if (tok[r]) atomicAdd(L.d.tokens_per_rank + r, tok[r]);  // integer sum: order-free
+  g.sync();
+  block_psum<false>(L, hist, cap_check, al, pad, gincl, pad_s, psum_s, publish, g);
+  if (publish)
+    for (int e = tid; e < E; e += g.n) L.d.cnt[e] = hist[e];
+
+  // 3. assign: warp bases from the expert's segment start and the chunk's offset, then the pairs
+  for (int e = tid; e < E; e += g.n) {
+    int32_t base = psum_s[e] - al[e] + off[e];
+    for (int w = 0; w < W; ++w) {
+      const int32_t v = whist[w * E + e];
+      whist[w * E + e] = base;
+      base += v;
+    }
+  }
+  g.sync();
+  bool overflow = assign_round(L, p, mine, ev, wv, whist + warp * E, rec_slot, rec_rank, tid);
+  overflow |= row_map_padding(L, pad_s, psum_s, (int64_t)blockIdx.x * W + warp, (int64_t)gridDim.x * W);
+  if (overflow) atomicOr(L.d.status, kStatusCapacity);
 }
 
 }  // namespace moe

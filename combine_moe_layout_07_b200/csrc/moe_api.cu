@@ -529,11 +529,11 @@ int moe_layout_dispatch(const moe_params_t* p, const int64_t* topk_idx, const fl
     const int64_t cap = p->recv_capacity_rows;
     const DispatchLaunch D =
         expanded_dispatch(h, x, recv_x, recv_scales, recv_weights, cap, do_zero_padding, p->num_sms);
-    if (fused && L.num_chunks <= D.grid &&
-        layout_dispatch_fits(p->num_tokens, p->hidden, fp8, p->num_experts, p->num_logical_ranks, D.grid, L.chunk,
-                             L.k)) {
+    const int ld_chunk =
+        layout_dispatch_chunk(p->num_tokens, p->hidden, fp8, p->num_experts, p->num_logical_ranks, D.grid, L.k);
+    if (ld_chunk > 0) {
       err = cudaMemsetAsync(L.d.status, 0, (size_t)(32 + 8 * (int64_t)L.R + 4 * (int64_t)L.E), s);
-      if (err == cudaSuccess) err = launch_layout_dispatch(L, cap, D, fp8, s);
+      if (err == cudaSuccess) err = launch_layout_dispatch(L, cap, ld_chunk, D, fp8, s);
     } else {  // the same results from the layout's launches and the dispatch kernel
       err = layout_enqueue(p, L, fused, s);
       if (err == cudaSuccess) err = launch_dispatch(D, fp8, s);

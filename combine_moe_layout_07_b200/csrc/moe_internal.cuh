@@ -141,9 +141,9 @@ struct DispatchLaunch {
 };
 
 cudaError_t launch_dispatch(const DispatchLaunch& L, bool fp8, cudaStream_t s);
-bool layout_dispatch_fits(int64_t T, int64_t H, bool fp8, int E, int R, int grid, int chunk, int k);
-cudaError_t launch_layout_dispatch(const LayoutLaunch& LL, int64_t cap_check, const DispatchLaunch& L, bool fp8,
-                                   cudaStream_t s);
+int layout_dispatch_chunk(int64_t T, int64_t H, bool fp8, int E, int R, int grid, int k);
+cudaError_t launch_layout_dispatch(const LayoutLaunch& LL, int64_t cap_check, int chunk, const DispatchLaunch& L,
+                                   bool fp8, cudaStream_t st);
 
 struct CombineLaunch {
   const void* y;

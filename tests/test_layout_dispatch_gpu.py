@@ -93,6 +93,7 @@ def test_decode_shape_with_padding_and_masking(zero_padding):
     dict(hidden=7168, fp8=True, tokens_per_rank=1, ranks=1, experts=4, topk=1),   # one token
     dict(hidden=256, tokens_per_rank=64, ranks=8, experts=2048, topk=8, alignment=1),   # E = 2048
     dict(hidden=1024, fp8=True, tokens_per_rank=16, ranks=4, experts=64, topk=32),      # k = 32
+    dict(hidden=384, fp8=True, tokens_per_rank=50, ranks=2, experts=8, topk=3),         # 3 scales a row
 ])
 @pytest.mark.parametrize("zero_padding", [True, False])
 def test_small_batches_one_launch(kw, zero_padding):
