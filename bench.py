@@ -260,7 +260,7 @@ def reference_tokens(wl: W.Workload, steps: int, warmup: int) -> int:
     return t // wl.ranks * wl.ranks
 
 
-def workload_config(wl: W.Workload, cap: int, extra: dict | None = None) -> dict:
+def workload_config(wl: W.Workload, cap: int, extra: dict | None = None, step_bytes: int = 0) -> dict:
     cfg = {"workload": WORKLOAD_NAMES.get(wl.name, wl.name), "tokens": wl.tokens,
            "tokens_per_rank": wl.tokens_per_rank, "logical_ranks": wl.ranks, "hidden": wl.hidden,
            "experts": wl.experts, "topk": wl.topk, "expert_alignment": wl.alignment, "routing": wl.routing,
@@ -269,7 +269,8 @@ def workload_config(wl: W.Workload, cap: int, extra: dict | None = None) -> dict
                       + (", shared-expert bias" if wl.bias else ", no bias"),
            "do_cpu_sync": int(wl.cpu_sync), "do_zero_padding": int(wl.zero_padding),
            "num_sms": wl.num_sms or "all", "recv_capacity_rows": cap,
-           "l2": "no flush: every step moves several GB (> 126 MB L2)"}
+           "l2": (f"no flush: every step moves {step_bytes / 1e6:.0f} MB (> 126 MB L2)" if step_bytes
+                  else "no flush: every step moves more than the 126 MB L2")}
     if extra:
         cfg.update(extra)
     return cfg
@@ -665,7 +666,7 @@ def side_record(wl: W.Workload, rec: dict, clk: ClockSampler) -> dict:
            "rows_per_rank_max_over_mean": float(rec["rows"].max() / max(rec["rows"].mean(), 1e-9)),
            "roofline": rec["roofline"], "cpu_baseline": rec["cpu_baseline"],
            "clocks": clk.summary(*rec["window"]), "timed_window_unix_s": [round(v, 3) for v in rec["window"]],
-           "config": workload_config(wl, rec["cap"]), **rec["extras"]}
+           "config": workload_config(wl, rec["cap"], step_bytes=nb["dispatch"] + nb["combine"]), **rec["extras"]}
     return out
 
 
@@ -703,7 +704,8 @@ def run_ours(args) -> int:
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "data_types": {"x": "bf16", "recv": "e4m3 + f32 scales" if wl.fp8 else "bf16", "y,out": "bf16"},
                 "config": workload_config(wl, rec["cap"], {"parallelism": f"{world} independent replica(s), "
-                                                                          f"{wl.ranks} logical EP ranks each"}),
+                                                                          f"{wl.ranks} logical EP ranks each"},
+                                          step_bytes=nb["dispatch"] + nb["combine"]),
                 "frac_of_hbm_peak": rec["value"] / world / peak,
                 "frac_of_8tbs_nominal": rec["value"] / world / 8000.0,
                 "kernels_ms": k,
