@@ -17,7 +17,17 @@ pytestmark = pytest.mark.gpu
 FILL8, FILL16 = 0xA5, 0xA5A5
 
 
-def _round_trip(wl, mask=0.0, zero_padding=True, num_sms=0, cap=None, want_w=True, launches=None, bias=False):
+def _placed(t: torch.Tensor, offset_elems: int) -> torch.Tensor:
+    """A copy of t on the GPU starting offset_elems elements into a fresh allocation (an int64
+    table 8 but not 16 bytes aligned, fp32 scales 4 but not 16 bytes aligned, ...)."""
+    flat = torch.empty(t.numel() + offset_elems, dtype=t.dtype, device="cuda")
+    v = flat[offset_elems:].view(t.shape)
+    v.copy_(t.cuda() if not t.is_cuda else t)
+    return v
+
+
+def _round_trip(wl, mask=0.0, zero_padding=True, num_sms=0, cap=None, want_w=True, launches=None, bias=False,
+                idx_offset=0, scales_offset=0):
     idx, w, x = inputs(wl, mask)
     E, R, A, H = wl.experts, wl.ranks, wl.alignment, wl.hidden
     idx_n, w_n = idx.numpy(), w.numpy()
@@ -29,12 +39,12 @@ def _round_trip(wl, mask=0.0, zero_padding=True, num_sms=0, cap=None, want_w=Tru
     rw = torch.full((R, cap), float("nan"), device="cuda") if want_w else None
     if wl.fp8:
         recv = torch.full((R, cap, H), FILL8, dtype=torch.uint8, device="cuda")
-        scales = torch.full((R, cap, H // 128), float("nan"), device="cuda")
+        scales = _placed(torch.full((R, cap, H // 128), float("nan")), scales_offset)
     else:
         recv = torch.full((R, cap, H), FILL16 - 65536, dtype=torch.int16, device="cuda").view(torch.bfloat16)
         scales = None
     n0 = moe.moe_kernel_launch_count()
-    h = moe.moe_layout_dispatch(p, idx.cuda(), w.cuda(), x.cuda(),
+    h = moe.moe_layout_dispatch(p, _placed(idx, idx_offset), w.cuda(), x.cuda(),
                                 moe.MOE_DTYPE_FP8_E4M3 if wl.fp8 else moe.MOE_DTYPE_BF16, recv, scales, rw,
                                 do_zero_padding=zero_padding)
     if launches is not None:
@@ -99,6 +109,43 @@ def test_decode_shape_with_padding_and_masking(zero_padding):
 def test_small_batches_one_launch(kw, zero_padding):
     wl = W.WORKLOADS["tiny"].with_(**kw)
     _round_trip(wl, mask=0.1, zero_padding=zero_padding, launches=1)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(hidden=512, fp8=True, tokens_per_rank=150, experts=32, topk=8),             # 16-byte id pairs
+    dict(hidden=384, fp8=True, tokens_per_rank=25, ranks=1, experts=12, topk=3),     # T * k = 75: one id left
+])
+@pytest.mark.parametrize("idx_offset,scales_offset", [(1, 0), (0, 1), (1, 1)])
+def test_unaligned_routing_table_and_scales(kw, idx_offset, scales_offset):
+    """A routing table 8 but not 16 bytes aligned takes the batch-wide count one id at a time; FP8
+    scales not 16 bytes aligned are written 4 bytes at a time by the storer.  Same bytes."""
+    wl = W.WORKLOADS["tiny"].with_(**kw)
+    _round_trip(wl, mask=0.1, zero_padding=True, launches=1, idx_offset=idx_offset, scales_offset=scales_offset)
+
+
+def _random_case(seed: int):
+    rng = np.random.default_rng(3000 + seed)
+    R = int(rng.choice([1, 2, 4, 8, 16]))
+    E = R * int(rng.integers(1, 33))
+    k = int(rng.integers(1, min(E, 12) + 1))
+    fp8 = bool(rng.integers(0, 2))
+    H = 128 * int(rng.integers(1, 9)) if fp8 else 8 * int(rng.integers(1, 129))
+    tpr = int(rng.integers(1, 1100 // R + 1))
+    kw = dict(tokens_per_rank=tpr, ranks=R, experts=E, topk=k, hidden=H, fp8=fp8,
+              alignment=int(rng.choice([1, 4, 16, 128])), seed=seed)
+    opts = dict(mask=float(rng.choice([0.0, 0.05, 0.3])), zero_padding=bool(rng.integers(0, 2)),
+                want_w=bool(rng.integers(0, 2)), idx_offset=int(rng.integers(0, 2)),
+                scales_offset=int(rng.integers(0, 2)) if fp8 else 0)
+    return kw, opts
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_random_shapes_one_launch(seed):
+    """Seeded random shapes of at most 8 tokens per SM (one launch), every byte against the oracle."""
+    kw, opts = _random_case(seed)
+    wl = W.WORKLOADS["tiny"].with_(**kw)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    _round_trip(wl, launches=1 if wl.tokens <= 8 * sms else 2, **opts)
 
 
 def test_sm_cap():
