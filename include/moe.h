@@ -151,10 +151,11 @@ int moe_dispatch(const moe_handle_t* handle, const void* x, int out_dtype, void*
  * cap = params->recv_capacity_rows and num_sms = params->num_sms, and returns the handle as
  * moe_layout does.  params->do_cpu_sync must be 0 and params->flags 0 (MOE_ERR_INVALID_ARG
  * otherwise); the other arguments are those of moe_layout and moe_dispatch.  A bad expert id or
- * a capacity overflow is reported by moe_handle_status.  Small batches (at most 8 tokens per SM
- * of the budget, with the one-launch layout's limits) run as one cooperative kernel whose
- * dispatch warps load and quantise the tokens while its layout warps assign the rows; other
- * batches run the layout's launches and then the dispatch kernel.
+ * a capacity overflow is reported by moe_handle_status.  Small batches (chunks of at most 8
+ * tokens, one per SM of the budget, T * k < 65536, and shared memory for E experts) run as one
+ * kernel in which no CTA waits for another: each CTA's layout warps count the whole routing table
+ * and assign its own chunk's rows while its dispatch warps load and quantise that chunk's tokens.
+ * Other batches run the layout's launches and then the dispatch kernel.
  */
 int moe_layout_dispatch(const moe_params_t* params, const int64_t* topk_idx, const float* topk_weights,
                         const void* x, int out_dtype, void* recv_x, float* recv_scales, float* recv_weights,

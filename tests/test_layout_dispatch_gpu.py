@@ -104,6 +104,7 @@ def test_decode_shape_with_padding_and_masking(zero_padding):
     dict(hidden=256, tokens_per_rank=64, ranks=8, experts=2048, topk=8, alignment=1),   # E = 2048
     dict(hidden=1024, fp8=True, tokens_per_rank=16, ranks=4, experts=64, topk=32),      # k = 32
     dict(hidden=384, fp8=True, tokens_per_rank=50, ranks=2, experts=8, topk=3),         # 3 scales a row
+    dict(hidden=256, fp8=True, tokens_per_rank=2, ranks=128, experts=256, topk=4),      # R > 64
 ])
 @pytest.mark.parametrize("zero_padding", [True, False])
 def test_small_batches_one_launch(kw, zero_padding):
