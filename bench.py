@@ -50,6 +50,24 @@ def algorithmic_bytes(wl: W.Workload, valid_pairs: int, pad_rows: int, weighted:
     return {"dispatch": dispatch, "combine": combine, "layout": layout}
 
 
+def by_rank_bytes(wl: W.Workload, token_rank_rows: int) -> dict:
+    """Non-expanded round trip: dispatch reads x once and writes one FP8 row with its scales and
+    its top-k ids and weights per (token, rank) (BF16: a bf16 row), reading the routing and the
+    token rows; combine reads every row once, writes the output and reads the token rows."""
+    T, H, k, R = wl.tokens, wl.hidden, wl.topk, wl.ranks
+    row = (H + 4 * (H // 128)) if wl.fp8 else 2 * H
+    return {"dispatch_by_rank": T * H * 2 + token_rank_rows * (row + k * 8) + T * k * 12 + T * R * 4,
+            "combine_by_rank": token_rank_rows * H * 2 + T * H * 2 + (T * H * 2 if wl.bias else 0) + T * R * 4}
+
+
+def backward_bytes(wl: W.Workload, valid_pairs: int, pad_rows: int) -> dict:
+    """Cached dispatch (the forward dispatch's bytes) and the combine's backward: grad_out read
+    once, one bf16 grad row written per routed row, padding rows zeroed, the slots read."""
+    T, H, k = wl.tokens, wl.hidden, wl.topk
+    return {"dispatch_cached": algorithmic_bytes(wl, valid_pairs, pad_rows)["dispatch"],
+            "combine_backward": T * H * 2 + (valid_pairs + (pad_rows if wl.zero_padding else 0)) * H * 2 + T * k * 8}
+
+
 def kernel_source_digest(*files: str) -> str:
     """sha256 (first 12 hex digits) of the kernel's sources with comments and blank lines removed,
     so that a traffic record stays tied to the code it measured but survives comment edits."""
@@ -652,6 +670,167 @@ def measure_workload(moe, wl: W.Workload, args, world: int, rank: int, dev, stre
     return rec
 
 
+def next_rows_measurement(moe, wl: W.Workload, args, world: int, rank: int, dev, clk: ClockSampler,
+                          steps: int = 100, warmup: int = 5, cpu_tokens: int = 2048) -> dict:
+    """The two widened paths at the headline shape, each timed like the headline step (warm-up,
+    barrier-bracketed CUDA events, max over ranks) with its per-kernel times, roofline fraction,
+    timed window (the caller adds its clock record) and the oracle on a sample:
+      by_rank   non-expanded round trip: layout with the token rows -> by-rank FP8 dispatch (rows
+                plus the per-row top-k views) -> by-rank combine of per-rank partial sums;
+      backward  cached dispatch (a second dispatch with the step's handle, no layout) -> backward
+                of the combine (grad_out scattered to every routed row, padding rows zeroed)."""
+    import oracle
+    stream = torch.cuda.current_stream()
+    T, H, k, E, R, A = wl.tokens, wl.hidden, wl.topk, wl.experts, wl.ranks, wl.alignment
+    idx_c, w_c = W.gen_routing(wl)
+    idx, w, x = idx_c.to(dev), w_c.to(dev), W.gen_x(wl).to(dev)
+    peak, _ = hbm_peak()
+    out = {}
+
+    def timed(step, parts):
+        for _ in range(warmup):
+            step(None)
+        torch.cuda.synchronize()
+        ev = []
+        barrier()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0 = time.time()
+        t0.record(stream)
+        for _ in range(steps):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(parts + 1)]
+            step(e)
+            ev.append(e)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        w1 = time.time()
+        barrier()
+        ms = reduce_max(t0.elapsed_time(t1), dev) / steps
+        part_ms = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i in range(parts)]
+        return ms, part_ms, (w0, w1)
+
+    def record(names, part_ms, part_bytes, ms, window, cpu):
+        kern = {n: (t, b) for n, t, b in zip(names, part_ms, part_bytes) if b}
+        dom = max(kern, key=lambda n: kern[n][0])
+        achieved = kern[dom][1] / (kern[dom][0] * 1e-3) / 1e9
+        total = sum(part_bytes)
+        return {"value": world * total / (ms * 1e-3) / 1e9, "unit": UNIT, "us_per_step": ms * 1e3, "steps": steps,
+                "warmup": warmup, "kernels_us": {n: t * 1e3 for n, t in zip(names, part_ms)},
+                "kernels_gbs": {n: b / (t * 1e-3) / 1e9 for n, t, b in zip(names, part_ms, part_bytes) if b},
+                "bytes_per_step": dict(zip(names, part_bytes)),
+                "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                             "frac": achieved / peak, "algorithmic_bytes_per_launch": kern[dom][1], "traffic": None},
+                "cpu_baseline": cpu, "timed_window_unix_s": [round(v, 3) for v in window]}
+
+    def oracle_rate(run):
+        if not (world == 1 and rank == 0 and cpu_tokens > 0):
+            return None
+        best = min(run() for _ in range(3))
+        return {"value": best[1] / best[0] / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+                "sample": best[2] + "; best of 3 passes", "host": host_cpu()}
+
+    n_s = cpu_tokens // R * R
+    idx_s, w_s = idx_c[:n_s].numpy(), w_c[:n_s].numpy()
+    xb_s = W.gen_x(wl.with_(tokens_per_rank=n_s // R)).view(torch.int16).numpy().view(np.uint16)
+
+    # ---- by rank
+    pr = moe.params(T, R, E, k, H, A, recv_capacity_rows=0, do_cpu_sync=True, by_rank=True)
+    h0 = moe.moe_layout(pr, idx, w)
+    tpr = h0.tokens_per_rank().cpu().numpy()
+    moe.moe_handle_free(h0)
+    cap_r, nr = int(tpr.max()), int(tpr.sum())
+    recv = torch.empty(R, cap_r, H, dtype=torch.uint8, device=dev)
+    sc = torch.empty(R, cap_r, H // 128, dtype=torch.float32, device=dev)
+    ti = torch.empty(R, cap_r, k, dtype=torch.int32, device=dev)
+    tw = torch.empty(R, cap_r, k, dtype=torch.float32, device=dev)
+    y = W.gen_y_device(wl, cap_r, device=dev)
+    o = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+
+    def step_by_rank(e):
+        if e is not None:
+            e[0].record(stream)
+        h = moe.moe_layout(pr, idx, w, stream=stream)
+        if e is not None:
+            e[1].record(stream)
+        moe.moe_dispatch_by_rank(h, x, moe.MOE_DTYPE_FP8_E4M3, recv, sc, topk_idx=idx, recv_topk_idx=ti,
+                                 recv_topk_weights=tw, cap=cap_r, stream=stream)
+        if e is not None:
+            e[2].record(stream)
+        moe.moe_combine_by_rank(h, y, o, cap=cap_r, stream=stream)
+        if e is not None:
+            e[3].record(stream)
+        moe.moe_handle_free(h)
+
+    ms, part, win = timed(step_by_rank, 3)
+    bb = by_rank_bytes(wl.with_(bias=False), nr)
+
+    def run_by_rank():
+        t0 = time.perf_counter()
+        st, tr, rows = oracle.layout_by_rank(idx_s, E, R)
+        c = int(rows.max())
+        oracle.dispatch_by_rank(idx_s, w_s, tr, xb_s, E, R, c, True)
+        yb = np.zeros((R, c, H), np.uint16)
+        oracle.combine_by_rank(idx_s, tr, yb, E, R)
+        dt = time.perf_counter() - t0
+        b = sum(by_rank_bytes(wl.with_(tokens_per_rank=n_s // R, bias=False), int(rows.sum())).values())
+        return dt, b, (f"first {n_s} tokens ({n_s // R}/rank) of the batch; by-rank layout + dispatch + combine by "
+                       f"the single-threaded C oracle (zero expert outputs)")
+
+    out["by_rank"] = record(["layout", "dispatch_by_rank", "combine_by_rank"], part,
+                            [0, bb["dispatch_by_rank"], bb["combine_by_rank"]], ms, win, oracle_rate(run_by_rank))
+    out["by_rank"]["rows"] = {"token_rank_rows": nr, "expanded_rows": int((idx_c >= 0).sum()),
+                              "max_per_rank": cap_r}
+    del recv, sc, ti, tw, y, o
+    torch.cuda.empty_cache()
+
+    # ---- cached dispatch + backward of the combine
+    p = moe.params(T, R, E, k, H, A, recv_capacity_rows=0, do_cpu_sync=True)
+    h = moe.moe_layout(p, idx, w)
+    cap = int(h.host_rows_per_rank.max())
+    counts = h.counts().cpu().numpy()
+    rows = h.rows_per_rank().cpu().numpy()
+    valid, pad = int(counts.sum()), int(rows.sum()) - int(counts.sum())
+    recv = torch.empty(R, cap, H, dtype=torch.uint8, device=dev)
+    sc = torch.empty(R, cap, H // 128, dtype=torch.float32, device=dev)
+    g_out = W.gen_x(wl.with_(seed=wl.seed + 7)).to(dev)
+    g_y = torch.empty(R, cap, H, dtype=torch.bfloat16, device=dev)
+
+    def step_backward(e):
+        if e is not None:
+            e[0].record(stream)
+        moe.moe_dispatch(h, x, moe.MOE_DTYPE_FP8_E4M3, recv, sc, None, cap=cap, do_zero_padding=True, stream=stream)
+        if e is not None:
+            e[1].record(stream)
+        moe.moe_combine_backward(h, g_out, g_y, cap=cap, do_zero_padding=True, stream=stream)
+        if e is not None:
+            e[2].record(stream)
+
+    ms, part, win = timed(step_backward, 2)
+    bw = backward_bytes(wl.with_(zero_padding=True), valid, pad)
+
+    def run_backward():
+        t0 = time.perf_counter()
+        lay = oracle.layout(idx_s, w_s, E, R, A)
+        c = int(lay.rows_per_rank.max())
+        lay = oracle.layout(idx_s, w_s, E, R, A, cap=c)
+        oracle.dispatch_fp8(lay, idx_s, w_s, xb_s, E, R, A, c, True, want_w=False)
+        oracle.combine_backward(lay, idx_s, xb_s, E, R, A, c)
+        dt = time.perf_counter() - t0
+        v = int(lay.cnt.sum())
+        b = sum(backward_bytes(wl.with_(tokens_per_rank=n_s // R, zero_padding=True), v,
+                               int(lay.rows_per_rank.sum()) - v).values())
+        return dt, b, (f"first {n_s} tokens ({n_s // R}/rank) of the batch; layout + FP8 dispatch + combine "
+                       f"backward by the single-threaded C oracle")
+
+    out["backward"] = record(["dispatch_cached", "combine_backward"], part,
+                             [bw["dispatch_cached"], bw["combine_backward"]], ms, win, oracle_rate(run_backward))
+    moe.moe_handle_free(h)
+    del recv, sc, g_out, g_y, x, idx, w
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
 def side_record(wl: W.Workload, rec: dict, clk: ClockSampler) -> dict:
     """The compact record of a configuration measured beside the headline one."""
     k = rec["kernels_ms"]
@@ -693,6 +872,10 @@ def run_ours(args) -> int:
                                     max(3, args.warmup), 0 if args.no_cpu_baseline else spec["cpu_tokens"],
                                     want_e2e=False, headline=False)
             side[name] = srec
+    next_rows = None
+    if not args.no_side_workloads and wl.name == "deepseek":
+        next_rows = next_rows_measurement(moe, wl, args, world, rank, dev, clk,
+                                          cpu_tokens=0 if args.no_cpu_baseline else 2048)
     clk.stop(args.clock_log)
     clk.t0, clk.t1 = rec["window"]
 
@@ -722,6 +905,10 @@ def run_ours(args) -> int:
         if side:
             line["workloads"] = {WORKLOAD_NAMES[name]: side_record(W.WORKLOADS[name], srec, clk)
                                  for name, srec in side.items()}
+        if next_rows:
+            for r in next_rows.values():  # the sampler's records are read once it has stopped
+                r["clocks"] = clk.summary(*r["timed_window_unix_s"])
+            line["next_rows"] = next_rows
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized():

@@ -89,3 +89,29 @@ def test_clock_summary_falls_back_to_the_nearest_samples():
     assert s["reasons"] == []
     s = c.summary(t0 + 4.0, t0 + 4.1)                   # t0 + 5.0 and t0 + 5.1, one with hw_slowdown
     assert s["sm_mhz"] == float(np.median([1900, 1901])) and s["reasons"] == ["hw_slowdown"]
+
+
+def test_by_rank_and_backward_byte_models():
+    """The widened paths' byte models at the DeepSeek-V3 shape, from a count of the (token, rank)
+    rows made here from the routing: by rank, one FP8 row (7168 codes + 56 scales) with 8 ids and
+    8 weights per (token, rank); backward, one bf16 grad row per routed or padding row."""
+    wl = W.WORKLOADS["deepseek"]
+    idx, w = W.gen_routing(wl)
+    ranks = idx.numpy() // (wl.experts // wl.ranks)
+    token_rank_rows = sum(len(set(r.tolist())) for r in ranks)      # distinct ranks per token
+    st, tr, rows = oracle.layout_by_rank(idx.numpy(), wl.experts, wl.ranks)
+    assert st == oracle.OK and int(rows.sum()) == token_rank_rows
+    assert token_rank_rows <= 4 * wl.tokens                          # group-limited: at most 4 groups
+    T, H = wl.tokens, wl.hidden
+    b = bench.by_rank_bytes(wl, token_rank_rows)
+    assert b["dispatch_by_rank"] == (T * H * 2 + token_rank_rows * (7168 + 224 + 64)
+                                     + T * 8 * 12 + T * 8 * 4)
+    assert b["combine_by_rank"] == token_rank_rows * H * 2 + T * H * 2 + T * 8 * 4
+    lay = oracle.layout(idx.numpy(), w.numpy(), wl.experts, wl.ranks, wl.alignment)
+    valid = int(lay.cnt.sum())
+    pad = int(lay.rows_per_rank.sum()) - valid
+    bw = bench.backward_bytes(wl, valid, pad)
+    assert bw["dispatch_cached"] == bench.algorithmic_bytes(wl, valid, pad)["dispatch"]
+    assert bw["combine_backward"] == T * H * 2 + (valid + pad) * H * 2 + T * 8 * 8
+    assert bench.backward_bytes(wl.with_(zero_padding=False), valid, pad)["combine_backward"] == \
+        T * H * 2 + valid * H * 2 + T * 8 * 8
