@@ -649,8 +649,8 @@ __global__ void __launch_bounds__(kBulkThreads, 1) k_dispatch_bulk(DispatchLaunc
 //                then an arrive on lready; then the CTA's share of the padding rows, located from
 //                its own psum and padding prefix in shared memory;
 //   warps 10..17 FP8: quantise each item into its output stage as soon as its row lands (while
-//                the layout runs), the 1x128 scales into shared memory, then exit (warps left
-//                polling a barrier would take issue slots from the storer and the producer).
+//                the layout runs), the 1x128 scales into shared memory, then exit (the storer
+//                writes the scales with the rows).
 // Every wait is an mbarrier wait inside the CTA, bounded by wall-clock time.
 constexpr int kLdMaxItems = 8;     // items (tokens) per CTA
 constexpr int kLdThreads = 576;
