@@ -38,7 +38,8 @@ constexpr uint32_t kCombSmemBudget = 200 * 1024;
 
 struct CombMeta {
   float w[kMaxTopk];  // weights of the valid pairs in j order (weighted combine)
-  int32_t n;          // valid pairs
+  int32_t n;          // valid pairs (packed items: -1 ends the consumer group's loop)
+  int32_t q, c0, width, stride;  // packed items: the CTA's token index, columns, slot stride in bytes
   int32_t pad_[3];
 };
 
@@ -94,7 +95,12 @@ CombGeom combine_geometry(int64_t H, int k, bool bias) {
   return g;
 }
 
-template <bool kWeighted, bool kBias>
+// kPacked (the by-rank combine, whose tokens gather from at most one row per rank): a token with
+// n source rows takes mult = (k + bias) / (n + bias) chunks of columns per item, with its row
+// segments mult * cw columns wide, so the item fills the stage's k (+ bias) slots of cw columns
+// when n is small.  The item's token, columns and slot stride travel in its CombMeta, and after
+// the last item the producer sends one item with n = -1 to each consumer group.
+template <bool kWeighted, bool kBias, bool kPacked>
 __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, CombGeom g) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -148,8 +154,13 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
         const uint32_t m = __ballot_sync(0xffffffffu, src >= 0);
         const int pos = __popc(m & lanemask_lt());
         const int n = __popc(m);
-        for (int64_t c0 = 0; c0 < H; c0 += g.cw) {
-          const uint32_t bytes = (uint32_t)(min(g.cw, H - c0) * 2);
+        const int nb = kBias ? 1 : 0;
+        // (a token without rows, n + nb == 0, loads nothing: its items may span the whole stage)
+        const int mult = !kPacked ? 1 : (n + nb > 0 ? max(1, (L.k + nb) / (n + nb)) : max(1, L.k + nb));
+        const int64_t span = (int64_t)mult * g.cw;              // columns of one item
+        const uint32_t stride = (uint32_t)(span * 2);          // bytes between its row segments
+        for (int64_t c0 = 0; c0 < H; c0 += span) {
+          const uint32_t bytes = (uint32_t)(min(span, H - c0) * 2);
           if (i >= S) {
             bool ok = true;
             if (lane == 0) ok = mbar_wait(empty0 + 8 * s, par ^ 1u, L.status);
@@ -159,19 +170,28 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
             }
           }
           if (kWeighted && src >= 0) meta[s].w[pos] = cur.w;
-          if (lane == 0) meta[s].n = n;
+          if (lane == 0) {
+            meta[s].n = n;
+            if constexpr (kPacked) {
+              meta[s].q = (int32_t)(qb + q);
+              meta[s].c0 = (int32_t)c0;
+              meta[s].width = (int32_t)min(span, H - c0);
+              meta[s].stride = (int32_t)stride;
+            }
+          }
           __syncwarp();
           const uint32_t stage = base + g.data + (uint32_t)s * g.stage_bytes;
+          const uint32_t bias_off = kPacked ? (uint32_t)n * stride : (uint32_t)L.k * slot_bytes;
           if (lane == 0) {
-            mbar_arrive_expect_tx(full0 + 8 * s, bytes * (uint32_t)(n + (kBias ? 1 : 0)));
-            if (kBias && dbg_ok(t * H + c0 + bytes / 2 <= L.T * H, L.status, 101, t))
-              bulk_load(stage + (uint32_t)L.k * slot_bytes, bias + t * H + c0, bytes, full0 + 8 * s);
+            mbar_arrive_expect_tx(full0 + 8 * s, bytes * (uint32_t)(n + nb));
+            if (kBias && dbg_ok(t * H + c0 + bytes / 2 <= L.T * H && bias_off + bytes <= g.stage_bytes, L.status, 101, t))
+              bulk_load(stage + bias_off, bias + t * H + c0, bytes, full0 + 8 * s);
           }
           __syncwarp();
           if (src >= 0 && dbg_ok(src + c0 + bytes / 2 <= L.R * L.cap * H && pos < L.k &&
-                                     g.data + (uint32_t)s * g.stage_bytes + (uint32_t)pos * slot_bytes + bytes <= g.total,
+                                     (uint32_t)pos * stride + bytes <= g.stage_bytes,
                                  L.status, 102, src))
-            bulk_load(stage + (uint32_t)pos * slot_bytes, y + src + c0, bytes, full0 + 8 * s);
+            bulk_load(stage + (uint32_t)pos * stride, y + src + c0, bytes, full0 + 8 * s);
           __syncwarp();
           ++i;
           if (++s == S) {
@@ -181,6 +201,25 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
         }
       }
       cur = nxt;
+    }
+    if constexpr (kPacked) {  // one item with n = -1 per consumer group ends its loop
+      for (int gq = 0; gq < kCombGroups && !stop; ++gq) {
+        if (i >= S) {
+          bool ok = true;
+          if (lane == 0) ok = mbar_wait(empty0 + 8 * s, par ^ 1u, L.status);
+          if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        }
+        if (lane == 0) {
+          meta[s].n = -1;
+          mbar_arrive(full0 + 8 * s);
+        }
+        __syncwarp();
+        ++i;
+        if (++s == S) {
+          s = 0;
+          par ^= 1u;
+        }
+      }
     }
     // no load of this CTA may still be in flight when it exits: wait for the last S items
     if (lane == 0) {
@@ -208,12 +247,24 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
     }
     int s = grp % S;
     uint32_t par = (uint32_t)((grp / S) & 1);
-    for (; i < n_items; i += kCombGroups) {
-      const int64_t c0 = c * g.cw;
-      const int64_t width = min(g.cw, H - c0);
+    for (; kPacked || i < n_items; i += kCombGroups) {
       if (!mbar_wait_warp(full0 + 8 * s, par, L.status)) break;
       const int n = meta[s].n;
+      if (kPacked && n < 0) break;  // the producer's last item for this group
       if (!dbg_ok(n >= 0 && n <= L.k, L.status, 104, n)) break;
+      int64_t c0, width, qi;
+      uint32_t stride;
+      if constexpr (kPacked) {
+        qi = meta[s].q;
+        c0 = meta[s].c0;
+        width = meta[s].width;
+        stride = (uint32_t)meta[s].stride;
+      } else {
+        qi = q;
+        c0 = c * g.cw;
+        width = min(g.cw, H - c0);
+        stride = slot_bytes;
+      }
       const uint32_t stage = base + g.data + (uint32_t)s * g.stage_bytes;
       for (int64_t e = gtid * 8; e < width; e += kCombGroupThreads * 8) {
         float acc[8];
@@ -223,7 +274,7 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
         for (; j + 4 <= n; j += 4) {
           uint4 d[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) d[u] = lds_v4(stage + (uint32_t)(j + u) * slot_bytes + (uint32_t)e * 2);
+          for (int u = 0; u < 4; ++u) d[u] = lds_v4(stage + (uint32_t)(j + u) * stride + (uint32_t)e * 2);
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const uint32_t wd[4] = {d[u].x, d[u].y, d[u].z, d[u].w};
@@ -241,7 +292,7 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
           }
         }
         for (; j < n; ++j) {
-          const uint4 d = lds_v4(stage + (uint32_t)j * slot_bytes + (uint32_t)e * 2);
+          const uint4 d = lds_v4(stage + (uint32_t)j * stride + (uint32_t)e * 2);
           const uint32_t wd[4] = {d.x, d.y, d.z, d.w};
           const float wj = kWeighted ? meta[s].w[j] : 1.0f;
 #pragma unroll
@@ -256,7 +307,7 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
           }
         }
         if (kBias) {
-          const uint4 b = lds_v4(stage + (uint32_t)L.k * slot_bytes + (uint32_t)e * 2);
+          const uint4 b = lds_v4(stage + (kPacked ? (uint32_t)n * stride : (uint32_t)L.k * slot_bytes) + (uint32_t)e * 2);
           const uint32_t wb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
@@ -264,10 +315,9 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
             acc[2 * v + 1] = __fadd_rn(acc[2 * v + 1], bf16hi(wb[v]));
           }
         }
-        const int64_t t = cta_token(q);
-        if (!dbg_ok(q < n_tok && t < L.T && c0 + e + 8 <= H && n <= L.k &&
-                        g.data + (uint32_t)s * g.stage_bytes + (uint32_t)(n > 0 ? n - 1 : 0) * slot_bytes +
-                                (uint32_t)e * 2 + 16 <= g.total,
+        const int64_t t = cta_token(qi);
+        if (!dbg_ok(qi < n_tok && t < L.T && c0 + e + 8 <= H && n <= L.k &&
+                        (uint32_t)(n > 0 ? n - 1 : 0) * stride + (uint32_t)e * 2 + 16 <= g.stage_bytes,
                     L.status, 103, t * 65536 + e))
           continue;
         uint4 o;
@@ -280,10 +330,12 @@ __global__ void __launch_bounds__(kCombThreads, 1) k_combine(CombineLaunch L, Co
       __syncwarp();
       if (lane == 0) mbar_arrive(empty0 + 8 * s);
       // advance to item i + G
-      c += kCombGroups;
-      while (c >= g.nch) {
-        c -= g.nch;
-        ++q;
+      if constexpr (!kPacked) {
+        c += kCombGroups;
+        while (c >= g.nch) {
+          c -= g.nch;
+          ++q;
+        }
       }
       s += kCombGroups;
       while (s >= S) {
@@ -299,10 +351,12 @@ cudaError_t launch_combine(const CombineLaunch& L, cudaStream_t st) {
   const bool wgt = L.w != nullptr, has_bias = L.bias != nullptr;
   const CombGeom g = combine_geometry(L.H, L.k, has_bias);
   if (g.stages < kCombGroups || g.stages % kCombGroups != 0) return cudaErrorInvalidValue;
-  static unsigned long long done[4] = {0, 0, 0, 0};
-  const int variant = (wgt ? 2 : 0) + (has_bias ? 1 : 0);
-  auto kern = wgt ? (has_bias ? k_combine<true, true> : k_combine<true, false>)
-                  : (has_bias ? k_combine<false, true> : k_combine<false, false>);
+  static unsigned long long done[6] = {0, 0, 0, 0, 0, 0};
+  if (L.packed && wgt) return cudaErrorInvalidValue;  // packed items carry no weights
+  const int variant = L.packed ? 4 + (has_bias ? 1 : 0) : (wgt ? 2 : 0) + (has_bias ? 1 : 0);
+  auto kern = L.packed ? (has_bias ? k_combine<false, true, true> : k_combine<false, false, true>)
+              : wgt    ? (has_bias ? k_combine<true, true, false> : k_combine<true, false, false>)
+                       : (has_bias ? k_combine<false, true, false> : k_combine<false, false, false>);
   cudaError_t err = set_smem_limit_once(kern, (int)kCombSmemBudget, &done[variant]);
   if (err != cudaSuccess) return err;
   err = launch_pdl(kern, dim3(L.grid), dim3(kCombThreads), (size_t)g.total, st, L, g);

@@ -653,6 +653,7 @@ int moe_combine_by_rank(const moe_handle_t* h, const void* y, const void* bias, 
   L.pair_rank = h->d.pair_rank;
   L.slot = h->d.tslot;
   L.status = h->d.status;
+  L.packed = true;  // a token has at most one row per rank: items sized by its rows
   return launch_combine(L, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -157,6 +157,7 @@ struct CombineLaunch {
   const int32_t* pair_rank;
   const int32_t* slot;
   int32_t* status;
+  bool packed;  // items sized by the token's source rows (the by-rank combine), no weights
 };
 
 cudaError_t launch_combine(const CombineLaunch& L, cudaStream_t s);

@@ -80,6 +80,20 @@ def test_by_rank_wide_chunks_under_an_sm_cap():
     _round_trip(wl, num_sms=24)
 
 
+@pytest.mark.parametrize("with_bias", [False, True])
+@pytest.mark.parametrize("kw", [
+    dict(hidden=7168, fp8=True, tokens_per_rank=64, ranks=8, experts=64, topk=8),   # rows of 1..8 ranks
+    dict(hidden=1000, tokens_per_rank=50, ranks=4, experts=16, topk=2),              # H not a chunk multiple
+])
+def test_by_rank_combine_items_sized_by_rows(kw, with_bias):
+    """The by-rank combine takes as many column chunks per item as the token's rows leave room for
+    (one rank: the whole row at once; no rows and no bias: nothing loaded).  90 % of the routing
+    entries masked gives every row count from none to all ranks; every byte against the oracle."""
+    wl = W.WORKLOADS["tiny"].with_(**kw)
+    _round_trip(wl, mask=0.9, with_bias=with_bias)
+    _round_trip(wl.with_(seed=5), mask=0.3, with_bias=with_bias)
+
+
 def test_moe_dispatch_without_expansion():
     wl = W.WORKLOADS["tiny"].with_(hidden=256, tokens_per_rank=64, ranks=4, experts=16, topk=4)
     _round_trip(wl, via_moe_dispatch=True, with_bias=False)
