@@ -13,7 +13,9 @@
 // b, b + G, b + 2G, ..., so the grid reads neighbouring tokens together and the rows it gathers
 // from each expert's range lie close together (3-4 % faster at DeepSeek-V3 prefill than
 // contiguous token ranges per CTA).  A work item is one token and one column chunk of CW
-// elements (CW <= 2048, chosen so that several stages fit):
+// elements (CW <= 2048, chosen so that several stages fit); in the by-rank combine (packed
+// items), a token with n source rows takes (k + bias) / (n + bias) chunks per item, so that its
+// rows fill the stage's k (+ bias) row slots:
 //   warp 0      producer: reads the token's k (rank, slot) pairs from the handle and issues one
 //               cp.async.bulk load per valid source row segment (plus the bias segment) into a
 //               stage of a shared-memory ring, completed on the stage's mbarrier;
