@@ -564,18 +564,19 @@ def measure_workload(moe, wl: W.Workload, args, world: int, rank: int, dev, stre
     ev = {k: [] for k in ("l0", "l1", "d1", "c1")}
     # without host sync the layout and the dispatch are one call (moe_layout_dispatch)
     one_call = not wl.cpu_sync
+    prm = make_params(p_cap)  # made once, as a caller reusing its configuration would
 
     def step_parts(e, st):
         if e is not None:
             e[0].record(st)
         if one_call:
-            h = moe.moe_layout_dispatch(make_params(p_cap), idx, w, x, dtype_out, recv, scales, None,
+            h = moe.moe_layout_dispatch(prm, idx, w, x, dtype_out, recv, scales, None,
                                         do_zero_padding=wl.zero_padding, stream=st)
-            if e is not None:
+            if e is not None and e[1] is not None:
                 e[1].record(st)
         else:
-            h = moe.moe_layout(make_params(p_cap), idx, w, stream=st)
-            if e is not None:
+            h = moe.moe_layout(prm, idx, w, stream=st)
+            if e is not None and e[1] is not None:
                 e[1].record(st)
             moe.moe_dispatch(h, x, dtype_out, recv, scales, None, cap=cap, do_zero_padding=wl.zero_padding,
                              num_sms=wl.num_sms, stream=st)
@@ -587,10 +588,22 @@ def measure_workload(moe, wl: W.Workload, args, world: int, rank: int, dev, stre
             e[3].record(st)
         moe.moe_handle_free(h)
 
-    def step(record: bool):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if record else None
+    tev = {k: [] for k in ("l0", "d1", "c1")}
+
+    def step(record, timed: bool = False):
+        # timed: events at the step's start, after the dispatch and after the combine, none between
+        # the host's count wait and the dispatch launch (one there delays the dispatch)
+        if not record:
+            step_parts(None, stream)
+            return
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        if timed:
+            e[1] = None
         step_parts(e, stream)
-        if record:
+        if timed:
+            for key, val in zip(tev, (e[0], e[2], e[3])):
+                tev[key].append(val)
+        else:
             for key, val in zip(ev, e):
                 ev[key].append(val)
 
@@ -601,6 +614,9 @@ def measure_workload(moe, wl: W.Workload, args, world: int, rank: int, dev, stre
     assert moe.moe_handle_status(hc) == moe.MOE_OK
     moe.moe_handle_free(hc)
 
+    # the K timed steps record the combine's duration (the dominant kernel) and the layout +
+    # dispatch span; the layout / dispatch split comes from a second, instrumented run, because an
+    # event between the host's count wait and the dispatch launch would delay the dispatch
     barrier()
     torch.cuda.synchronize()
     launches0 = moe.moe_kernel_launch_count()
@@ -608,21 +624,30 @@ def measure_workload(moe, wl: W.Workload, args, world: int, rank: int, dev, stre
     w0 = time.time()
     t_start.record(stream)
     for _ in range(steps):
-        step(True)
+        step(True, timed=True)
     t_end.record(stream)
     torch.cuda.synchronize()
     w1 = time.time()
     barrier()
     launches = moe.moe_kernel_launch_count() - launches0
     ms = reduce_max(t_start.elapsed_time(t_end), dev) / steps
+    # the per-kernel breakdown from a second, instrumented run of the same step
+    for _ in range(max(3, min(steps, 50))):
+        step(True)
+    torch.cuda.synchronize()
     layout_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["l0"], ev["l1"]))
     dispatch_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["l1"], ev["d1"]))
-    combine_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["d1"], ev["c1"]))
+    combine_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(tev["d1"], tev["c1"]))  # timed steps
+    front_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(tev["l0"], tev["d1"]))   # layout + dispatch
     value = world * step_bytes / (ms * 1e-3) / 1e9
 
-    kernels_ms = ({"layout_dispatch": layout_ms + dispatch_ms, "combine": combine_ms} if one_call else
+    kernels_ms = ({"layout_dispatch": front_ms, "combine": combine_ms} if one_call else
                   {"layout": layout_ms, "dispatch": dispatch_ms, "combine": combine_ms})
     rec = {"value": value, "ms_per_step": ms, "steps": steps, "warmup": warmup, "cap": cap,
+           "kernel_times": ("combine and layout+dispatch: CUDA events over the timed steps" if one_call else
+                            "combine: CUDA events over the timed steps (layout + dispatch there: "
+                            f"{front_ms:.4f} ms); layout and dispatch apart: an instrumented run of the "
+                            "same step after them"),
            "window": (w0, w1), "launches": launches, "nb": nb, "valid_pairs": valid_pairs, "pad_rows": pad_rows,
            "rows": rows, "kernels_ms": kernels_ms, "one_call": one_call}
     # end to end through the public API: pinned host inputs -> device, round trip, result -> host
@@ -837,7 +862,7 @@ def side_record(wl: W.Workload, rec: dict, clk: ClockSampler) -> dict:
     nb = rec["nb"]
     out = {"value": rec["value"], "unit": UNIT, "us_per_step": rec["ms_per_step"] * 1e3, "steps": rec["steps"],
            "warmup": rec["warmup"], "frac_of_hbm_peak": rec["value"] / rec["peak"],
-           "kernels_us": {key: val * 1e3 for key, val in k.items()},
+           "kernels_us": {key: val * 1e3 for key, val in k.items()}, "kernel_times": rec["kernel_times"],
            "kernels_gbs": {("layout_dispatch" if rec["one_call"] else "dispatch"):
                            nb["dispatch"] / k["layout_dispatch" if rec["one_call"] else "dispatch"] / 1e6,
                            "combine": nb["combine"] / k["combine"] / 1e6},
@@ -891,7 +916,7 @@ def run_ours(args) -> int:
                                           step_bytes=nb["dispatch"] + nb["combine"]),
                 "frac_of_hbm_peak": rec["value"] / world / peak,
                 "frac_of_8tbs_nominal": rec["value"] / world / 8000.0,
-                "kernels_ms": k,
+                "kernels_ms": k, "kernel_times": rec["kernel_times"],
                 "kernels_gbs": {("layout_dispatch" if rec["one_call"] else "dispatch"):
                                 nb["dispatch"] / k["layout_dispatch" if rec["one_call"] else "dispatch"] / 1e6,
                                 "combine": nb["combine"] / k["combine"] / 1e6},
